@@ -1,0 +1,209 @@
+/*
+ * hisa.h — C ABI of the B200 (sm_100a) HISA token-selection indexer.
+ *
+ * Hierarchical indexed sparse attention (HISA) replaces the flat DeepSeek-style
+ * (DSA) indexer of a sparse-attention layer.  The method, as summarised on
+ * aitrends.kr, "HISA: 세밀한 희소 어텐션을 위한 효율적인 계층적 인덱싱":
+ *   - block partition and mean pooling: the index keys of a sequence form
+ *     contiguous blocks of B tokens; each block is represented by the mean of
+ *     its keys (paragraph on block partition and pooling);
+ *   - stage 1: each query scores every block representative with a dot
+ *     product, blocks wholly after the query are masked, the first block and
+ *     the last two blocks are always kept, and the top-m blocks survive
+ *     (paragraph on stage 1);
+ *   - stage 2: only the tokens of the surviving blocks are scored with the
+ *     original DSA dot product and the top-k token indices are emitted in the
+ *     layout the sparse attention operator consumes (paragraph on stage 2, and
+ *     the paragraph on keeping the DSA output structure);
+ *   - the representatives can be maintained as keys are appended to the KV
+ *     cache (paragraph on KV-cache maintenance).
+ * The flat DSA scan (idea.jsleekr.com, "긴 컨텍스트 LLM이 느려지는 이유와 희소
+ * 어텐션(sparse attention)으로 해결하는 방법", section "DSA: 딥시크의 희소 어텐션")
+ * scores every earlier key and keeps the top-k; it is provided for comparison
+ * and as the m = M identity (HISA with every block selected is the flat scan).
+ *
+ * Readings of points the pages leave open (fixed by this library):
+ *   - "last two blocks" are the query's own block and the block before it; the
+ *     forced blocks count inside m; when at most m blocks are eligible all of
+ *     them are selected; with m < 3 forced blocks are kept in the order own,
+ *     previous, first;
+ *   - the token score is the single-head dot product q.k over d = 64 index
+ *     dimensions, accumulated in fp32;
+ *   - every output row is ordered by score descending; equal scores go to the
+ *     lower index (stage 1: lower block, stage 2: lower token); rows with fewer
+ *     than k candidates are padded with -1; -0.0 and +0.0 compare equal;
+ *   - indices are positions local to their sequence.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *   - Every array argument is a caller-owned DEVICE pointer; the library never
+ *     allocates, frees or keeps a pointer after the call returns.  Scratch comes
+ *     from a caller workspace sized by the matching *_workspace_size function.
+ *   - Calls are asynchronous on the caller's stream (a cudaStream_t passed as
+ *     void*; NULL = the legacy default stream) and never synchronise the host.
+ *   - Every call returns a hisa_status; nothing throws across the ABI.
+ *     Argument errors visible on the host are returned directly and nothing is
+ *     launched.  Errors that only the device can see (a region start that is
+ *     not a multiple of B, lengths that do not fit their region, an append past
+ *     the region's capacity, a wait that timed out) are OR-ed into a sticky
+ *     per-device status word, read with hisa_device_status(); the rows or
+ *     sequences concerned are skipped (their output rows are filled with -1).
+ *   - bf16 values are passed as their 16-bit patterns (hisa_bf16).
+ *   - Row-major layouts; q/k rows are d = 64 bf16 (128 bytes); every pointer
+ *     must be 16-byte aligned (HISA_ERR_UNALIGNED otherwise).
+ *   - The GPU path is built for d = HISA_INDEX_DIM (64) and B = HISA_BLOCK (128);
+ *     any other B is rejected with HISA_ERR_INVALID_ARG.
+ *
+ * Sequence layout (prefill, decode and packed varlen alike)
+ * ----------------------------------------------------------
+ *   cu_seqlens_k  int32 [num_seqs+1]: sequence s owns key rows
+ *                 [cu_seqlens_k[s], cu_seqlens_k[s+1]) of k_idx (its "region");
+ *                 region starts must be multiples of B, so blocks never cross
+ *                 sequences and the representative of the block holding key row
+ *                 r is row r / B of reps.
+ *   seqlens_k     int32 [num_seqs] or NULL: live key count of each sequence;
+ *                 NULL means the whole region is live.
+ *   cu_seqlens_q  int32 [num_seqs+1]: sequence s owns query rows
+ *                 [cu_seqlens_q[s], cu_seqlens_q[s+1]) of q_idx; they are the
+ *                 LAST q_len_s positions of the sequence (query r sits at
+ *                 position len_s - q_len_s + r).  Prefill: q_len = len; decode:
+ *                 q_len = 1.
+ *   total_q       = cu_seqlens_q[num_seqs] (host copy, sizes the grids).
+ *   max_seqlen_k  >= every live length (host copy, sizes the grids).
+ */
+#ifndef HISA_H_
+#define HISA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define HISA_INDEX_DIM 64
+#define HISA_BLOCK 128
+#define HISA_MAX_M 128      /* m * B candidates are held on chip per query */
+#define HISA_MAX_TOPK 2048  /* largest k accepted by hisa_select / dsa_flat_select */
+
+typedef uint16_t hisa_bf16;  /* bf16 bit pattern */
+typedef void *hisa_stream_t; /* cudaStream_t */
+
+typedef enum {
+  HISA_OK = 0,
+  HISA_ERR_INVALID_ARG = 1,    /* bad size, count, B, m or k; inconsistent lengths */
+  HISA_ERR_UNALIGNED = 2,      /* pointer not 16-byte aligned, region start not a multiple of B */
+  HISA_ERR_WORKSPACE = 3,      /* workspace missing or smaller than *_workspace_size() */
+  HISA_ERR_CUDA = 4,           /* a CUDA runtime call failed (launch, attribute, copy) */
+  HISA_ERR_TIMEOUT = 5,        /* a bounded device-side wait gave up */
+  HISA_ERR_NOT_IMPLEMENTED = 6,
+  HISA_ERR_CAPACITY = 7        /* hisa_append_keys would write past a region's end */
+} hisa_status;
+
+/* Text for a status code (static storage; never NULL). */
+const char *hisa_status_string(hisa_status s);
+
+/* Library version (major*10000 + minor*100 + patch). */
+int hisa_version(void);
+
+/*
+ * hisa_pool_blocks — mean-pool the index keys of every sequence into one
+ * representative per block of B tokens (HISA summary page, paragraph on block
+ * partition and mean pooling).
+ *
+ *   k_idx         bf16 [rows_k, 64]; rows_k = cu_seqlens_k[num_seqs].
+ *   reps (out)    fp32 [ceil(rows_k / B), 64]; row r/B receives the mean of the
+ *                 live keys of the block containing key row r.  A partial last
+ *                 block (len not a multiple of B) is divided by the number of
+ *                 keys present.  Rows of blocks with no live key are untouched.
+ * The sum runs over the block's keys in increasing row order in fp32 and is then
+ * divided (round to nearest) by the count; hisa_append_keys uses the same order,
+ * so representatives maintained incrementally are bit-identical to a re-pool.
+ */
+hisa_status hisa_pool_blocks(const hisa_bf16 *k_idx, const int32_t *cu_seqlens_k,
+                             const int32_t *seqlens_k, int num_seqs, int max_seqlen_k, int B,
+                             float *reps, hisa_stream_t stream);
+
+/*
+ * hisa_append_keys — decode-time KV-cache update (HISA summary page, paragraph
+ * on maintaining representatives at KV-cache update time).
+ *
+ *   k_cache (in/out)   bf16 [rows_k, 64]; new rows are written at region row
+ *                      seqlens_k[s] .. seqlens_k[s] + n_new - 1 of sequence s.
+ *   reps (in/out)      fp32 [rows_k / B, 64]; every block touched by the new keys
+ *                      is re-pooled (same order and rounding as hisa_pool_blocks).
+ *   cu_seqlens_k       int32 [num_seqs+1] region starts; a region's size is its
+ *                      capacity.
+ *   seqlens_k (in/out) int32 [num_seqs] live lengths, incremented by n_new on the
+ *                      device.
+ *   new_keys           bf16 [num_seqs, n_new, 64].
+ * A sequence whose region cannot take n_new more keys is left unchanged and
+ * HISA_ERR_CAPACITY is raised in the device status word.
+ */
+hisa_status hisa_append_keys(hisa_bf16 *k_cache, float *reps, const int32_t *cu_seqlens_k,
+                             int32_t *seqlens_k, const hisa_bf16 *new_keys, int n_new,
+                             int num_seqs, int B, hisa_stream_t stream);
+
+/*
+ * hisa_select — the HISA indexer: stage 1 (block scores and top-m) followed by
+ * stage 2 (scores of the tokens of the selected blocks and top-k).
+ *
+ *   q_idx          bf16 [total_q, 64] index queries.
+ *   k_idx          bf16 [rows_k, 64] index keys (the same buffer that was pooled).
+ *   reps           fp32 [rows_k / B, 64] block representatives (hisa_pool_blocks /
+ *                  hisa_append_keys).
+ *   m              blocks kept per query, 1 <= m <= HISA_MAX_M.  Blocks 0, the own
+ *                  block and the previous block are forced and count inside m;
+ *                  if the query sees at most m blocks, all are kept.
+ *   k              tokens kept per query, 1 <= k <= HISA_MAX_TOPK.  m*B < k is
+ *                  accepted (rows are then padded with -1).
+ *   out_idx (out)  int32 [total_q, k]: sequence-local token positions j <= i of
+ *                  the selected tokens, by score descending (ties: lower j), -1
+ *                  padded.
+ *   out_scores     fp32 [total_q, k] or NULL: the scores of out_idx (0 where -1).
+ *   out_blocks     int32 [total_q, m] or NULL: the selected blocks (sequence-local
+ *                  block numbers), ascending, -1 padded.
+ *   ws, ws_bytes   device workspace of at least hisa_select_workspace_size(...)
+ *                  bytes, 256-byte aligned; it must not be used by another call
+ *                  that runs at the same time.
+ */
+hisa_status hisa_select(const hisa_bf16 *q_idx, const hisa_bf16 *k_idx, const float *reps,
+                        const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
+                        const int32_t *seqlens_k, int num_seqs, int total_q, int max_seqlen_k,
+                        int B, int m, int k, int32_t *out_idx, float *out_scores,
+                        int32_t *out_blocks, void *ws, size_t ws_bytes, hisa_stream_t stream);
+
+size_t hisa_select_workspace_size(int total_q, int num_seqs, int max_seqlen_k, int B, int m,
+                                  int k);
+
+/*
+ * dsa_flat_select — the flat DSA indexer: every causal key j <= i of the query's
+ * sequence is scored with q.k and the top-k are emitted with the same ordering,
+ * padding and layout as hisa_select (idea.jsleekr.com, section "DSA: 딥시크의
+ * 희소 어텐션").  Token scores are computed with the same fp32 arithmetic as
+ * hisa_select's stage 2, so hisa_select with m >= the number of blocks returns
+ * exactly the rows of this function.
+ *
+ *   ws, ws_bytes   device workspace of at least dsa_flat_workspace_size(...) bytes.
+ */
+hisa_status dsa_flat_select(const hisa_bf16 *q_idx, const hisa_bf16 *k_idx,
+                            const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
+                            const int32_t *seqlens_k, int num_seqs, int total_q,
+                            int max_seqlen_k, int k, int32_t *out_idx, float *out_scores,
+                            void *ws, size_t ws_bytes, hisa_stream_t stream);
+
+size_t dsa_flat_workspace_size(int total_q, int num_seqs, int max_seqlen_k, int k);
+
+/*
+ * hisa_device_status — wait for `stream`, then copy the sticky device status word
+ * of the current device into *status (0 = no device-side error; otherwise the
+ * OR of (1 << hisa_status) bits).  clear != 0 resets the word afterwards.
+ * Meant for tests and debugging: it synchronises the stream.
+ */
+hisa_status hisa_device_status(int32_t *status, int clear, hisa_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HISA_H_ */

@@ -1,0 +1,24 @@
+"""B200-native (sm_100a) HISA token-selection indexer.
+
+The work happens in ``libhisa.so`` (hand-written CUDA kernels behind the C ABI
+of ``include/hisa.h``); this package is its thin Python binding.  PyTorch only
+provides device memory and streams.
+"""
+
+from .binding import (  # noqa: F401
+    EXPORTED,
+    HISA_BLOCK,
+    HISA_INDEX_DIM,
+    HISA_MAX_M,
+    HISA_MAX_TOPK,
+    HisaError,
+    LIB_PATH,
+    dsa_flat_select,
+    dsa_flat_workspace_size,
+    hisa_append_keys,
+    hisa_device_status,
+    hisa_pool_blocks,
+    hisa_select,
+    hisa_select_workspace_size,
+    lib,
+)

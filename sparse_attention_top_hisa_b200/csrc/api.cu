@@ -1,0 +1,230 @@
+// C ABI of the HISA indexer library: argument validation, workspace carving and
+// kernel launches.  Declarations and the contract of every entry point are in
+// include/hisa.h.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace hisa {
+cudaError_t launch_pool(const uint16_t *k, const int32_t *cu_k, const int32_t *seqlens,
+                        int num_seqs, int max_seqlen_k, float *reps, int *status,
+                        cudaStream_t st);
+cudaError_t launch_append(uint16_t *kc, float *reps, const int32_t *cu_k, int32_t *seqlens,
+                          const uint16_t *new_keys, int n_new, int num_seqs, int *status,
+                          cudaStream_t st);
+cudaError_t launch_block_select(const uint16_t *q, const float *reps, const int32_t *cu_q,
+                                const int32_t *cu_k, const int32_t *seqlens, int S,
+                                int total_q, int max_seqlen_k, int m, int32_t *blk,
+                                int32_t *out_blocks, int *status, cudaStream_t st);
+cudaError_t launch_token_select(const uint16_t *q, const uint16_t *k, const int32_t *cu_q,
+                                const int32_t *cu_k, const int32_t *seqlens, int S, int total_q,
+                                int m, int topk, const int32_t *blk, uint32_t *scratch,
+                                int num_sms, int32_t *out_idx, float *out_scores, int *status,
+                                cudaStream_t st);
+size_t token_scratch_bytes(int total_q, int m, int num_sms);
+cudaError_t launch_dsa(const uint16_t *q, const uint16_t *k, const int32_t *cu_q,
+                       const int32_t *cu_k, const int32_t *seqlens, int S, int total_q,
+                       int max_seqlen_k, int topk, int32_t *out_idx, float *out_scores,
+                       uint8_t *ws, int *status, cudaStream_t st);
+size_t dsa_workspace_bytes(int total_q, int num_seqs, int max_seqlen_k, int topk);
+}  // namespace hisa
+
+using namespace hisa;
+
+// Sticky device status word (one per device that loads the library).
+static __device__ int g_hisa_status;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+int *g_status_ptr[kMaxDevices];
+int g_num_sms[kMaxDevices];
+
+int current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return -1;
+  return dev;
+}
+
+// Device address of the status word on the current device (set up once per device).
+int *status_word() {
+  const int dev = current_device();
+  if (dev < 0) return nullptr;
+  if (!g_status_ptr[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_hisa_status) != cudaSuccess) return nullptr;
+    g_status_ptr[dev] = static_cast<int *>(p);
+  }
+  return g_status_ptr[dev];
+}
+
+int num_sms() {
+  const int dev = current_device();
+  if (dev < 0) return 148;
+  if (!g_num_sms[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    g_num_sms[dev] = n;
+  }
+  return g_num_sms[dev];
+}
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+hisa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? HISA_OK : HISA_ERR_CUDA; }
+
+struct SelectPlan {
+  size_t off_blk, off_scratch, total;
+};
+
+SelectPlan select_plan(int total_q, int m) {
+  SelectPlan p;
+  size_t off = 0;
+  p.off_blk = off;
+  off = align256(off + (size_t)(total_q > 0 ? total_q : 1) * m * 4);
+  p.off_scratch = off;
+  off = align256(off + token_scratch_bytes(total_q, m, num_sms()));
+  p.total = off;
+  return p;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *hisa_status_string(hisa_status s) {
+  switch (s) {
+    case HISA_OK: return "ok";
+    case HISA_ERR_INVALID_ARG: return "invalid argument";
+    case HISA_ERR_UNALIGNED: return "unaligned pointer or region start";
+    case HISA_ERR_WORKSPACE: return "workspace missing or too small";
+    case HISA_ERR_CUDA: return "CUDA runtime error";
+    case HISA_ERR_TIMEOUT: return "device-side wait timed out";
+    case HISA_ERR_NOT_IMPLEMENTED: return "not implemented";
+    case HISA_ERR_CAPACITY: return "key region capacity exceeded";
+  }
+  return "unknown status";
+}
+
+int hisa_version(void) { return 100; }
+
+hisa_status hisa_pool_blocks(const hisa_bf16 *k_idx, const int32_t *cu_seqlens_k,
+                             const int32_t *seqlens_k, int num_seqs, int max_seqlen_k, int B,
+                             float *reps, hisa_stream_t stream) {
+  if (B != HISA_BLOCK || num_seqs < 0 || max_seqlen_k < 0) return HISA_ERR_INVALID_ARG;
+  if (num_seqs == 0 || max_seqlen_k == 0) return HISA_OK;
+  if (!k_idx || !cu_seqlens_k || !reps) return HISA_ERR_INVALID_ARG;
+  if (!aligned(k_idx, 16) || !aligned(reps, 16) || !aligned(cu_seqlens_k, 4) ||
+      !aligned(seqlens_k, 4))
+    return HISA_ERR_UNALIGNED;
+  int *st = status_word();
+  if (!st) return HISA_ERR_CUDA;
+  return from_cuda(launch_pool(k_idx, cu_seqlens_k, seqlens_k, num_seqs, max_seqlen_k, reps, st,
+                               static_cast<cudaStream_t>(stream)));
+}
+
+hisa_status hisa_append_keys(hisa_bf16 *k_cache, float *reps, const int32_t *cu_seqlens_k,
+                             int32_t *seqlens_k, const hisa_bf16 *new_keys, int n_new,
+                             int num_seqs, int B, hisa_stream_t stream) {
+  if (B != HISA_BLOCK || num_seqs < 0 || n_new < 0) return HISA_ERR_INVALID_ARG;
+  if (num_seqs == 0 || n_new == 0) return HISA_OK;
+  if (!k_cache || !reps || !cu_seqlens_k || !seqlens_k || !new_keys) return HISA_ERR_INVALID_ARG;
+  if (!aligned(k_cache, 16) || !aligned(reps, 16) || !aligned(new_keys, 16) ||
+      !aligned(cu_seqlens_k, 4) || !aligned(seqlens_k, 4))
+    return HISA_ERR_UNALIGNED;
+  int *st = status_word();
+  if (!st) return HISA_ERR_CUDA;
+  return from_cuda(launch_append(k_cache, reps, cu_seqlens_k, seqlens_k, new_keys, n_new,
+                                 num_seqs, st, static_cast<cudaStream_t>(stream)));
+}
+
+size_t hisa_select_workspace_size(int total_q, int num_seqs, int max_seqlen_k, int B, int m,
+                                  int k) {
+  (void)num_seqs;
+  (void)max_seqlen_k;
+  (void)B;
+  (void)k;
+  if (total_q < 0 || m < 1) return 0;
+  return select_plan(total_q, m).total;
+}
+
+hisa_status hisa_select(const hisa_bf16 *q_idx, const hisa_bf16 *k_idx, const float *reps,
+                        const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
+                        const int32_t *seqlens_k, int num_seqs, int total_q, int max_seqlen_k,
+                        int B, int m, int k, int32_t *out_idx, float *out_scores,
+                        int32_t *out_blocks, void *ws, size_t ws_bytes, hisa_stream_t stream) {
+  if (B != HISA_BLOCK || m < 1 || m > HISA_MAX_M || k < 1 || k > HISA_MAX_TOPK)
+    return HISA_ERR_INVALID_ARG;
+  if (num_seqs < 0 || total_q < 0 || max_seqlen_k < 0) return HISA_ERR_INVALID_ARG;
+  if (total_q == 0) return HISA_OK;
+  if (num_seqs == 0) return HISA_ERR_INVALID_ARG;
+  if (!q_idx || !k_idx || !reps || !cu_seqlens_q || !cu_seqlens_k || !out_idx)
+    return HISA_ERR_INVALID_ARG;
+  if (!aligned(q_idx, 16) || !aligned(k_idx, 16) || !aligned(reps, 16) ||
+      !aligned(cu_seqlens_q, 4) || !aligned(cu_seqlens_k, 4) || !aligned(seqlens_k, 4) ||
+      !aligned(out_idx, 4) || !aligned(out_scores, 4) || !aligned(out_blocks, 4))
+    return HISA_ERR_UNALIGNED;
+  const SelectPlan p = select_plan(total_q, m);
+  if (!ws || ws_bytes < p.total) return HISA_ERR_WORKSPACE;
+  if (!aligned(ws, 256)) return HISA_ERR_UNALIGNED;
+  int *st = status_word();
+  if (!st) return HISA_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t *w = static_cast<uint8_t *>(ws);
+  int32_t *blk = reinterpret_cast<int32_t *>(w + p.off_blk);
+  uint32_t *scratch = reinterpret_cast<uint32_t *>(w + p.off_scratch);
+  cudaError_t e = launch_block_select(q_idx, reps, cu_seqlens_q, cu_seqlens_k, seqlens_k,
+                                      num_seqs, total_q, max_seqlen_k, m, blk, out_blocks, st, s);
+  if (e != cudaSuccess) return HISA_ERR_CUDA;
+  e = launch_token_select(q_idx, k_idx, cu_seqlens_q, cu_seqlens_k, seqlens_k, num_seqs, total_q,
+                          m, k, blk, scratch, num_sms(), out_idx, out_scores, st, s);
+  return from_cuda(e);
+}
+
+size_t dsa_flat_workspace_size(int total_q, int num_seqs, int max_seqlen_k, int k) {
+  if (total_q < 0 || num_seqs < 0 || max_seqlen_k < 0 || k < 1) return 0;
+  return dsa_workspace_bytes(total_q, num_seqs, max_seqlen_k, k);
+}
+
+hisa_status dsa_flat_select(const hisa_bf16 *q_idx, const hisa_bf16 *k_idx,
+                            const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
+                            const int32_t *seqlens_k, int num_seqs, int total_q,
+                            int max_seqlen_k, int k, int32_t *out_idx, float *out_scores,
+                            void *ws, size_t ws_bytes, hisa_stream_t stream) {
+  if (k < 1 || k > HISA_MAX_TOPK || num_seqs < 0 || total_q < 0 || max_seqlen_k < 0)
+    return HISA_ERR_INVALID_ARG;
+  if (total_q == 0) return HISA_OK;
+  if (num_seqs == 0) return HISA_ERR_INVALID_ARG;
+  if (!q_idx || !k_idx || !cu_seqlens_q || !cu_seqlens_k || !out_idx) return HISA_ERR_INVALID_ARG;
+  if (!aligned(q_idx, 16) || !aligned(k_idx, 16) || !aligned(cu_seqlens_q, 4) ||
+      !aligned(cu_seqlens_k, 4) || !aligned(seqlens_k, 4) || !aligned(out_idx, 4) ||
+      !aligned(out_scores, 4))
+    return HISA_ERR_UNALIGNED;
+  const size_t need = dsa_workspace_bytes(total_q, num_seqs, max_seqlen_k, k);
+  if (!ws || ws_bytes < need) return HISA_ERR_WORKSPACE;
+  if (!aligned(ws, 256)) return HISA_ERR_UNALIGNED;
+  int *st = status_word();
+  if (!st) return HISA_ERR_CUDA;
+  return from_cuda(launch_dsa(q_idx, k_idx, cu_seqlens_q, cu_seqlens_k, seqlens_k, num_seqs,
+                              total_q, max_seqlen_k, k, out_idx, out_scores,
+                              static_cast<uint8_t *>(ws), st, static_cast<cudaStream_t>(stream)));
+}
+
+hisa_status hisa_device_status(int32_t *status, int clear, hisa_stream_t stream) {
+  if (!status) return HISA_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return HISA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_hisa_status, sizeof(int)) != cudaSuccess) return HISA_ERR_CUDA;
+  *status = v;
+  if (clear) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_hisa_status, &zero, sizeof(int)) != cudaSuccess) return HISA_ERR_CUDA;
+  }
+  return HISA_OK;
+}
+
+}  // extern "C"

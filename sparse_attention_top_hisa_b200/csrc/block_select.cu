@@ -1,0 +1,151 @@
+// Stage 1 of HISA: block scores and top-m block selection (CUDA-core path).
+//
+// HISA summary page (aitrends.kr), paragraph on stage 1: the query is scored
+// against every block representative with a dot product, blocks lying wholly
+// after the query are masked, the first block and the last two blocks (read as
+// the query's own block and the one before it) are always kept, and the top-m
+// blocks survive.  The forced blocks count inside m; a query that sees at most
+// m blocks keeps all of them; ties between block scores go to the lower block.
+//
+// One warp per query.  The scores of the eligible, non-forced blocks are
+// turned into order-preserving keys in shared memory; a 32-step bitwise search
+// finds the key of the (m - |forced|)-th best block; ballots over ascending
+// block numbers resolve ties and emit the selected blocks in ascending order.
+#include "common.cuh"
+
+namespace hisa {
+
+constexpr int BS_WARPS = 4;
+
+__device__ __forceinline__ float rep_score(const QRegs &q, const float *rep) {
+  const float4 *p = reinterpret_cast<const float4 *>(rep);
+  float a = 0.f, b = 0.f;
+#pragma unroll
+  for (int c = 0; c < 8; c++) {
+    float4 x = __ldg(p + c);
+    float4 y = __ldg(p + c + 8);
+    a = fmaf(q.v[4 * c + 0], x.x, a);
+    a = fmaf(q.v[4 * c + 1], x.y, a);
+    a = fmaf(q.v[4 * c + 2], x.z, a);
+    a = fmaf(q.v[4 * c + 3], x.w, a);
+    b = fmaf(q.v[32 + 4 * c + 0], y.x, b);
+    b = fmaf(q.v[32 + 4 * c + 1], y.y, b);
+    b = fmaf(q.v[32 + 4 * c + 2], y.z, b);
+    b = fmaf(q.v[32 + 4 * c + 3], y.w, b);
+  }
+  return a + b;
+}
+
+__global__ void __launch_bounds__(BS_WARPS * 32)
+block_select_kernel(const uint16_t *__restrict__ q, const float *__restrict__ reps,
+                    const int32_t *__restrict__ cu_q, const int32_t *__restrict__ cu_k,
+                    const int32_t *__restrict__ seqlens, int S, int total_q, int m, int emax,
+                    int32_t *__restrict__ blk, int32_t *__restrict__ out_blocks,
+                    int *status) {
+  extern __shared__ uint32_t bs_smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.x * BS_WARPS + warp;
+  if (row >= total_q) return;
+  uint32_t *keys = bs_smem + (size_t)warp * emax;
+  int32_t *dst = blk + (size_t)row * m;
+  int32_t *dst2 = out_blocks ? out_blocks + (size_t)row * m : nullptr;
+
+  const QueryInfo qi = locate(cu_q, cu_k, seqlens, S, row, status);
+  if (!qi.ok) {
+    for (int i = lane; i < m; i += 32) {
+      dst[i] = -1;
+      if (dst2) dst2[i] = -1;
+    }
+    return;
+  }
+  const int own = qi.pos / BLK, E = own + 1;
+  if (E > emax) {  // max_seqlen_k understated by the caller
+    if (lane == 0) raise_status(status, HISA_ERR_INVALID_ARG);
+    for (int i = lane; i < m; i += 32) {
+      dst[i] = -1;
+      if (dst2) dst2[i] = -1;
+    }
+    return;
+  }
+  if (E <= m) {  // every eligible block is kept
+    for (int i = lane; i < m; i += 32) {
+      int v = i < E ? i : -1;
+      dst[i] = v;
+      if (dst2) dst2[i] = v;
+    }
+    return;
+  }
+  const int nf = min(m, 3);  // forced: own, previous, first (E > m >= 3 makes them distinct)
+  const int mfree = m - nf;
+  auto forced = [&](int b) {
+    return b == own || (nf >= 2 && b == own - 1) || (nf >= 3 && b == 0);
+  };
+
+  QRegs qr;
+  load_q(qr, q + (size_t)row * D);
+  const float *rbase = reps + (size_t)(qi.kbase / BLK) * D;
+  for (int b = lane; b < E; b += 32)
+    keys[b] = forced(b) ? 0u : score_key(rep_score(qr, rbase + (size_t)b * D));
+  __syncwarp();
+
+  // T = key of the mfree-th best free block (0 if none are needed)
+  uint32_t T = 0u;
+  if (mfree > 0) {
+    for (int bit = 31; bit >= 0; bit--) {
+      const uint32_t cand = T | (1u << bit);
+      int cnt = 0;
+      for (int b = lane; b < E; b += 32) cnt += keys[b] >= cand;
+      cnt = __reduce_add_sync(0xffffffffu, cnt);
+      if (cnt >= mfree) T = cand;
+    }
+  }
+  int ngt = 0;
+  if (mfree > 0) {
+    for (int b = lane; b < E; b += 32) ngt += keys[b] > T;
+    ngt = __reduce_add_sync(0xffffffffu, ngt);
+  }
+  const int need_eq = mfree - ngt;
+  const unsigned lt = (1u << lane) - 1u;
+  int eqr = 0, outp = 0;
+  for (int b0 = 0; b0 < E; b0 += 32) {
+    const int b = b0 + lane;
+    const uint32_t u = b < E ? keys[b] : 0u;
+    const bool is_eq = mfree > 0 && u != 0u && u == T;
+    const unsigned beq = __ballot_sync(0xffffffffu, is_eq);
+    const bool sel = (b < E && forced(b)) || (mfree > 0 && u > T) ||
+                     (is_eq && eqr + __popc(beq & lt) < need_eq);
+    const unsigned bsel = __ballot_sync(0xffffffffu, sel);
+    if (sel) {
+      const int p = outp + __popc(bsel & lt);
+      dst[p] = b;
+      if (dst2) dst2[p] = b;
+    }
+    eqr += __popc(beq);
+    outp += __popc(bsel);
+  }
+  for (int i = outp + lane; i < m; i += 32) {  // only reachable if fewer than m exist
+    dst[i] = -1;
+    if (dst2) dst2[i] = -1;
+  }
+}
+
+cudaError_t launch_block_select(const uint16_t *q, const float *reps, const int32_t *cu_q,
+                                const int32_t *cu_k, const int32_t *seqlens, int S,
+                                int total_q, int max_seqlen_k, int m, int32_t *blk,
+                                int32_t *out_blocks, int *status, cudaStream_t st) {
+  if (total_q == 0) return cudaSuccess;
+  const int emax = (max_seqlen_k + BLK - 1) / BLK;
+  const size_t smem = (size_t)BS_WARPS * (emax > 0 ? emax : 1) * sizeof(uint32_t);
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(block_select_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  dim3 grid((total_q + BS_WARPS - 1) / BS_WARPS);
+  block_select_kernel<<<grid, BS_WARPS * 32, smem, st>>>(q, reps, cu_q, cu_k, seqlens, S, total_q,
+                                                       m, emax > 0 ? emax : 1, blk, out_blocks,
+                                                       status);
+  return cudaGetLastError();
+}
+
+}  // namespace hisa

@@ -1,0 +1,358 @@
+// Flat DSA indexer (dsa_flat_select): exact top-k over every causal key.
+//
+// idea.jsleekr.com, section "DSA: 딥시크의 희소 어텐션": each query scores every
+// earlier key with a light dot product and keeps the best few.  Ordering, tie
+// rule and output layout are the ones of hisa_select, and token scores use the
+// same fp32 evaluation, so HISA with every block selected reproduces these rows.
+//
+// Schedule (the score matrix is never materialised):
+//   1. key_norm_kernel: per sequence the largest key norm |k|max, so that every
+//      score of query q lies in [-R, R] with R = |q| |k|max (Cauchy-Schwarz).
+//   2. dsa_filter_kernel: one thread per query, 128 queries per CTA share key
+//      tiles staged in shared memory.  Pass 1 histograms the scores into 128
+//      linear buckets over [-R, R] (bucket 0 = highest); the bucket holding the
+//      k-th best score is b*.  Pass 2 recomputes the scores and appends every
+//      candidate in buckets <= b* (a superset of the top-k, in token order) to
+//      the query's candidate list.  Bucketing is monotone in the score, so the
+//      superset property holds exactly whatever the rounding.
+//   3. dsa_select_kernel: exact top-k of each candidate list (shared routine).
+//   4. dsa_fallback_kernel: a row whose list overflowed its capacity (many equal
+//      scores) is redone exactly from a full score row in scratch memory.
+#include "select.cuh"
+
+namespace hisa {
+
+constexpr int DSA_Q = 128;   // queries per filter CTA
+constexpr int DSA_NB = 128;  // score buckets
+constexpr int DSA_KT = 64;   // keys per staged tile
+constexpr int DSA_SEL_THREADS = 256;
+constexpr int DSA_FB_CTAS = 16;
+
+__global__ void __launch_bounds__(256)
+key_norm_kernel(const uint16_t *__restrict__ k, const int32_t *__restrict__ cu_k,
+                const int32_t *__restrict__ seqlens, float *__restrict__ kmax) {
+  const int s = blockIdx.y;
+  const int j = blockIdx.x * blockDim.x + threadIdx.x;
+  const int start = cu_k[s], cap = cu_k[s + 1] - start;
+  const int len = seqlens ? seqlens[s] : cap;
+  if (start % BLK != 0 || len < 0 || len > cap) return;  // reported by the filter
+  float nrm = 0.f;
+  if (j < len) {
+    const uint4 *p = reinterpret_cast<const uint4 *>(k + (size_t)(start + j) * D);
+    float acc = 0.f;
+#pragma unroll
+    for (int c = 0; c < 8; c++) {
+      uint4 w = __ldg(p + c);
+      uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int u = 0; u < 4; u++) {
+        float a = bf_lo(ws[u]), b = bf_hi(ws[u]);
+        acc = fmaf(a, a, acc);
+        acc = fmaf(b, b, acc);
+      }
+    }
+    nrm = sqrtf(acc);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) nrm = fmaxf(nrm, __shfl_xor_sync(0xffffffffu, nrm, o));
+  if ((threadIdx.x & 31) == 0 && nrm > 0.f) atomicMax(reinterpret_cast<int *>(kmax + s), __float_as_int(nrm));
+}
+
+__device__ __forceinline__ int score_bucket(float s, float R, float inv) {
+  int b = __float2int_rz((R - s) * inv);
+  return min(max(b, 0), DSA_NB - 1);
+}
+
+struct DsaShared {
+  uint32_t hist[DSA_Q * (DSA_NB + 1)];
+  uint4 tile[DSA_KT * 8];
+  int jmax;
+  int srange[2];
+};
+
+__global__ void __launch_bounds__(DSA_Q)
+dsa_filter_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ k,
+                  const int32_t *__restrict__ cu_q, const int32_t *__restrict__ cu_k,
+                  const int32_t *__restrict__ seqlens, int S, int row0, int nrows, int topk,
+                  int cap, const float *__restrict__ kmax, uint32_t *__restrict__ buf_key,
+                  int32_t *__restrict__ buf_j, int32_t *__restrict__ cnt_out, int *status) {
+  extern __shared__ __align__(16) uint8_t dsa_smem[];
+  DsaShared &sh = *reinterpret_cast<DsaShared *>(dsa_smem);
+  const int tid = threadIdx.x;
+  const int local = blockIdx.x * DSA_Q + tid;  // row within the chunk
+  const int row = row0 + local;
+  const bool in_range = local < nrows;
+  QueryInfo qi;
+  qi.ok = false;
+  qi.seq = -1;
+  if (in_range) qi = locate(cu_q, cu_k, seqlens, S, row, status);
+  uint32_t *hist = sh.hist + tid * (DSA_NB + 1);
+  int count = 0;
+
+  QRegs qr;
+  float R = 0.f, inv = 0.f;
+  if (in_range && qi.ok) {
+    load_q(qr, q + (size_t)row * D);
+    float qq = 0.f;
+#pragma unroll
+    for (int c = 0; c < D; c++) qq = fmaf(qr.v[c], qr.v[c], qq);
+    R = sqrtf(qq) * kmax[qi.seq] * (1.0f + 1.0f / 1024.0f);
+    inv = R > 0.f ? (float)DSA_NB / (2.0f * R) : 0.f;
+  }
+  if (tid == 0) {
+    sh.srange[0] = in_range ? find_seq(cu_q, S, row) : 0;
+    int last = min(row0 + nrows, row0 + (int)(blockIdx.x + 1) * DSA_Q) - 1;
+    sh.srange[1] = find_seq(cu_q, S, last);
+  }
+  __syncthreads();
+  const int s_lo = sh.srange[0], s_hi = sh.srange[1];
+
+  for (int s = s_lo; s <= s_hi; s++) {
+    const bool active = in_range && qi.ok && qi.seq == s;
+    if (tid == 0) sh.jmax = -1;
+    __syncthreads();
+    if (active) atomicMax(&sh.jmax, qi.pos);
+    __syncthreads();
+    const int jmax = sh.jmax;
+    if (jmax < 0) continue;  // block-uniform
+    const uint4 *kseq = reinterpret_cast<const uint4 *>(k + (size_t)__ldg(cu_k + s) * D);
+
+    // pass 1: histogram
+    if (active)
+      for (int b = 0; b <= DSA_NB; b++) hist[b] = 0u;
+    for (int j0 = 0; j0 <= jmax; j0 += DSA_KT) {
+      const int nk = min(DSA_KT, jmax + 1 - j0);
+      __syncthreads();
+      for (int i = tid; i < nk * 8; i += DSA_Q) sh.tile[i] = __ldg(kseq + (size_t)j0 * 8 + i);
+      __syncthreads();
+      if (active) {
+        const int jend = min(nk, qi.pos + 1 - j0);
+        for (int jj = 0; jj < jend; jj++) {
+          uint4 w[8];
+#pragma unroll
+          for (int c = 0; c < 8; c++) w[c] = sh.tile[jj * 8 + c];
+          hist[score_bucket(token_score(qr, w), R, inv)]++;
+        }
+      }
+    }
+    // bucket of the k-th best score
+    int bstar = DSA_NB - 1;
+    if (active) {
+      int cum = 0;
+      for (int b = 0; b < DSA_NB; b++) {
+        cum += (int)hist[b];
+        if (cum >= topk) {
+          bstar = b;
+          break;
+        }
+      }
+    }
+    // pass 2: collect candidates in buckets <= b*
+    uint32_t *bk = buf_key + (size_t)local * cap;
+    int32_t *bj = buf_j + (size_t)local * cap;
+    for (int j0 = 0; j0 <= jmax; j0 += DSA_KT) {
+      const int nk = min(DSA_KT, jmax + 1 - j0);
+      __syncthreads();
+      for (int i = tid; i < nk * 8; i += DSA_Q) sh.tile[i] = __ldg(kseq + (size_t)j0 * 8 + i);
+      __syncthreads();
+      if (active) {
+        const int jend = min(nk, qi.pos + 1 - j0);
+        for (int jj = 0; jj < jend; jj++) {
+          uint4 w[8];
+#pragma unroll
+          for (int c = 0; c < 8; c++) w[c] = sh.tile[jj * 8 + c];
+          const float sc = token_score(qr, w);
+          if (score_bucket(sc, R, inv) <= bstar) {
+            if (count < cap) {
+              bk[count] = score_key(sc);
+              bj[count] = j0 + jj;
+            }
+            count++;
+          }
+        }
+      }
+    }
+  }
+  if (in_range) cnt_out[local] = count;
+}
+
+struct DsaOut {
+  int32_t *idx;
+  float *scores;
+  const int32_t *bj;
+  __device__ void operator()(int r, int c, uint32_t u) const {
+    idx[r] = bj[c];
+    if (scores) scores[r] = key_score(u);
+  }
+};
+
+struct DirectOut {
+  int32_t *idx;
+  float *scores;
+  __device__ void operator()(int r, int c, uint32_t u) const {
+    idx[r] = c;
+    if (scores) scores[r] = key_score(u);
+  }
+};
+
+struct DsaPad {
+  int32_t *idx;
+  float *scores;
+  __device__ void operator()(int r) const {
+    idx[r] = -1;
+    if (scores) scores[r] = 0.f;
+  }
+};
+
+__host__ __device__ inline size_t dsa_select_smem(int cap, int topk) {
+  return (size_t)cap * 4 + (size_t)16 * topk + sizeof(SelectShared);
+}
+
+__global__ void __launch_bounds__(DSA_SEL_THREADS)
+dsa_select_kernel(int row0, int topk, int cap, const uint32_t *__restrict__ buf_key,
+                  const int32_t *__restrict__ buf_j, const int32_t *__restrict__ cnt,
+                  int32_t *__restrict__ out_idx, float *__restrict__ out_scores) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  const int local = blockIdx.x, row = row0 + local;
+  const int n = cnt[local];
+  if (n > cap) return;  // the fallback kernel owns this row
+  uint32_t *keys = reinterpret_cast<uint32_t *>(smem);
+  uint8_t *rest = smem + (size_t)cap * 4;
+  uint32_t *sel_key = reinterpret_cast<uint32_t *>(rest);
+  int *sel_c = reinterpret_cast<int *>(rest + (size_t)4 * topk);
+  uint32_t *tmp_key = reinterpret_cast<uint32_t *>(rest + (size_t)8 * topk);
+  int *tmp_c = reinterpret_cast<int *>(rest + (size_t)12 * topk);
+  SelectShared &sh = *reinterpret_cast<SelectShared *>(rest + (size_t)16 * topk);
+  const uint32_t *src = buf_key + (size_t)local * cap;
+  for (int i = threadIdx.x; i < n; i += DSA_SEL_THREADS) keys[i] = src[i];
+  __syncthreads();
+  int32_t *oi = out_idx + (size_t)row * topk;
+  float *os = out_scores ? out_scores + (size_t)row * topk : nullptr;
+  select_topk<DSA_SEL_THREADS>(keys, n, topk, sh, sel_key, sel_c, tmp_key, tmp_c,
+                               DsaOut{oi, os, buf_j + (size_t)local * cap}, DsaPad{oi, os});
+}
+
+__global__ void __launch_bounds__(DSA_SEL_THREADS)
+dsa_fallback_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ k,
+                    const int32_t *__restrict__ cu_q, const int32_t *__restrict__ cu_k,
+                    const int32_t *__restrict__ seqlens, int S, int row0, int nrows, int topk,
+                    int cap, const int32_t *__restrict__ cnt, uint32_t *scratch,
+                    size_t scratch_stride, int32_t *__restrict__ out_idx,
+                    float *__restrict__ out_scores, int *status) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  uint32_t *sel_key = reinterpret_cast<uint32_t *>(smem);
+  int *sel_c = reinterpret_cast<int *>(smem + (size_t)4 * topk);
+  uint32_t *tmp_key = reinterpret_cast<uint32_t *>(smem + (size_t)8 * topk);
+  int *tmp_c = reinterpret_cast<int *>(smem + (size_t)12 * topk);
+  SelectShared &sh = *reinterpret_cast<SelectShared *>(smem + (size_t)16 * topk);
+  uint32_t *keys = scratch + (size_t)blockIdx.x * scratch_stride;
+  for (int local = blockIdx.x; local < nrows; local += gridDim.x) {
+    if (cnt[local] <= cap) continue;
+    const int row = row0 + local;
+    const QueryInfo qi = locate(cu_q, cu_k, seqlens, S, row, nullptr);
+    if (!qi.ok) continue;
+    if ((size_t)qi.pos + 1 > scratch_stride) {  // max_seqlen_k understated by the caller
+      if (threadIdx.x == 0) raise_status(status, HISA_ERR_INVALID_ARG);
+      continue;
+    }
+    QRegs qr;
+    load_q(qr, q + (size_t)row * D);
+    const uint4 *kseq = reinterpret_cast<const uint4 *>(k + (size_t)qi.kbase * D);
+    for (int j = threadIdx.x; j <= qi.pos; j += DSA_SEL_THREADS) {
+      uint4 w[8];
+#pragma unroll
+      for (int c = 0; c < 8; c++) w[c] = __ldg(kseq + (size_t)j * 8 + c);
+      keys[j] = score_key(token_score(qr, w));
+    }
+    __syncthreads();
+    int32_t *oi = out_idx + (size_t)row * topk;
+    float *os = out_scores ? out_scores + (size_t)row * topk : nullptr;
+    select_topk<DSA_SEL_THREADS>(keys, qi.pos + 1, topk, sh, sel_key, sel_c, tmp_key, tmp_c,
+                                 DirectOut{oi, os}, DsaPad{oi, os});
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+
+struct DsaPlan {
+  int cap;        // candidate-list capacity per row
+  int chunk;      // rows per filter/select round
+  size_t off_kmax, off_cnt, off_key, off_j, off_fb, total;
+};
+
+static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+DsaPlan dsa_plan(int total_q, int num_seqs, int max_seqlen_k, int topk) {
+  DsaPlan p;
+  p.cap = topk + 2048;
+  // keep the candidate lists to about 512 MiB
+  long long chunk = (512ll << 20) / ((long long)p.cap * 8);
+  chunk = chunk < DSA_Q ? DSA_Q : chunk;
+  chunk = chunk > total_q ? total_q : chunk;
+  p.chunk = (int)(chunk < 1 ? 1 : chunk);
+  size_t off = 0;
+  p.off_kmax = off;
+  off = align256(off + (size_t)(num_seqs > 0 ? num_seqs : 1) * 4);
+  p.off_cnt = off;
+  off = align256(off + (size_t)p.chunk * 4);
+  p.off_key = off;
+  off = align256(off + (size_t)p.chunk * p.cap * 4);
+  p.off_j = off;
+  off = align256(off + (size_t)p.chunk * p.cap * 4);
+  p.off_fb = off;
+  off = align256(off + (size_t)DSA_FB_CTAS * (size_t)(max_seqlen_k > 0 ? max_seqlen_k : 1) * 4);
+  p.total = off;
+  return p;
+}
+
+cudaError_t launch_dsa(const uint16_t *q, const uint16_t *k, const int32_t *cu_q,
+                       const int32_t *cu_k, const int32_t *seqlens, int S, int total_q,
+                       int max_seqlen_k, int topk, int32_t *out_idx, float *out_scores,
+                       uint8_t *ws, int *status, cudaStream_t st) {
+  if (total_q == 0) return cudaSuccess;
+  const DsaPlan p = dsa_plan(total_q, S, max_seqlen_k, topk);
+  float *kmax = reinterpret_cast<float *>(ws + p.off_kmax);
+  int32_t *cnt = reinterpret_cast<int32_t *>(ws + p.off_cnt);
+  uint32_t *bkey = reinterpret_cast<uint32_t *>(ws + p.off_key);
+  int32_t *bj = reinterpret_cast<int32_t *>(ws + p.off_j);
+  uint32_t *fb = reinterpret_cast<uint32_t *>(ws + p.off_fb);
+  cudaError_t e = cudaMemsetAsync(kmax, 0, (size_t)S * 4, st);
+  if (e != cudaSuccess) return e;
+  if (max_seqlen_k > 0) {
+    key_norm_kernel<<<dim3((max_seqlen_k + 255) / 256, S), 256, 0, st>>>(k, cu_k, seqlens, kmax);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  const size_t fsm = sizeof(DsaShared);
+  const size_t ssm = dsa_select_smem(p.cap, topk);
+  const size_t bsm = (size_t)16 * topk + sizeof(SelectShared);
+  if ((e = cudaFuncSetAttribute(dsa_filter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)fsm)) != cudaSuccess)
+    return e;
+  if ((e = cudaFuncSetAttribute(dsa_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)ssm)) != cudaSuccess)
+    return e;
+  if ((e = cudaFuncSetAttribute(dsa_fallback_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)bsm)) != cudaSuccess)
+    return e;
+  for (int row0 = 0; row0 < total_q; row0 += p.chunk) {
+    const int nrows = min(p.chunk, total_q - row0);
+    dsa_filter_kernel<<<(nrows + DSA_Q - 1) / DSA_Q, DSA_Q, fsm, st>>>(
+        q, k, cu_q, cu_k, seqlens, S, row0, nrows, topk, p.cap, kmax, bkey, bj, cnt, status);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    dsa_select_kernel<<<nrows, DSA_SEL_THREADS, ssm, st>>>(row0, topk, p.cap, bkey, bj, cnt,
+                                                            out_idx, out_scores);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    dsa_fallback_kernel<<<DSA_FB_CTAS, DSA_SEL_THREADS, bsm, st>>>(
+        q, k, cu_q, cu_k, seqlens, S, row0, nrows, topk, p.cap, cnt, fb,
+        (size_t)(max_seqlen_k > 0 ? max_seqlen_k : 1), out_idx, out_scores, status);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+size_t dsa_workspace_bytes(int total_q, int num_seqs, int max_seqlen_k, int topk) {
+  return dsa_plan(total_q, num_seqs, max_seqlen_k, topk).total;
+}
+
+}  // namespace hisa

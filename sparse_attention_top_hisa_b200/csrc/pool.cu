@@ -1,0 +1,117 @@
+// Block pooling (hisa_pool_blocks) and decode-time append (hisa_append_keys).
+//
+// HISA summary page (aitrends.kr), paragraph on block partition and mean pooling:
+// each block of B = 128 consecutive keys is represented by the mean of its keys.
+// Paragraph on KV-cache maintenance: the representatives are refreshed when keys
+// are appended.  Both kernels pool with the same warp routine (keys summed in
+// increasing row order in fp32, then one correctly rounded division by the count),
+// so incrementally maintained representatives equal a fresh pool bit for bit.
+#include "common.cuh"
+
+namespace hisa {
+
+// One warp pools one block: lane l owns dims 2l and 2l+1 (one 32-bit word per row).
+// Plain (coherent) loads: the append kernel reads rows written earlier in the same CTA.
+__device__ __forceinline__ void pool_block_warp(const uint32_t *rows, int count, float *rep) {
+  const int lane = threadIdx.x & 31;
+  float a = 0.f, b = 0.f;
+  int t = 0;
+  for (; t + 8 <= count; t += 8) {
+    uint32_t w[8];
+#pragma unroll
+    for (int u = 0; u < 8; u++) w[u] = rows[(t + u) * 32 + lane];
+#pragma unroll
+    for (int u = 0; u < 8; u++) {
+      a += bf_lo(w[u]);
+      b += bf_hi(w[u]);
+    }
+  }
+  for (; t < count; t++) {
+    uint32_t w = rows[t * 32 + lane];
+    a += bf_lo(w);
+    b += bf_hi(w);
+  }
+  const float cnt = (float)count;
+  float2 r = make_float2(__fdiv_rn(a, cnt), __fdiv_rn(b, cnt));
+  reinterpret_cast<float2 *>(rep)[lane] = r;
+}
+
+constexpr int POOL_WARPS = 4;
+
+__global__ void __launch_bounds__(POOL_WARPS * 32)
+pool_blocks_kernel(const uint16_t *__restrict__ k, const int32_t *__restrict__ cu_k,
+                   const int32_t *__restrict__ seqlens, float *__restrict__ reps, int *status) {
+  const int s = blockIdx.y;
+  const int b = blockIdx.x * POOL_WARPS + (threadIdx.x >> 5);
+  const int start = cu_k[s], cap = cu_k[s + 1] - start;
+  const int len = seqlens ? seqlens[s] : cap;
+  if (start % BLK != 0) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) raise_status(status, HISA_ERR_UNALIGNED);
+    return;
+  }
+  if (len < 0 || len > cap) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) raise_status(status, HISA_ERR_INVALID_ARG);
+    return;
+  }
+  if (b * BLK >= len) return;
+  const int count = min(BLK, len - b * BLK);
+  const int row0 = start + b * BLK;
+  pool_block_warp(reinterpret_cast<const uint32_t *>(k + (size_t)row0 * D), count,
+                  reps + (size_t)(row0 / BLK) * D);
+}
+
+__global__ void __launch_bounds__(128)
+append_keys_kernel(uint16_t *__restrict__ kc, float *__restrict__ reps,
+                   const int32_t *__restrict__ cu_k, int32_t *__restrict__ seqlens,
+                   const uint16_t *__restrict__ new_keys, int n_new, int *status) {
+  const int s = blockIdx.x, tid = threadIdx.x, warp = tid >> 5;
+  const int start = cu_k[s], cap = cu_k[s + 1] - start;
+  const int len = seqlens[s];
+  if (start % BLK != 0) {
+    if (tid == 0) raise_status(status, HISA_ERR_UNALIGNED);
+    return;
+  }
+  if (len < 0 || len > cap) {
+    if (tid == 0) raise_status(status, HISA_ERR_INVALID_ARG);
+    return;
+  }
+  if (len + n_new > cap) {
+    if (tid == 0) raise_status(status, HISA_ERR_CAPACITY);
+    return;
+  }
+  // copy the new rows (16-byte chunks)
+  const uint4 *src = reinterpret_cast<const uint4 *>(new_keys + (size_t)s * n_new * D);
+  uint4 *dst = reinterpret_cast<uint4 *>(kc + (size_t)(start + len) * D);
+  for (int i = tid; i < n_new * (ROW_BYTES / 16); i += blockDim.x) dst[i] = src[i];
+  __syncthreads();
+  // re-pool every block the new rows touched
+  const int nlen = len + n_new;
+  const int first = len / BLK, last = (nlen - 1) / BLK;
+  for (int b = first + warp; b <= last; b += blockDim.x / 32) {
+    const int row0 = start + b * BLK;
+    pool_block_warp(reinterpret_cast<const uint32_t *>(kc + (size_t)row0 * D),
+                    min(BLK, nlen - b * BLK), reps + (size_t)(row0 / BLK) * D);
+  }
+  __syncthreads();
+  if (tid == 0) seqlens[s] = nlen;
+}
+
+cudaError_t launch_pool(const uint16_t *k, const int32_t *cu_k, const int32_t *seqlens,
+                        int num_seqs, int max_seqlen_k, float *reps, int *status,
+                        cudaStream_t st) {
+  const int nblk = (max_seqlen_k + BLK - 1) / BLK;
+  if (nblk == 0 || num_seqs == 0) return cudaSuccess;
+  dim3 grid((nblk + POOL_WARPS - 1) / POOL_WARPS, num_seqs);
+  pool_blocks_kernel<<<grid, POOL_WARPS * 32, 0, st>>>(k, cu_k, seqlens, reps, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_append(uint16_t *kc, float *reps, const int32_t *cu_k, int32_t *seqlens,
+                          const uint16_t *new_keys, int n_new, int num_seqs, int *status,
+                          cudaStream_t st) {
+  if (num_seqs == 0 || n_new == 0) return cudaSuccess;
+  append_keys_kernel<<<num_seqs, 128, 0, st>>>(kc, reps, cu_k, seqlens, new_keys, n_new, status);
+  return cudaGetLastError();
+}
+
+}  // namespace hisa

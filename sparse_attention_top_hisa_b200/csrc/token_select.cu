@@ -1,0 +1,223 @@
+// Stage 2 of HISA: gather-score the tokens of the selected blocks and keep the top-k.
+//
+// HISA summary page (aitrends.kr), paragraph on stage 2: only the tokens inside
+// the m selected blocks are scored with the original DSA dot product, and the k
+// best token indices go to the sparse attention operator (the output keeps the
+// DSA layout, paragraph on KV-cache maintenance and compatibility).
+//
+// Candidate c of a query is token j = blk[c / 128] * 128 + c % 128 of the query's
+// sequence; blocks are listed in ascending order, so candidate order is token
+// order.  The token causal mask admits j <= i.
+//
+// Two schedules share the scoring and selection code:
+//   * fused: one CTA per query stages its selected blocks through shared memory
+//     (cp.async, XOR-swizzled 16-byte chunks so that each thread reads its own key
+//     row without bank conflicts), scores them into shared memory and selects;
+//   * split: for few queries (decode) the blocks of each query are scored by
+//     several CTAs into a global scratch row, then one CTA per query selects.
+#include "select.cuh"
+
+namespace hisa {
+
+constexpr int TS_THREADS = 256;
+constexpr int STAGE_ROWS = 256;  // two blocks per staging round
+
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
+  unsigned s = (unsigned)__cvta_generic_to_shared(smem);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit_wait() {
+  asm volatile("cp.async.commit_group;\n" ::: "memory");
+  asm volatile("cp.async.wait_all;\n" ::: "memory");
+}
+
+// Scores selected-block slots [s0, s1) of one query; dst(candidate, key).
+template <class Dst>
+__device__ __forceinline__ void score_slots(const QRegs &q, const uint16_t *kseq, int pos,
+                                            const int32_t *blkrow, int s0, int s1,
+                                            uint8_t *stage, Dst dst) {
+  const int tid = threadIdx.x;
+  for (int p = s0; p < s1; p += 2) {
+    const int nb2 = min(2, s1 - p);
+    for (int i = tid; i < nb2 * BLK * 8; i += TS_THREADS) {
+      const int r = i >> 3, c = i & 7;
+      const int j = blkrow[p + (r >> 7)] * BLK + (r & 127);
+      if (j <= pos)
+        cp_async16(stage + r * ROW_BYTES + ((c ^ (r & 7)) << 4), kseq + (size_t)j * D + c * 8);
+    }
+    cp_async_commit_wait();
+    __syncthreads();
+    if (tid < nb2 * BLK) {
+      const int r = tid;
+      const int j = blkrow[p + (r >> 7)] * BLK + (r & 127);
+      uint32_t key = 0u;
+      if (j <= pos) {
+        uint4 w[8];
+#pragma unroll
+        for (int c = 0; c < 8; c++)
+          w[c] = *reinterpret_cast<const uint4 *>(stage + r * ROW_BYTES + ((c ^ (r & 7)) << 4));
+        key = score_key(token_score(q, w));
+      }
+      dst((p << 7) + r, key);
+    }
+    __syncthreads();
+  }
+}
+
+__device__ __forceinline__ int count_selected(const int32_t *blkrow, int m) {
+  int n = 0;
+  while (n < m && blkrow[n] >= 0) n++;
+  return n;
+}
+
+struct TokenOut {
+  int32_t *idx;
+  float *scores;
+  const int32_t *blkrow;
+  __device__ void operator()(int r, int c, uint32_t u) const {
+    idx[r] = blkrow[c >> 7] * BLK + (c & 127);
+    if (scores) scores[r] = key_score(u);
+  }
+};
+
+struct RowPad {
+  int32_t *idx;
+  float *scores;
+  __device__ void operator()(int r) const {
+    idx[r] = -1;
+    if (scores) scores[r] = 0.f;
+  }
+};
+
+// shared-memory layout of the selecting kernels
+__host__ __device__ inline size_t stage_bytes(int topk) {
+  size_t a = (size_t)STAGE_ROWS * ROW_BYTES, b = (size_t)16 * topk;
+  return a > b ? a : b;
+}
+__host__ __device__ inline size_t token_smem_bytes(int m, int topk) {
+  return (size_t)m * BLK * 4 + stage_bytes(topk) + sizeof(SelectShared);
+}
+
+__global__ void __launch_bounds__(TS_THREADS)
+token_fused_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ k,
+                   const int32_t *__restrict__ cu_q, const int32_t *__restrict__ cu_k,
+                   const int32_t *__restrict__ seqlens, int S, int m, int topk,
+                   const int32_t *__restrict__ blk, int32_t *__restrict__ out_idx,
+                   float *__restrict__ out_scores, int *status) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  uint32_t *keys = reinterpret_cast<uint32_t *>(smem);
+  uint8_t *stage = smem + (size_t)m * BLK * 4;
+  SelectShared &sh = *reinterpret_cast<SelectShared *>(stage + stage_bytes(topk));
+  const int row = blockIdx.x;
+  RowPad pad{out_idx + (size_t)row * topk, out_scores ? out_scores + (size_t)row * topk : nullptr};
+  const QueryInfo qi = locate(cu_q, cu_k, seqlens, S, row, nullptr);
+  if (!qi.ok) {  // already reported by the block stage
+    for (int r = threadIdx.x; r < topk; r += TS_THREADS) pad(r);
+    return;
+  }
+  const int32_t *blkrow = blk + (size_t)row * m;
+  const int nsel = count_selected(blkrow, m);
+  QRegs qr;
+  load_q(qr, q + (size_t)row * D);
+  score_slots(qr, k + (size_t)qi.kbase * D, qi.pos, blkrow, 0, nsel, stage,
+              [&](int c, uint32_t key) { keys[c] = key; });
+  uint32_t *sel_key = reinterpret_cast<uint32_t *>(stage);
+  int *sel_c = reinterpret_cast<int *>(stage + (size_t)4 * topk);
+  uint32_t *tmp_key = reinterpret_cast<uint32_t *>(stage + (size_t)8 * topk);
+  int *tmp_c = reinterpret_cast<int *>(stage + (size_t)12 * topk);
+  TokenOut out{pad.idx, pad.scores, blkrow};
+  select_topk<TS_THREADS>(keys, nsel * BLK, topk, sh, sel_key, sel_c, tmp_key, tmp_c, out, pad);
+}
+
+__global__ void __launch_bounds__(TS_THREADS)
+token_score_split_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ k,
+                         const int32_t *__restrict__ cu_q, const int32_t *__restrict__ cu_k,
+                         const int32_t *__restrict__ seqlens, int S, int m,
+                         const int32_t *__restrict__ blk, int slots_per_cta,
+                         uint32_t *__restrict__ scratch) {
+  __shared__ __align__(16) uint8_t stage[STAGE_ROWS * ROW_BYTES];
+  const int row = blockIdx.x;
+  const QueryInfo qi = locate(cu_q, cu_k, seqlens, S, row, nullptr);
+  if (!qi.ok) return;
+  const int32_t *blkrow = blk + (size_t)row * m;
+  const int nsel = count_selected(blkrow, m);
+  const int s0 = blockIdx.y * slots_per_cta, s1 = min(nsel, s0 + slots_per_cta);
+  if (s0 >= s1) return;
+  QRegs qr;
+  load_q(qr, q + (size_t)row * D);
+  uint32_t *dst = scratch + (size_t)row * m * BLK;
+  score_slots(qr, k + (size_t)qi.kbase * D, qi.pos, blkrow, s0, s1, stage,
+              [&](int c, uint32_t key) { dst[c] = key; });
+}
+
+__global__ void __launch_bounds__(TS_THREADS)
+token_select_scratch_kernel(const int32_t *__restrict__ cu_q, const int32_t *__restrict__ cu_k,
+                            const int32_t *__restrict__ seqlens, int S, int m, int topk,
+                            const int32_t *__restrict__ blk, const uint32_t *__restrict__ scratch,
+                            int32_t *__restrict__ out_idx, float *__restrict__ out_scores) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  uint32_t *keys = reinterpret_cast<uint32_t *>(smem);
+  uint8_t *stage = smem + (size_t)m * BLK * 4;
+  SelectShared &sh = *reinterpret_cast<SelectShared *>(stage + stage_bytes(topk));
+  const int row = blockIdx.x;
+  RowPad pad{out_idx + (size_t)row * topk, out_scores ? out_scores + (size_t)row * topk : nullptr};
+  const QueryInfo qi = locate(cu_q, cu_k, seqlens, S, row, nullptr);
+  if (!qi.ok) {
+    for (int r = threadIdx.x; r < topk; r += TS_THREADS) pad(r);
+    return;
+  }
+  const int32_t *blkrow = blk + (size_t)row * m;
+  const int nsel = count_selected(blkrow, m);
+  const uint4 *src = reinterpret_cast<const uint4 *>(scratch + (size_t)row * m * BLK);
+  for (int i = threadIdx.x; i < nsel * BLK / 4; i += TS_THREADS)
+    reinterpret_cast<uint4 *>(keys)[i] = src[i];
+  __syncthreads();
+  uint32_t *sel_key = reinterpret_cast<uint32_t *>(stage);
+  int *sel_c = reinterpret_cast<int *>(stage + (size_t)4 * topk);
+  uint32_t *tmp_key = reinterpret_cast<uint32_t *>(stage + (size_t)8 * topk);
+  int *tmp_c = reinterpret_cast<int *>(stage + (size_t)12 * topk);
+  TokenOut out{pad.idx, pad.scores, blkrow};
+  select_topk<TS_THREADS>(keys, nsel * BLK, topk, sh, sel_key, sel_c, tmp_key, tmp_c, out, pad);
+}
+
+// Split schedule when there are too few queries to fill the GPU with one CTA each.
+bool token_use_split(int total_q, int num_sms) { return total_q < 2 * num_sms; }
+
+size_t token_scratch_bytes(int total_q, int m, int num_sms) {
+  return token_use_split(total_q, num_sms) ? (size_t)total_q * m * BLK * 4 : 0;
+}
+
+cudaError_t launch_token_select(const uint16_t *q, const uint16_t *k, const int32_t *cu_q,
+                                const int32_t *cu_k, const int32_t *seqlens, int S, int total_q,
+                                int m, int topk, const int32_t *blk, uint32_t *scratch,
+                                int num_sms, int32_t *out_idx, float *out_scores, int *status,
+                                cudaStream_t st) {
+  if (total_q == 0) return cudaSuccess;
+  const size_t smem = token_smem_bytes(m, topk);
+  if (token_use_split(total_q, num_sms)) {
+    // spread each query's blocks over enough CTAs to cover the SMs about twice
+    int splits = (2 * num_sms + total_q - 1) / total_q;
+    splits = splits < 1 ? 1 : (splits > m ? m : splits);
+    int slots = (m + splits - 1) / splits;
+    slots = (slots + 1) & ~1;  // whole staging rounds
+    splits = (m + slots - 1) / slots;
+    token_score_split_kernel<<<dim3(total_q, splits), TS_THREADS, 0, st>>>(
+        q, k, cu_q, cu_k, seqlens, S, m, blk, slots, scratch);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(token_select_scratch_kernel,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    token_select_scratch_kernel<<<total_q, TS_THREADS, smem, st>>>(
+        cu_q, cu_k, seqlens, S, m, topk, blk, scratch, out_idx, out_scores);
+    return cudaGetLastError();
+  }
+  cudaError_t e = cudaFuncSetAttribute(token_fused_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  token_fused_kernel<<<total_q, TS_THREADS, smem, st>>>(q, k, cu_q, cu_k, seqlens, S, m, topk,
+                                                        blk, out_idx, out_scores, status);
+  return cudaGetLastError();
+}
+
+}  // namespace hisa
