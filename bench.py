@@ -1,0 +1,579 @@
+#!/usr/bin/env python
+"""Benchmark of the HISA token-selection indexer on one node.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step is one HISA selection over the 131072-token prefill (1 sequence, q/k
+bf16 ~ N(0,1), d = 64, B = 128, m = 64, k = 2048): block pooling, stage 1
+(block scores, top-m) and stage 2 (gather-score, top-k), all through the
+library's C ABI.  Inputs live in HBM before the timed region; L2 is flushed
+(a 256 MiB write) before every timed step, outside the step's CUDA events.
+The same run measures, and reports under "details": the flat DSA scan on the
+same input (the HISA/DSA speedup), the 32768-token needle prefill (speedup,
+IoU and needle recall), and decode (16 sequences x 32768 keys, one append and
+one selection per step, 256 steps in a CUDA graph over four independent
+decode states so that the key caches cannot stay in L2).
+
+Under torchrun (N > 1) every rank runs the same workload on its own GPU (weak
+scaling, no collective on the data path); times are the maximum over ranks.
+``--impl reference`` times the CPU oracle instead (the only other place this
+script runs the oracle) on seeded samples of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "HISA top-k selection queries/s & ms at 32K/128K; HBM GB/s vs peak"
+UNIT = "queries/s"
+WORKLOAD = "prefill_L131072 (1 seq, q/k bf16 N(0,1), d=64, B=128, m=64, k=2048)"
+L2_FLUSH_BYTES = 256 << 20
+
+# DRAM bytes per launch read from an ncu capture, keyed by kernel kind, with the
+# sha256 of the kernel source the capture was taken on (a changed source voids it).
+TRAFFIC = {}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-extras", action="store_true", help="skip the details measurements")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
+    return ap.parse_args()
+
+
+def cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# clocks during the measured region
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap,pci.bus_id")
+
+    def __init__(self, bus_id: str):
+        self.bus_id = bus_id.lower()
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        threading.Thread(target=self._read, daemon=True).start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in list(self.lines):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            bus = parts[7].lower()
+            if self.bus_id and not (bus.endswith(self.bus_id) or self.bus_id.endswith(bus)):
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# helpers
+
+def dist_setup(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    import torch
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def to_dev_bf16(a):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def to_dev_i32(a):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).cuda()
+
+
+def candidates_per_query(pos: np.ndarray, B: int, m: int) -> np.ndarray:
+    """Stage-2 candidates of a query at position p (single sequence): every token of the
+    selected blocks up to p; m blocks are selected, all full except the own block."""
+    full = pos + 1
+    capped = (m - 1) * B + (pos % B) + 1
+    return np.minimum(full, capped)
+
+
+def iou_rows(a: np.ndarray, b: np.ndarray) -> float:
+    vals = []
+    for x, y in zip(a, b):
+        x = x[x >= 0]
+        y = y[y >= 0]
+        u = np.union1d(x, y).size
+        vals.append(np.intersect1d(x, y).size / u if u else 1.0)
+    return float(np.mean(vals))
+
+
+def source_sha(name: str) -> str:
+    path = os.path.join(ROOT, "sparse_attention_top_hisa_b200", "csrc", name)
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+# ---------------------------------------------------------------------------
+# our arm
+
+def run_ours(args, world, rank):
+    import torch
+    import sparse_attention_top_hisa_b200 as H
+    from synth import config_workload
+
+    hbm_peak, tc_peak, peak_src = peaks()
+    dev = torch.cuda.current_device()
+    props = torch.cuda.get_device_properties(dev)
+    bus = ""
+    try:
+        bus = "%04x:%02x:%02x.0" % (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
+    except AttributeError:
+        pass
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+
+    w = config_workload(4)
+    B, m, K = w.B, w.m, w.topk
+    nq = w.total_q
+    q, k = to_dev_bf16(w.q), to_dev_bf16(w.k)
+    cu_q, cu_k, sl = to_dev_i32(w.cu_q), to_dev_i32(w.cu_k), to_dev_i32(w.seqlens)
+    out = torch.empty(nq, K, dtype=torch.int32, device="cuda")
+    reps = torch.zeros(w.rep_rows, 64, dtype=torch.float32, device="cuda")
+    ws = torch.empty(max(H.hisa_select_workspace_size(nq, 1, w.max_seqlen_k, m, K), 256),
+                     dtype=torch.uint8, device="cuda")
+
+    def step():
+        H.hisa_pool_blocks(k, cu_k, sl, w.max_seqlen_k, reps=reps)
+        H.hisa_select(q, k, reps, cu_q, cu_k, sl, w.max_seqlen_k, m, K, out_idx=out, workspace=ws)
+
+    H.hisa_device_status(clear=True)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert H.hisa_device_status() == 0, "device-side error during warm-up"
+
+    sampler = ClockSampler(bus) if rank == 0 else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+
+    # ---- timed region ----------------------------------------------------------
+    H.hisa_timing_collect(reset=True)
+    H.hisa_timing_enable(True)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    barrier(world)
+    t_wall = time.perf_counter()
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    barrier(world)
+    t_wall = time.perf_counter() - t_wall
+    H.hisa_timing_enable(False)
+    kt = H.hisa_timing_collect(reset=True)
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    ms = max_over_ranks(sum(step_ms) / len(step_ms), world)
+    launches = int(sum(v["launches"] for v in kt.values()))
+    value = world * nq / (ms / 1e3)
+
+    # ---- end to end: host buffers through the public API --------------------------
+    hq = torch.from_numpy(np.ascontiguousarray(w.q).view(np.int16)).view(torch.bfloat16).pin_memory()
+    hk = torch.from_numpy(np.ascontiguousarray(w.k).view(np.int16)).view(torch.bfloat16).pin_memory()
+    hcq = torch.from_numpy(w.cu_q.astype(np.int32)).pin_memory()
+    hck = torch.from_numpy(w.cu_k.astype(np.int32)).pin_memory()
+    hsl = torch.from_numpy(w.seqlens.astype(np.int32)).pin_memory()
+    hout = torch.empty(nq, K, dtype=torch.int32).pin_memory()
+    e2e_steps = max(2, min(args.steps, 5))
+    e2e_ms = []
+    for i in range(e2e_steps + 1):
+        flush.fill_(i & 0xFF)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        q.copy_(hq, non_blocking=True)
+        k.copy_(hk, non_blocking=True)
+        cu_q.copy_(hcq, non_blocking=True)
+        cu_k.copy_(hck, non_blocking=True)
+        sl.copy_(hsl, non_blocking=True)
+        step()
+        hout.copy_(out, non_blocking=True)
+        b.record(stream)
+        b.synchronize()
+        if i > 0:
+            e2e_ms.append(a.elapsed_time(b))
+    e2e = max_over_ranks(sum(e2e_ms) / len(e2e_ms), world)
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hcq, hck, hsl))
+    d2h = hout.numel() * hout.element_size()
+
+    # ---- roofline of the dominant kernel -------------------------------------------
+    dom = max(kt.items(), key=lambda kv: kv[1]["ms"])
+    dname, dstat = dom[0], dom[1]
+    per_launch_ms = dstat["ms"] / max(dstat["timed"], 1)
+    pos = np.arange(nq)
+    if dname == "token_fused":
+        cands = float(candidates_per_query(pos, B, m).sum())
+        flops = cands * 64 * 2
+        alu_peak = 148 * 128 * 2 * 1.965e9 / 1e12  # FP32 lanes x 2 flop x max SM clock, TFLOP/s
+        achieved = flops / (per_launch_ms / 1e3) / 1e12
+        roof = {"kernel": dname, "bound": "alu", "achieved": round(achieved, 3),
+                "peak": round(alu_peak, 2), "unit": "TFLOP/s", "frac": round(achieved / alu_peak, 4),
+                "peak_source": "148 SMs x 128 FP32 lanes x 2 x 1965 MHz",
+                "algorithmic": f"{cands:.4g} candidates x 64 FMA",
+                "launch_ms": round(per_launch_ms, 4)}
+    else:
+        nbytes = {"pool_blocks": nq * 128 + w.rep_rows * 256,
+                  "block_select": nq * 128 + nq * m * 4}.get(dname, 0)
+        achieved = nbytes / (per_launch_ms / 1e3) / 1e9
+        roof = {"kernel": dname, "bound": "hbm", "achieved": round(achieved, 1),
+                "peak": hbm_peak, "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
+                "launch_ms": round(per_launch_ms, 4)}
+    t = TRAFFIC.get(dname)
+    roof["traffic"] = t[0] if t and t[1] == source_sha(t[2]) else None
+    roof["peak_source"] = roof.get("peak_source", f"MEASURED_PEAKS.json ({peak_src})")
+
+    details = {"hisa_128k": {"ms": round(ms, 4), "queries_per_s": round(nq / (ms / 1e3), 1),
+                             "kernels": {n: {"ms_per_step": round(v["ms"] / args.steps, 4),
+                                             "launches": v["launches"]}
+                                         for n, v in kt.items() if v["launches"]}}}
+    if rank == 0 and not args.no_extras:
+        details.update(extras(args, w, q, k, cu_q, cu_k, sl, out, flush, stream, hbm_peak))
+
+    clocks = sampler.stop() if sampler else None
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "seq_len": 131072, "queries_per_step": nq * world,
+                   "d": 64, "B": B, "m": m, "k": K, "inputs": "bf16 q/k, PCG64 seed 20264",
+                   "l2": "256 MiB flush before every timed step (outside the step events)",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "e2e": {"value": round(world * nq / (e2e / 1e3), 1), "unit": UNIT,
+                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+                "ms_per_step": round(e2e, 3)},
+        "gpu_launches": launches,
+        "roofline": roof,
+        "clocks": clocks,
+        "wall_s_timed_region": round(t_wall, 3),
+        "details": details,
+    }
+    if rank == 0 and not args.no_cpu:
+        line["cpu_baseline"] = cpu_baseline(w)
+    return line
+
+
+def time_events(fn, reps, flush, stream):
+    import torch
+    out = []
+    for i in range(reps):
+        flush.fill_(i & 0xFF)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        b.synchronize()
+        out.append(a.elapsed_time(b))
+    return out
+
+
+def extras(args, w4, q4, k4, cu_q4, cu_k4, sl4, out4, flush, stream, hbm_peak):
+    """Flat DSA at 128K, the 32K needle prefill, decode, IoU."""
+    import torch
+    import sparse_attention_top_hisa_b200 as H
+    from synth import config_workload
+    det = {}
+    nq, K = w4.total_q, w4.topk
+    # flat DSA at 128K
+    dout = torch.empty(nq, K, dtype=torch.int32, device="cuda")
+    dws = torch.empty(H.dsa_flat_workspace_size(nq, 1, w4.max_seqlen_k, K), dtype=torch.uint8,
+                      device="cuda")
+    dsa = lambda: H.dsa_flat_select(q4, k4, cu_q4, cu_k4, sl4, w4.max_seqlen_k, K, out_idx=dout,
+                                    workspace=dws)
+    dsa()
+    dms = time_events(dsa, 2, flush, stream)
+    hms = None
+    rows = np.random.Generator(np.random.PCG64(1)).choice(nq, 2048, replace=False)
+    iou = iou_rows(out4.cpu().numpy()[rows], dout.cpu().numpy()[rows])
+    det["dsa_128k"] = {"ms": round(min(dms), 3), "iou_hisa_vs_dsa_2048_rows": round(iou, 4)}
+    del dout, dws
+    torch.cuda.empty_cache()
+
+    # 32K needle prefill
+    w3 = config_workload(3)
+    q3, k3 = to_dev_bf16(w3.q), to_dev_bf16(w3.k)
+    cq3, ck3, sl3 = to_dev_i32(w3.cu_q), to_dev_i32(w3.cu_k), to_dev_i32(w3.seqlens)
+    reps3 = torch.zeros(w3.rep_rows, 64, dtype=torch.float32, device="cuda")
+    o3 = torch.empty(w3.total_q, w3.topk, dtype=torch.int32, device="cuda")
+    d3 = torch.empty_like(o3)
+    ws3 = torch.empty(H.hisa_select_workspace_size(w3.total_q, 1, w3.max_seqlen_k, w3.m, w3.topk),
+                      dtype=torch.uint8, device="cuda")
+    dws3 = torch.empty(H.dsa_flat_workspace_size(w3.total_q, 1, w3.max_seqlen_k, w3.topk),
+                       dtype=torch.uint8, device="cuda")
+
+    def h3():
+        H.hisa_pool_blocks(k3, ck3, sl3, w3.max_seqlen_k, reps=reps3)
+        H.hisa_select(q3, k3, reps3, cq3, ck3, sl3, w3.max_seqlen_k, w3.m, w3.topk, out_idx=o3,
+                      workspace=ws3)
+
+    def f3():
+        H.dsa_flat_select(q3, k3, cq3, ck3, sl3, w3.max_seqlen_k, w3.topk, out_idx=d3,
+                          workspace=dws3)
+    h3()
+    f3()
+    hm3 = statistics.median(time_events(h3, 5, flush, stream))
+    dm3 = statistics.median(time_events(f3, 3, flush, stream))
+    a3, b3 = o3.cpu().numpy(), d3.cpu().numpy()
+    rec_h = np.mean([j in a3[i] for i, j in w3.needles])
+    rec_d = np.mean([j in b3[i] for i, j in w3.needles])
+    rows3 = np.random.Generator(np.random.PCG64(2)).choice(w3.total_q, 4096, replace=False)
+    det["prefill_32k"] = {"hisa_ms": round(hm3, 3), "dsa_ms": round(dm3, 3),
+                          "hisa_speedup_over_dsa": round(dm3 / hm3, 2),
+                          "hisa_queries_per_s": round(w3.total_q / (hm3 / 1e3), 1),
+                          "iou_hisa_vs_dsa_4096_rows": round(iou_rows(a3[rows3], b3[rows3]), 4),
+                          "needle_recall_hisa": float(rec_h), "needle_recall_dsa": float(rec_d)}
+    det["dsa_128k"]["hisa_speedup_over_dsa"] = None  # filled by the caller
+    del q3, k3, o3, d3, ws3, dws3
+    torch.cuda.empty_cache()
+    det["decode"] = decode_bench(flush, stream, hbm_peak)
+    return det
+
+
+def decode_bench(flush, stream, hbm_peak, n_states=4, steps=256):
+    """16 sequences x 32768 keys; each step appends one key per sequence and selects
+    for one query per sequence. Steps rotate over n_states independent decode states
+    (4 x 67.6 MB of key cache > L2) and the 256 steps run as one CUDA graph."""
+    import torch
+    import sparse_attention_top_hisa_b200 as H
+    from synth import config_workload
+    dw = config_workload(2, steps=steps)
+    S, cap, m, K = dw.num_seqs, dw.capacity, dw.m, dw.topk
+    cu_k = to_dev_i32(dw.cu_k)
+    cu_q = to_dev_i32(np.arange(S + 1))
+    states = []
+    for r in range(n_states):
+        kc = to_dev_bf16(dw.k_cache)
+        lens = to_dev_i32(dw.seqlens0)
+        reps = H.hisa_pool_blocks(kc, cu_k, lens, cap)
+        out = torch.empty(S, K, dtype=torch.int32, device="cuda")
+        states.append((kc, lens, reps, out))
+    lens0 = to_dev_i32(dw.seqlens0)
+    newk = to_dev_bf16(dw.new_keys)  # [steps, S, 1, 64]
+    qs = to_dev_bf16(dw.queries.reshape(steps * S, 64)).view(steps, S, 64)
+    ws = torch.empty(H.hisa_select_workspace_size(S, S, cap, m, K), dtype=torch.uint8, device="cuda")
+
+    def run_steps():
+        for i in range(steps):
+            kc, lens, reps, out = states[i % n_states]
+            H.hisa_append_keys(kc, reps, cu_k, lens, newk[i])
+            H.hisa_select(qs[i], kc, reps, cu_q, cu_k, lens, cap, m, K, out_idx=out, workspace=ws)
+
+    def reset():
+        for kc, lens, reps, out in states:
+            lens.copy_(lens0)
+
+    # warm-up (sets kernel attributes), then capture
+    run_steps()
+    torch.cuda.synchronize()
+    reset()
+    H.hisa_timing_collect(reset=True)
+    g = torch.cuda.CUDAGraph()
+    s2 = torch.cuda.Stream()
+    s2.wait_stream(stream)
+    with torch.cuda.stream(s2):
+        with torch.cuda.graph(g, stream=s2):
+            run_steps()
+    torch.cuda.current_stream().wait_stream(s2)
+    launches_per_graph = int(sum(v["launches"] for v in H.hisa_timing_collect(reset=True).values()))
+    times = []
+    for i in range(3):
+        reset()
+        flush.fill_(i)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        g.replay()
+        b.record(stream)
+        b.synchronize()
+        times.append(a.elapsed_time(b))
+    assert H.hisa_device_status() == 0
+    per_step_us = min(times) / steps * 1e3
+    # algorithmic bytes per sequence-step: reps of the eligible blocks, the m*B gathered
+    # keys, the query, the k output indices, and the append (last block re-read + one row
+    # + one representative written)
+    eligible = (int(dw.seqlens0[0]) + steps // 2) // 128 + 1
+    per_seq = eligible * 256 + m * 128 * 128 + 128 + K * 4 + (128 * 128 + 128 + 256)
+    gbs = per_seq * S / (per_step_us * 1e-6) / 1e9
+    del g
+    return {"us_per_step": round(per_step_us, 2), "steps_per_graph": steps,
+            "launches_per_step": launches_per_graph / steps,
+            "algorithmic_MB_per_step": round(per_seq * S / 1e6, 2),
+            "GBs": round(gbs, 1), "frac_of_hbm_peak": round(gbs / hbm_peak, 4),
+            "states": n_states}
+
+
+def cpu_baseline(w, budget_s: float = 15.0):
+    """The oracle (unchanged) on the host cores, on a seeded sample of query rows."""
+    import oracle
+    n = cores()
+    rng = np.random.Generator(np.random.PCG64(99))
+    rows = np.sort(rng.choice(w.total_q, 512, replace=False)).astype(np.int32)
+    t0 = time.perf_counter()
+    oracle.hisa_workload(w, rows=rows, nthreads=n)
+    t1 = time.perf_counter() - t0
+    target = int(min(w.total_q, max(512, 512 * budget_s / max(t1, 1e-3))))
+    rows = np.sort(rng.choice(w.total_q, target, replace=False)).astype(np.int32)
+    t0 = time.perf_counter()
+    oracle.hisa_workload(w, rows=rows, nthreads=n)
+    t1 = time.perf_counter() - t0
+    return {"value": round(target / t1, 2), "unit": UNIT, "cores": n, "kind": "oracle",
+            "sample": f"{target} seeded query rows of the 131072 (pooling over all keys each call)",
+            "seconds": round(t1, 2)}
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the CPU oracle
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return None
+    import oracle
+    from synth import config_workload
+    w = config_workload(4)
+    n = cores()
+    rng = np.random.Generator(np.random.PCG64(7))
+    sample = 4096
+    times = []
+    for i in range(args.warmup + args.steps):
+        rows = np.sort(rng.choice(w.total_q, sample, replace=False)).astype(np.int32)
+        t0 = time.perf_counter()
+        oracle.hisa_workload(w, rows=rows, nthreads=n)
+        dt = time.perf_counter() - t0
+        if i >= args.warmup:
+            times.append(dt)
+    ms = 1e3 * sum(times) / len(times)
+    v = sample / (ms / 1e3)
+    return {"impl": "reference", "metric": METRIC, "value": round(v, 2), "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "seq_len": 131072, "d": 64, "B": 128, "m": 64,
+                       "k": 2048, "sample_rows_per_step": sample},
+            "cpu_baseline": {"value": round(v, 2), "unit": UNIT, "cores": n, "kind": "oracle",
+                             "sample": f"{sample} seeded query rows of the 131072 per step"},
+            "e2e": {"value": round(v, 2), "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        line = run_reference(args, world, rank)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    world, rank, _ = dist_setup(args)
+    line = run_ours(args, world, rank)
+    if rank == 0:
+        d = line["details"]
+        if "dsa_128k" in d:
+            d["dsa_128k"]["hisa_speedup_over_dsa"] = round(d["dsa_128k"]["ms"] / line["ms_per_step"], 2)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -202,6 +202,27 @@ size_t dsa_flat_workspace_size(int total_q, int num_seqs, int max_seqlen_k, int 
  */
 hisa_status hisa_device_status(int32_t *status, int clear, hisa_stream_t stream);
 
+/*
+ * Launch accounting, for benchmarks and tests (no counterpart on the pages).
+ * Every kernel launch made by this library is counted per kernel kind.  With
+ * timing enabled, each launch is also bracketed by a pair of CUDA events
+ * recorded on its launch stream.  Host-side state shared by all callers of the
+ * process; not thread-safe; leave timing off while capturing a CUDA graph.
+ *
+ * hisa_timing_enable  — turn event timing on (1) or off (0).
+ * hisa_kernel_kinds   — number of kernel kinds; hisa_kernel_name(i) names kind i.
+ * hisa_timing_collect — wait for every recorded event, then write per kind the
+ *                       total event time in ms (ms[i]), the launches counted
+ *                       (launches[i]) and the launches timed (timed[i]) since the
+ *                       last reset, for i < n; any of the arrays may be NULL.
+ *                       reset != 0 zeroes the counters afterwards.
+ */
+hisa_status hisa_timing_enable(int on);
+int hisa_kernel_kinds(void);
+const char *hisa_kernel_name(int kind);
+hisa_status hisa_timing_collect(double *ms, long long *launches, long long *timed, int n,
+                                int reset);
+
 #ifdef __cplusplus
 }
 #endif

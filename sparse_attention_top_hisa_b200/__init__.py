@@ -20,5 +20,7 @@ from .binding import (  # noqa: F401
     hisa_pool_blocks,
     hisa_select,
     hisa_select_workspace_size,
+    hisa_timing_collect,
+    hisa_timing_enable,
     lib,
 )

@@ -46,6 +46,10 @@ EXPORTED = (
     "dsa_flat_select",
     "dsa_flat_workspace_size",
     "hisa_device_status",
+    "hisa_timing_enable",
+    "hisa_kernel_kinds",
+    "hisa_kernel_name",
+    "hisa_timing_collect",
 )
 
 
@@ -79,6 +83,13 @@ def lib() -> ctypes.CDLL:
         L.dsa_flat_workspace_size.argtypes = [I, I, I, I]
         L.dsa_flat_workspace_size.restype = Z
         L.hisa_device_status.argtypes = [P, I, P]
+        L.hisa_timing_enable.argtypes = [I]
+        L.hisa_timing_enable.restype = I
+        L.hisa_kernel_kinds.restype = I
+        L.hisa_kernel_name.argtypes = [I]
+        L.hisa_kernel_name.restype = ctypes.c_char_p
+        L.hisa_timing_collect.argtypes = [P, P, P, I, I]
+        L.hisa_timing_collect.restype = I
         for f in ("hisa_pool_blocks", "hisa_append_keys", "hisa_select", "dsa_flat_select",
                   "hisa_device_status"):
             getattr(L, f).restype = I
@@ -227,3 +238,21 @@ def hisa_device_status(clear: bool = True, stream=None) -> int:
     _check(lib().hisa_device_status(ctypes.byref(v), 1 if clear else 0, _stream(stream)),
            "hisa_device_status")
     return int(v.value)
+
+
+def hisa_timing_enable(on: bool) -> None:
+    """Bracket every library kernel launch with CUDA events on its stream (or stop)."""
+    _check(lib().hisa_timing_enable(1 if on else 0), "hisa_timing_enable")
+
+
+def hisa_timing_collect(reset: bool = True) -> dict:
+    """Per kernel kind: {'ms': total event time, 'launches': count, 'timed': timed count}."""
+    L = lib()
+    n = L.hisa_kernel_kinds()
+    ms = (ctypes.c_double * n)()
+    launches = (ctypes.c_longlong * n)()
+    timed = (ctypes.c_longlong * n)()
+    _check(L.hisa_timing_collect(ms, launches, timed, n, 1 if reset else 0),
+           "hisa_timing_collect")
+    return {L.hisa_kernel_name(i).decode(): {"ms": ms[i], "launches": launches[i],
+                                             "timed": timed[i]} for i in range(n)}

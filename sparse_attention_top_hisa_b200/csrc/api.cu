@@ -4,7 +4,10 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <vector>
+
 #include "common.cuh"
+#include "prof.cuh"
 
 namespace hisa {
 cudaError_t launch_pool(const uint16_t *k, const int32_t *cu_k, const int32_t *seqlens,
@@ -31,6 +34,55 @@ size_t dsa_workspace_bytes(int total_q, int num_seqs, int max_seqlen_k, int topk
 }  // namespace hisa
 
 using namespace hisa;
+
+// ---------------------------------------------------------------------------
+// launch accounting (see prof.cuh); host-side state, not thread-safe
+
+namespace {
+const char *kKindNames[K_NUM_KINDS] = {
+    "pool_blocks",        "append_keys",         "block_select",   "token_fused",
+    "token_score_split",  "token_select_scratch", "key_norm",      "dsa_filter",
+    "dsa_select",         "dsa_fallback"};
+long long g_launches[K_NUM_KINDS];
+double g_ms[K_NUM_KINDS];
+long long g_timed[K_NUM_KINDS];
+bool g_timing = false;
+struct Pending {
+  int kind;
+  cudaEvent_t a, b;
+};
+std::vector<Pending> g_pending;
+std::vector<cudaEvent_t> g_free_events;
+Pending g_open{-1, nullptr, nullptr};
+
+cudaEvent_t take_event() {
+  if (!g_free_events.empty()) {
+    cudaEvent_t e = g_free_events.back();
+    g_free_events.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+  return e;
+}
+}  // namespace
+
+namespace hisa {
+void prof_before(int kind, cudaStream_t st) {
+  if (kind >= 0 && kind < K_NUM_KINDS) g_launches[kind]++;
+  if (!g_timing) return;
+  g_open.kind = kind;
+  g_open.a = take_event();
+  g_open.b = take_event();
+  if (g_open.a) cudaEventRecord(g_open.a, st);
+}
+void prof_after(int kind, cudaStream_t st) {
+  if (!g_timing || g_open.kind != kind || !g_open.a || !g_open.b) return;
+  cudaEventRecord(g_open.b, st);
+  g_pending.push_back(g_open);
+  g_open.kind = -1;
+}
+}  // namespace hisa
 
 // Sticky device status word (one per device that loads the library).
 static __device__ int g_hisa_status;
@@ -212,6 +264,47 @@ hisa_status dsa_flat_select(const hisa_bf16 *q_idx, const hisa_bf16 *k_idx,
   return from_cuda(launch_dsa(q_idx, k_idx, cu_seqlens_q, cu_seqlens_k, seqlens_k, num_seqs,
                               total_q, max_seqlen_k, k, out_idx, out_scores,
                               static_cast<uint8_t *>(ws), st, static_cast<cudaStream_t>(stream)));
+}
+
+hisa_status hisa_timing_enable(int on) {
+  g_timing = on != 0;
+  return HISA_OK;
+}
+
+int hisa_kernel_kinds(void) { return K_NUM_KINDS; }
+
+const char *hisa_kernel_name(int kind) {
+  return (kind >= 0 && kind < K_NUM_KINDS) ? kKindNames[kind] : "";
+}
+
+hisa_status hisa_timing_collect(double *ms, long long *launches, long long *timed, int n,
+                                int reset) {
+  hisa_status rc = HISA_OK;
+  for (const Pending &p : g_pending) {
+    float t = 0.f;
+    if (cudaEventSynchronize(p.b) != cudaSuccess || cudaEventElapsedTime(&t, p.a, p.b) != cudaSuccess) {
+      rc = HISA_ERR_CUDA;
+    } else if (p.kind >= 0 && p.kind < K_NUM_KINDS) {
+      g_ms[p.kind] += t;
+      g_timed[p.kind]++;
+    }
+    g_free_events.push_back(p.a);
+    g_free_events.push_back(p.b);
+  }
+  g_pending.clear();
+  for (int i = 0; i < n && i < K_NUM_KINDS; i++) {
+    if (ms) ms[i] = g_ms[i];
+    if (launches) launches[i] = g_launches[i];
+    if (timed) timed[i] = g_timed[i];
+  }
+  if (reset) {
+    for (int i = 0; i < K_NUM_KINDS; i++) {
+      g_ms[i] = 0.0;
+      g_launches[i] = 0;
+      g_timed[i] = 0;
+    }
+  }
+  return rc;
 }
 
 hisa_status hisa_device_status(int32_t *status, int clear, hisa_stream_t stream) {

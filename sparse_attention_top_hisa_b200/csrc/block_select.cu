@@ -12,6 +12,7 @@
 // finds the key of the (m - |forced|)-th best block; ballots over ascending
 // block numbers resolve ties and emit the selected blocks in ascending order.
 #include "common.cuh"
+#include "prof.cuh"
 
 namespace hisa {
 
@@ -136,15 +137,18 @@ cudaError_t launch_block_select(const uint16_t *q, const float *reps, const int3
   if (total_q == 0) return cudaSuccess;
   const int emax = (max_seqlen_k + BLK - 1) / BLK;
   const size_t smem = (size_t)BS_WARPS * (emax > 0 ? emax : 1) * sizeof(uint32_t);
+  static int attr[64];
   if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(block_select_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = set_smem_once((const void *)block_select_kernel, smem, attr);
     if (e != cudaSuccess) return e;
   }
   dim3 grid((total_q + BS_WARPS - 1) / BS_WARPS);
-  block_select_kernel<<<grid, BS_WARPS * 32, smem, st>>>(q, reps, cu_q, cu_k, seqlens, S, total_q,
-                                                       m, emax > 0 ? emax : 1, blk, out_blocks,
-                                                       status);
+  {
+    ProfScope ps(K_BLOCK_SELECT, st);
+    block_select_kernel<<<grid, BS_WARPS * 32, smem, st>>>(q, reps, cu_q, cu_k, seqlens, S,
+                                                         total_q, m, emax > 0 ? emax : 1, blk,
+                                                         out_blocks, status);
+  }
   return cudaGetLastError();
 }
 

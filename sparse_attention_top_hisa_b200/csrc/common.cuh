@@ -167,4 +167,15 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int *warp_tot, int *t
   return excl;
 }
 
+// Raise a kernel's dynamic shared-memory limit once per device; later calls (for
+// example while a CUDA graph is being captured) find it already set.
+inline cudaError_t set_smem_once(const void *func, size_t bytes, int *cache /*[64]*/) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
+  if (cache[dev] >= (int)bytes) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess) cache[dev] = (int)bytes;
+  return e;
+}
+
 }  // namespace hisa

@@ -18,6 +18,7 @@
 //   3. dsa_select_kernel: exact top-k of each candidate list (shared routine).
 //   4. dsa_fallback_kernel: a row whose list overflowed its capacity (many equal
 //      scores) is redone exactly from a full score row in scratch memory.
+#include "prof.cuh"
 #include "select.cuh"
 
 namespace hisa {
@@ -320,32 +321,37 @@ cudaError_t launch_dsa(const uint16_t *q, const uint16_t *k, const int32_t *cu_q
   cudaError_t e = cudaMemsetAsync(kmax, 0, (size_t)S * 4, st);
   if (e != cudaSuccess) return e;
   if (max_seqlen_k > 0) {
+    ProfScope ps(K_KEY_NORM, st);
     key_norm_kernel<<<dim3((max_seqlen_k + 255) / 256, S), 256, 0, st>>>(k, cu_k, seqlens, kmax);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   const size_t fsm = sizeof(DsaShared);
   const size_t ssm = dsa_select_smem(p.cap, topk);
   const size_t bsm = (size_t)16 * topk + sizeof(SelectShared);
-  if ((e = cudaFuncSetAttribute(dsa_filter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)fsm)) != cudaSuccess)
-    return e;
-  if ((e = cudaFuncSetAttribute(dsa_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)ssm)) != cudaSuccess)
-    return e;
-  if ((e = cudaFuncSetAttribute(dsa_fallback_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)bsm)) != cudaSuccess)
-    return e;
+  static int attr_f[64], attr_s[64], attr_b[64];
+  if ((e = set_smem_once((const void *)dsa_filter_kernel, fsm, attr_f)) != cudaSuccess) return e;
+  if ((e = set_smem_once((const void *)dsa_select_kernel, ssm, attr_s)) != cudaSuccess) return e;
+  if ((e = set_smem_once((const void *)dsa_fallback_kernel, bsm, attr_b)) != cudaSuccess) return e;
   for (int row0 = 0; row0 < total_q; row0 += p.chunk) {
     const int nrows = min(p.chunk, total_q - row0);
-    dsa_filter_kernel<<<(nrows + DSA_Q - 1) / DSA_Q, DSA_Q, fsm, st>>>(
-        q, k, cu_q, cu_k, seqlens, S, row0, nrows, topk, p.cap, kmax, bkey, bj, cnt, status);
+    {
+      ProfScope ps(K_DSA_FILTER, st);
+      dsa_filter_kernel<<<(nrows + DSA_Q - 1) / DSA_Q, DSA_Q, fsm, st>>>(
+          q, k, cu_q, cu_k, seqlens, S, row0, nrows, topk, p.cap, kmax, bkey, bj, cnt, status);
+    }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    dsa_select_kernel<<<nrows, DSA_SEL_THREADS, ssm, st>>>(row0, topk, p.cap, bkey, bj, cnt,
-                                                            out_idx, out_scores);
+    {
+      ProfScope ps(K_DSA_SELECT, st);
+      dsa_select_kernel<<<nrows, DSA_SEL_THREADS, ssm, st>>>(row0, topk, p.cap, bkey, bj, cnt,
+                                                              out_idx, out_scores);
+    }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    dsa_fallback_kernel<<<DSA_FB_CTAS, DSA_SEL_THREADS, bsm, st>>>(
-        q, k, cu_q, cu_k, seqlens, S, row0, nrows, topk, p.cap, cnt, fb,
-        (size_t)(max_seqlen_k > 0 ? max_seqlen_k : 1), out_idx, out_scores, status);
+    {
+      ProfScope ps(K_DSA_FALLBACK, st);
+      dsa_fallback_kernel<<<DSA_FB_CTAS, DSA_SEL_THREADS, bsm, st>>>(
+          q, k, cu_q, cu_k, seqlens, S, row0, nrows, topk, p.cap, cnt, fb,
+          (size_t)(max_seqlen_k > 0 ? max_seqlen_k : 1), out_idx, out_scores, status);
+    }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   return cudaSuccess;

@@ -7,6 +7,7 @@
 // increasing row order in fp32, then one correctly rounded division by the count),
 // so incrementally maintained representatives equal a fresh pool bit for bit.
 #include "common.cuh"
+#include "prof.cuh"
 
 namespace hisa {
 
@@ -102,7 +103,10 @@ cudaError_t launch_pool(const uint16_t *k, const int32_t *cu_k, const int32_t *s
   const int nblk = (max_seqlen_k + BLK - 1) / BLK;
   if (nblk == 0 || num_seqs == 0) return cudaSuccess;
   dim3 grid((nblk + POOL_WARPS - 1) / POOL_WARPS, num_seqs);
-  pool_blocks_kernel<<<grid, POOL_WARPS * 32, 0, st>>>(k, cu_k, seqlens, reps, status);
+  {
+    ProfScope ps(K_POOL, st);
+    pool_blocks_kernel<<<grid, POOL_WARPS * 32, 0, st>>>(k, cu_k, seqlens, reps, status);
+  }
   return cudaGetLastError();
 }
 
@@ -110,7 +114,11 @@ cudaError_t launch_append(uint16_t *kc, float *reps, const int32_t *cu_k, int32_
                           const uint16_t *new_keys, int n_new, int num_seqs, int *status,
                           cudaStream_t st) {
   if (num_seqs == 0 || n_new == 0) return cudaSuccess;
-  append_keys_kernel<<<num_seqs, 128, 0, st>>>(kc, reps, cu_k, seqlens, new_keys, n_new, status);
+  {
+    ProfScope ps(K_APPEND, st);
+    append_keys_kernel<<<num_seqs, 128, 0, st>>>(kc, reps, cu_k, seqlens, new_keys, n_new,
+                                                 status);
+  }
   return cudaGetLastError();
 }
 

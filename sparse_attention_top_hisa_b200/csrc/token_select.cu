@@ -15,6 +15,7 @@
 //     row without bank conflicts), scores them into shared memory and selects;
 //   * split: for few queries (decode) the blocks of each query are scored by
 //     several CTAs into a global scratch row, then one CTA per query selects.
+#include "prof.cuh"
 #include "select.cuh"
 
 namespace hisa {
@@ -201,22 +202,31 @@ cudaError_t launch_token_select(const uint16_t *q, const uint16_t *k, const int3
     int slots = (m + splits - 1) / splits;
     slots = (slots + 1) & ~1;  // whole staging rounds
     splits = (m + slots - 1) / slots;
-    token_score_split_kernel<<<dim3(total_q, splits), TS_THREADS, 0, st>>>(
-        q, k, cu_q, cu_k, seqlens, S, m, blk, slots, scratch);
+    {
+      ProfScope ps(K_TOKEN_SCORE_SPLIT, st);
+      token_score_split_kernel<<<dim3(total_q, splits), TS_THREADS, 0, st>>>(
+          q, k, cu_q, cu_k, seqlens, S, m, blk, slots, scratch);
+    }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(token_select_scratch_kernel,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    static int attr_sel[64];
+    e = set_smem_once((const void *)token_select_scratch_kernel, smem, attr_sel);
     if (e != cudaSuccess) return e;
-    token_select_scratch_kernel<<<total_q, TS_THREADS, smem, st>>>(
-        cu_q, cu_k, seqlens, S, m, topk, blk, scratch, out_idx, out_scores);
+    {
+      ProfScope ps(K_TOKEN_SELECT_SCRATCH, st);
+      token_select_scratch_kernel<<<total_q, TS_THREADS, smem, st>>>(
+          cu_q, cu_k, seqlens, S, m, topk, blk, scratch, out_idx, out_scores);
+    }
     return cudaGetLastError();
   }
-  cudaError_t e = cudaFuncSetAttribute(token_fused_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  static int attr_fused[64];
+  cudaError_t e = set_smem_once((const void *)token_fused_kernel, smem, attr_fused);
   if (e != cudaSuccess) return e;
-  token_fused_kernel<<<total_q, TS_THREADS, smem, st>>>(q, k, cu_q, cu_k, seqlens, S, m, topk,
-                                                        blk, out_idx, out_scores, status);
+  {
+    ProfScope ps(K_TOKEN_FUSED, st);
+    token_fused_kernel<<<total_q, TS_THREADS, smem, st>>>(q, k, cu_q, cu_k, seqlens, S, m, topk,
+                                                          blk, out_idx, out_scores, status);
+  }
   return cudaGetLastError();
 }
 
