@@ -203,6 +203,41 @@ size_t dsa_flat_workspace_size(int total_q, int num_seqs, int max_seqlen_k, int 
 hisa_status hisa_device_status(int32_t *status, int clear, hisa_stream_t stream);
 
 /*
+ * hisa_select_noalloc — hisa_select without a workspace (the pages have no
+ * counterpart; it exists for callers of this library that cannot allocate).
+ *
+ * Some callers cannot allocate device memory at the moment they need a
+ * selection: a plug-in running inside an inference engine whose memory plan is
+ * fixed before it starts, or a latency-critical decode path where a cudaMalloc
+ * would synchronise the device.  This entry point takes the same arguments and
+ * produces the same outputs as hisa_select, minus ws/ws_bytes: its scratch is a
+ * fixed array of HISA_NOALLOC_SCRATCH_BYTES bytes inside the library.  It calls
+ * no cudaMalloc, cudaFree or other allocating routine.
+ *
+ *   - The array exists once per device and every device that loads the library
+ *     holds it until the process exits.
+ *   - Problems whose scratch exceeds HISA_NOALLOC_SCRATCH_BYTES are rejected with
+ *     HISA_ERR_WORKSPACE before anything is launched.  The scratch needed equals
+ *     hisa_select_workspace_size() for the same arguments; at m = 64 every batch
+ *     of up to 65536 queries fits.
+ *   - Every call shares the array and it keeps the last call's contents; nothing
+ *     in it needs to start at zero.  Calls whose kernels overlap on the GPU (on
+ *     different streams, or from different host threads) race on the array and
+ *     give wrong results: order them on one stream or serialise them.
+ *   - The first call on a device looks up the array's device address (once per
+ *     device, with that device current); make that first call before any stream
+ *     capture.
+ *   - Inputs, outputs, ordering, errors and the device status word are those of
+ *     hisa_select.
+ */
+#define HISA_NOALLOC_SCRATCH_BYTES (16u << 20)
+hisa_status hisa_select_noalloc(const hisa_bf16 *q_idx, const hisa_bf16 *k_idx, const float *reps,
+                                const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
+                                const int32_t *seqlens_k, int num_seqs, int total_q,
+                                int max_seqlen_k, int B, int m, int k, int32_t *out_idx,
+                                float *out_scores, int32_t *out_blocks, hisa_stream_t stream);
+
+/*
  * Launch accounting, for benchmarks and tests (no counterpart on the pages).
  * Every kernel launch made by this library is counted per kernel kind.  With
  * timing enabled, each launch is also bracketed by a pair of CUDA events

@@ -50,6 +50,7 @@ EXPORTED = (
     "hisa_kernel_kinds",
     "hisa_kernel_name",
     "hisa_timing_collect",
+    "hisa_select_noalloc",
 )
 
 

@@ -321,3 +321,68 @@ hisa_status hisa_device_status(int32_t *status, int clear, hisa_stream_t stream)
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// hisa_select_noalloc: hisa_select for callers that cannot allocate device memory
+// when they need a selection (for example a plug-in inside an inference engine
+// whose memory plan is fixed before it runs, or a latency-critical path where a
+// cudaMalloc would synchronise the device).  Its scratch is a fixed array inside
+// this library instead of a caller workspace.
+
+// Every device that loads the library holds this array until the process exits.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[HISA_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+uint8_t *g_noalloc_ptr[kMaxDevices];
+
+// Device address of the scratch array on the current device.  Host code only has a
+// host-side stand-in for the symbol, so the address is looked up once per device
+// (with that device current) and cached.
+uint8_t *noalloc_scratch() {
+  const int dev = current_device();
+  if (dev < 0) return nullptr;
+  if (!g_noalloc_ptr[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return nullptr;
+    g_noalloc_ptr[dev] = static_cast<uint8_t *>(p);
+  }
+  return g_noalloc_ptr[dev];
+}
+}  // namespace
+
+extern "C" hisa_status hisa_select_noalloc(const hisa_bf16 *q_idx, const hisa_bf16 *k_idx,
+                                           const float *reps, const int32_t *cu_seqlens_q,
+                                           const int32_t *cu_seqlens_k, const int32_t *seqlens_k,
+                                           int num_seqs, int total_q, int max_seqlen_k, int B,
+                                           int m, int k, int32_t *out_idx, float *out_scores,
+                                           int32_t *out_blocks, hisa_stream_t stream) {
+  if (B != HISA_BLOCK || m < 1 || m > HISA_MAX_M || k < 1 || k > HISA_MAX_TOPK)
+    return HISA_ERR_INVALID_ARG;
+  if (num_seqs < 0 || total_q < 0 || max_seqlen_k < 0) return HISA_ERR_INVALID_ARG;
+  if (total_q == 0) return HISA_OK;
+  if (num_seqs == 0) return HISA_ERR_INVALID_ARG;
+  if (!q_idx || !k_idx || !reps || !cu_seqlens_q || !cu_seqlens_k || !out_idx)
+    return HISA_ERR_INVALID_ARG;
+  if (!aligned(q_idx, 16) || !aligned(k_idx, 16) || !aligned(reps, 16) ||
+      !aligned(cu_seqlens_q, 4) || !aligned(cu_seqlens_k, 4) || !aligned(seqlens_k, 4) ||
+      !aligned(out_idx, 4) || !aligned(out_scores, 4) || !aligned(out_blocks, 4))
+    return HISA_ERR_UNALIGNED;
+  // the same scratch layout hisa_select carves from its workspace must fit the array
+  const SelectPlan p = select_plan(total_q, m);
+  if (p.total > (size_t)HISA_NOALLOC_SCRATCH_BYTES) return HISA_ERR_WORKSPACE;
+  uint8_t *w = noalloc_scratch();
+  if (!w) return HISA_ERR_CUDA;
+  int *st = status_word();
+  if (!st) return HISA_ERR_CUDA;
+  // Nothing in the scratch has to start at zero: the block lists are written in full by
+  // the block stage and every score row is written before it is read.
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int32_t *blk = reinterpret_cast<int32_t *>(w + p.off_blk);
+  uint32_t *scratch = reinterpret_cast<uint32_t *>(w + p.off_scratch);
+  cudaError_t e = launch_block_select(q_idx, reps, cu_seqlens_q, cu_seqlens_k, seqlens_k,
+                                      num_seqs, total_q, max_seqlen_k, m, blk, out_blocks, st, s);
+  if (e != cudaSuccess) return HISA_ERR_CUDA;
+  e = launch_token_select(q_idx, k_idx, cu_seqlens_q, cu_seqlens_k, seqlens_k, num_seqs, total_q,
+                          m, k, blk, scratch, num_sms(), out_idx, out_scores, st, s);
+  return from_cuda(e);
+}
