@@ -218,8 +218,9 @@ hisa_status hisa_device_status(int32_t *status, int clear, hisa_stream_t stream)
  *     holds it until the process exits.
  *   - Problems whose scratch exceeds HISA_NOALLOC_SCRATCH_BYTES are rejected with
  *     HISA_ERR_WORKSPACE before anything is launched.  The scratch needed equals
- *     hisa_select_workspace_size() for the same arguments; at m = 64 every batch
- *     of up to 65536 queries fits.
+ *     hisa_select_workspace_size() for the same arguments (about m * 516 bytes per
+ *     query); at m = 64 every batch of up to 500 queries fits, which covers decode
+ *     batches.
  *   - Every call shares the array and it keeps the last call's contents; nothing
  *     in it needs to start at zero.  Calls whose kernels overlap on the GPU (on
  *     different streams, or from different host threads) race on the array and

@@ -22,10 +22,10 @@ cudaError_t launch_block_select(const uint16_t *q, const float *reps, const int3
                                 int32_t *out_blocks, int *status, cudaStream_t st);
 cudaError_t launch_token_select(const uint16_t *q, const uint16_t *k, const int32_t *cu_q,
                                 const int32_t *cu_k, const int32_t *seqlens, int S, int total_q,
-                                int m, int topk, const int32_t *blk, uint32_t *scratch,
-                                int num_sms, int32_t *out_idx, float *out_scores, int *status,
-                                cudaStream_t st);
-size_t token_scratch_bytes(int total_q, int m, int num_sms);
+                                int max_seqlen_k, int m, int topk, const int32_t *blk,
+                                uint8_t *ws, int num_sms, int32_t *out_idx, float *out_scores,
+                                int *status, cudaStream_t st);
+size_t token_scratch_bytes(int total_q, int num_seqs, int max_seqlen_k, int m, int num_sms);
 cudaError_t launch_dsa(const uint16_t *q, const uint16_t *k, const int32_t *cu_q,
                        const int32_t *cu_k, const int32_t *seqlens, int S, int total_q,
                        int max_seqlen_k, int topk, int32_t *out_idx, float *out_scores,
@@ -42,7 +42,8 @@ namespace {
 const char *kKindNames[K_NUM_KINDS] = {
     "pool_blocks",        "append_keys",         "block_select",   "token_fused",
     "token_score_split",  "token_select_scratch", "key_norm",      "dsa_filter",
-    "dsa_select",         "dsa_fallback"};
+    "dsa_select",         "dsa_fallback",         "inv_lists",      "inv_scan",
+    "token_score_tc"};
 long long g_launches[K_NUM_KINDS];
 double g_ms[K_NUM_KINDS];
 long long g_timed[K_NUM_KINDS];
@@ -133,13 +134,13 @@ struct SelectPlan {
   size_t off_blk, off_scratch, total;
 };
 
-SelectPlan select_plan(int total_q, int m) {
+SelectPlan select_plan(int total_q, int num_seqs, int max_seqlen_k, int m) {
   SelectPlan p;
   size_t off = 0;
   p.off_blk = off;
   off = align256(off + (size_t)(total_q > 0 ? total_q : 1) * m * 4);
   p.off_scratch = off;
-  off = align256(off + token_scratch_bytes(total_q, m, num_sms()));
+  off = align256(off + token_scratch_bytes(total_q, num_seqs, max_seqlen_k, m, num_sms()));
   p.total = off;
   return p;
 }
@@ -196,12 +197,10 @@ hisa_status hisa_append_keys(hisa_bf16 *k_cache, float *reps, const int32_t *cu_
 
 size_t hisa_select_workspace_size(int total_q, int num_seqs, int max_seqlen_k, int B, int m,
                                   int k) {
-  (void)num_seqs;
-  (void)max_seqlen_k;
   (void)B;
   (void)k;
-  if (total_q < 0 || m < 1) return 0;
-  return select_plan(total_q, m).total;
+  if (total_q < 0 || m < 1 || num_seqs < 0 || max_seqlen_k < 0) return 0;
+  return select_plan(total_q, num_seqs, max_seqlen_k, m).total;
 }
 
 hisa_status hisa_select(const hisa_bf16 *q_idx, const hisa_bf16 *k_idx, const float *reps,
@@ -220,7 +219,8 @@ hisa_status hisa_select(const hisa_bf16 *q_idx, const hisa_bf16 *k_idx, const fl
       !aligned(cu_seqlens_q, 4) || !aligned(cu_seqlens_k, 4) || !aligned(seqlens_k, 4) ||
       !aligned(out_idx, 4) || !aligned(out_scores, 4) || !aligned(out_blocks, 4))
     return HISA_ERR_UNALIGNED;
-  const SelectPlan p = select_plan(total_q, m);
+  if (total_q >= (1 << 25)) return HISA_ERR_INVALID_ARG;
+  const SelectPlan p = select_plan(total_q, num_seqs, max_seqlen_k, m);
   if (!ws || ws_bytes < p.total) return HISA_ERR_WORKSPACE;
   if (!aligned(ws, 256)) return HISA_ERR_UNALIGNED;
   int *st = status_word();
@@ -228,12 +228,12 @@ hisa_status hisa_select(const hisa_bf16 *q_idx, const hisa_bf16 *k_idx, const fl
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t *w = static_cast<uint8_t *>(ws);
   int32_t *blk = reinterpret_cast<int32_t *>(w + p.off_blk);
-  uint32_t *scratch = reinterpret_cast<uint32_t *>(w + p.off_scratch);
   cudaError_t e = launch_block_select(q_idx, reps, cu_seqlens_q, cu_seqlens_k, seqlens_k,
                                       num_seqs, total_q, max_seqlen_k, m, blk, out_blocks, st, s);
   if (e != cudaSuccess) return HISA_ERR_CUDA;
   e = launch_token_select(q_idx, k_idx, cu_seqlens_q, cu_seqlens_k, seqlens_k, num_seqs, total_q,
-                          m, k, blk, scratch, num_sms(), out_idx, out_scores, st, s);
+                          max_seqlen_k, m, k, blk, w + p.off_scratch, num_sms(), out_idx,
+                          out_scores, st, s);
   return from_cuda(e);
 }
 
@@ -368,7 +368,8 @@ extern "C" hisa_status hisa_select_noalloc(const hisa_bf16 *q_idx, const hisa_bf
       !aligned(out_idx, 4) || !aligned(out_scores, 4) || !aligned(out_blocks, 4))
     return HISA_ERR_UNALIGNED;
   // the same scratch layout hisa_select carves from its workspace must fit the array
-  const SelectPlan p = select_plan(total_q, m);
+  if (total_q >= (1 << 25)) return HISA_ERR_INVALID_ARG;
+  const SelectPlan p = select_plan(total_q, num_seqs, max_seqlen_k, m);
   if (p.total > (size_t)HISA_NOALLOC_SCRATCH_BYTES) return HISA_ERR_WORKSPACE;
   uint8_t *w = noalloc_scratch();
   if (!w) return HISA_ERR_CUDA;
@@ -378,11 +379,11 @@ extern "C" hisa_status hisa_select_noalloc(const hisa_bf16 *q_idx, const hisa_bf
   // the block stage and every score row is written before it is read.
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int32_t *blk = reinterpret_cast<int32_t *>(w + p.off_blk);
-  uint32_t *scratch = reinterpret_cast<uint32_t *>(w + p.off_scratch);
   cudaError_t e = launch_block_select(q_idx, reps, cu_seqlens_q, cu_seqlens_k, seqlens_k,
                                       num_seqs, total_q, max_seqlen_k, m, blk, out_blocks, st, s);
   if (e != cudaSuccess) return HISA_ERR_CUDA;
   e = launch_token_select(q_idx, k_idx, cu_seqlens_q, cu_seqlens_k, seqlens_k, num_seqs, total_q,
-                          m, k, blk, scratch, num_sms(), out_idx, out_scores, st, s);
+                          max_seqlen_k, m, k, blk, w + p.off_scratch, num_sms(), out_idx,
+                          out_scores, st, s);
   return from_cuda(e);
 }

@@ -18,6 +18,9 @@ enum KernelKind {
   K_DSA_FILTER,
   K_DSA_SELECT,
   K_DSA_FALLBACK,
+  K_INV_LISTS,
+  K_INV_SCAN,
+  K_TOKEN_SCORE_TC,
   K_NUM_KINDS
 };
 

@@ -9,12 +9,13 @@
 // sequence; blocks are listed in ascending order, so candidate order is token
 // order.  The token causal mask admits j <= i.
 //
-// Two schedules share the scoring and selection code:
-//   * fused: one CTA per query stages its selected blocks through shared memory
-//     (cp.async, XOR-swizzled 16-byte chunks so that each thread reads its own key
-//     row without bank conflicts), scores them into shared memory and selects;
-//   * split: for few queries (decode) the blocks of each query are scored by
-//     several CTAs into a global scratch row, then one CTA per query selects.
+// Two schedules produce each query's score row (order-preserving keys, candidate
+// order) in workspace memory; one CTA per query then selects from it:
+//   * many queries (prefill): the block-major tensor-core path of token_tc.cu;
+//   * few queries (decode): the selected blocks of each query are split over several
+//     CTAs that stage them through shared memory (cp.async, XOR-swizzled 16-byte
+//     chunks, so each thread reads its own key row without bank conflicts) and score
+//     them on the CUDA cores -- a memory-bound stream with no reuse to exploit.
 #include "prof.cuh"
 #include "select.cuh"
 
@@ -100,37 +101,6 @@ __host__ __device__ inline size_t token_smem_bytes(int m, int topk) {
 }
 
 __global__ void __launch_bounds__(TS_THREADS)
-token_fused_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ k,
-                   const int32_t *__restrict__ cu_q, const int32_t *__restrict__ cu_k,
-                   const int32_t *__restrict__ seqlens, int S, int m, int topk,
-                   const int32_t *__restrict__ blk, int32_t *__restrict__ out_idx,
-                   float *__restrict__ out_scores, int *status) {
-  extern __shared__ __align__(16) uint8_t smem[];
-  uint32_t *keys = reinterpret_cast<uint32_t *>(smem);
-  uint8_t *stage = smem + (size_t)m * BLK * 4;
-  SelectShared &sh = *reinterpret_cast<SelectShared *>(stage + stage_bytes(topk));
-  const int row = blockIdx.x;
-  RowPad pad{out_idx + (size_t)row * topk, out_scores ? out_scores + (size_t)row * topk : nullptr};
-  const QueryInfo qi = locate(cu_q, cu_k, seqlens, S, row, nullptr);
-  if (!qi.ok) {  // already reported by the block stage
-    for (int r = threadIdx.x; r < topk; r += TS_THREADS) pad(r);
-    return;
-  }
-  const int32_t *blkrow = blk + (size_t)row * m;
-  const int nsel = count_selected(blkrow, m);
-  QRegs qr;
-  load_q(qr, q + (size_t)row * D);
-  score_slots(qr, k + (size_t)qi.kbase * D, qi.pos, blkrow, 0, nsel, stage,
-              [&](int c, uint32_t key) { keys[c] = key; });
-  uint32_t *sel_key = reinterpret_cast<uint32_t *>(stage);
-  int *sel_c = reinterpret_cast<int *>(stage + (size_t)4 * topk);
-  uint32_t *tmp_key = reinterpret_cast<uint32_t *>(stage + (size_t)8 * topk);
-  int *tmp_c = reinterpret_cast<int *>(stage + (size_t)12 * topk);
-  TokenOut out{pad.idx, pad.scores, blkrow};
-  select_topk<TS_THREADS>(keys, nsel * BLK, topk, sh, sel_key, sel_c, tmp_key, tmp_c, out, pad);
-}
-
-__global__ void __launch_bounds__(TS_THREADS)
 token_score_split_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ k,
                          const int32_t *__restrict__ cu_q, const int32_t *__restrict__ cu_k,
                          const int32_t *__restrict__ seqlens, int S, int m,
@@ -181,20 +151,29 @@ token_select_scratch_kernel(const int32_t *__restrict__ cu_q, const int32_t *__r
   select_topk<TS_THREADS>(keys, nsel * BLK, topk, sh, sel_key, sel_c, tmp_key, tmp_c, out, pad);
 }
 
-// Split schedule when there are too few queries to fill the GPU with one CTA each.
+// Split schedule when there are too few queries to fill the GPU with tensor-core tiles.
 bool token_use_split(int total_q, int num_sms) { return total_q < 2 * num_sms; }
 
-size_t token_scratch_bytes(int total_q, int m, int num_sms) {
-  return token_use_split(total_q, num_sms) ? (size_t)total_q * m * BLK * 4 : 0;
+size_t tc_workspace_bytes(int total_q, int num_seqs, int max_seqlen_k, int m);
+cudaError_t launch_token_score_tc(const uint16_t *q, const uint16_t *k, const int32_t *cu_q,
+                                  const int32_t *cu_k, const int32_t *seqlens, int S,
+                                  int total_q, int max_seqlen_k, int m, const int32_t *blk,
+                                  uint8_t *ws, uint32_t **scores_out, int num_sms, int *status,
+                                  cudaStream_t st);
+
+size_t token_scratch_bytes(int total_q, int num_seqs, int max_seqlen_k, int m, int num_sms) {
+  if (token_use_split(total_q, num_sms)) return (size_t)total_q * m * BLK * 4;
+  return tc_workspace_bytes(total_q, num_seqs, max_seqlen_k, m);
 }
 
 cudaError_t launch_token_select(const uint16_t *q, const uint16_t *k, const int32_t *cu_q,
                                 const int32_t *cu_k, const int32_t *seqlens, int S, int total_q,
-                                int m, int topk, const int32_t *blk, uint32_t *scratch,
-                                int num_sms, int32_t *out_idx, float *out_scores, int *status,
-                                cudaStream_t st) {
+                                int max_seqlen_k, int m, int topk, const int32_t *blk,
+                                uint8_t *ws, int num_sms, int32_t *out_idx, float *out_scores,
+                                int *status, cudaStream_t st) {
   if (total_q == 0) return cudaSuccess;
-  const size_t smem = token_smem_bytes(m, topk);
+  cudaError_t e;
+  uint32_t *scores = reinterpret_cast<uint32_t *>(ws);
   if (token_use_split(total_q, num_sms)) {
     // spread each query's blocks over enough CTAs to cover the SMs about twice
     int splits = (2 * num_sms + total_q - 1) / total_q;
@@ -205,27 +184,22 @@ cudaError_t launch_token_select(const uint16_t *q, const uint16_t *k, const int3
     {
       ProfScope ps(K_TOKEN_SCORE_SPLIT, st);
       token_score_split_kernel<<<dim3(total_q, splits), TS_THREADS, 0, st>>>(
-          q, k, cu_q, cu_k, seqlens, S, m, blk, slots, scratch);
+          q, k, cu_q, cu_k, seqlens, S, m, blk, slots, scores);
     }
-    cudaError_t e = cudaGetLastError();
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  } else {
+    e = launch_token_score_tc(q, k, cu_q, cu_k, seqlens, S, total_q, max_seqlen_k, m, blk, ws,
+                              &scores, num_sms, status, st);
     if (e != cudaSuccess) return e;
-    static int attr_sel[64];
-    e = set_smem_once((const void *)token_select_scratch_kernel, smem, attr_sel);
-    if (e != cudaSuccess) return e;
-    {
-      ProfScope ps(K_TOKEN_SELECT_SCRATCH, st);
-      token_select_scratch_kernel<<<total_q, TS_THREADS, smem, st>>>(
-          cu_q, cu_k, seqlens, S, m, topk, blk, scratch, out_idx, out_scores);
-    }
-    return cudaGetLastError();
   }
-  static int attr_fused[64];
-  cudaError_t e = set_smem_once((const void *)token_fused_kernel, smem, attr_fused);
-  if (e != cudaSuccess) return e;
+  const size_t smem = token_smem_bytes(m, topk);
+  static int attr_sel[64];
+  if ((e = set_smem_once((const void *)token_select_scratch_kernel, smem, attr_sel)) != cudaSuccess)
+    return e;
   {
-    ProfScope ps(K_TOKEN_FUSED, st);
-    token_fused_kernel<<<total_q, TS_THREADS, smem, st>>>(q, k, cu_q, cu_k, seqlens, S, m, topk,
-                                                          blk, out_idx, out_scores, status);
+    ProfScope ps(K_TOKEN_SELECT_SCRATCH, st);
+    token_select_scratch_kernel<<<total_q, TS_THREADS, smem, st>>>(
+        cu_q, cu_k, seqlens, S, m, topk, blk, scores, out_idx, out_scores);
   }
   return cudaGetLastError();
 }

@@ -1,0 +1,335 @@
+// Stage 2 of HISA on the tensor cores: block-major gather-scoring.
+//
+// HISA summary page (aitrends.kr), paragraph on stage 2: every query scores the
+// tokens of its m selected blocks with the original DSA dot product.  Grouped by
+// key block instead of by query, this is a dense contraction: for key block b and
+// the queries that selected it, S = K_b [128 x 64] . Q_sel^T [64 x N].  Each key
+// block then crosses the memory hierarchy once per 256 selecting queries instead of
+// once per query.
+//
+//   1. inv_lists_kernel (count, then fill): the (query, slot) pairs are bucketed by
+//      key block, with warp-aggregated atomics (block 0 is selected by every query);
+//   2. inv_scan_kernel: list offsets per key block and tile descriptors (one tile =
+//      one key block and up to 256 of its selecting queries);
+//   3. token_score_tc_kernel: persistent CTAs; per tile the key block arrives by TMA
+//      (or by guarded cp.async when it is the partial last block of a sequence), the
+//      selecting queries are gathered with cp.async into the 128-byte-swizzled
+//      K-major layout, one thread issues four tcgen05.mma (K = 4 x 16) into a
+//      128 x N fp32 accumulator in TMEM, and four warps move it out (warp w owns
+//      TMEM lanes 32w..32w+31, i.e. key rows) into each query's score row;
+//   4. the exact select of token_select.cu reads the score rows.
+// Key j of block b is admitted for a query at position i only when j <= i.
+#include <cudaTypedefs.h>
+
+#include "prof.cuh"
+#include "tc.cuh"
+
+namespace hisa {
+
+constexpr int TC_N = 256;          // selecting queries per tile (MMA N, at most)
+constexpr int TC_THREADS = 128;    // four warps, one TMEM lane quarter each
+constexpr uint32_t TC_TMEM_COLS = 256;
+
+struct TileDesc {
+  int list_off;  // first list entry of the tile
+  int cb;        // compact key block: sequence * emax + block
+  int n;         // entries in the tile (1..TC_N)
+  int pad;
+};
+
+struct TcSmem {
+  uint8_t a[BLK * ROW_BYTES];   // key block, 1024-byte aligned
+  uint8_t b[TC_N * ROW_BYTES];  // gathered queries, 1024-byte aligned
+  uint32_t ent[TC_N];
+  uint64_t bar_tma;
+  uint64_t bar_mma;
+  uint32_t tmem_base;
+};
+// request enough shared memory that at most two CTAs share an SM (2 x 256 TMEM columns)
+constexpr size_t TC_SMEM_BYTES = 110 * 1024;
+static_assert(sizeof(TcSmem) + 1024 <= TC_SMEM_BYTES, "tile does not fit");
+
+// ---------------------------------------------------------------------------
+// inverted lists
+
+// mode 0: count pairs per compact key block; mode 1: write them into the lists.
+__global__ void __launch_bounds__(256)
+inv_lists_kernel(const int32_t *__restrict__ blk, int total_q, int m,
+                 const int32_t *__restrict__ cu_q, int S, int emax, int mode,
+                 int *__restrict__ cnt, int *__restrict__ cursor, uint32_t *__restrict__ list) {
+  const int lane = threadIdx.x & 31;
+  const int row = ((blockIdx.x * blockDim.x + threadIdx.x) >> 5) * 32 + lane;
+  const bool valid = row < total_q;
+  const int s = valid ? find_seq(cu_q, S, row) : 0;
+  const unsigned lt = (1u << lane) - 1u;
+  for (int slot = 0; slot < m; slot++) {
+    const int b = valid ? __ldg(blk + (size_t)row * m + slot) : -1;
+    const int key = b >= 0 ? s * emax + b : -1;
+    const unsigned peers = __match_any_sync(0xffffffffu, key);
+    const int leader = __ffs(peers) - 1;
+    if (mode == 0) {
+      if (key >= 0 && lane == leader) atomicAdd(cnt + key, __popc(peers));
+    } else {
+      int base = 0;
+      if (key >= 0 && lane == leader) base = atomicAdd(cursor + key, __popc(peers));
+      base = __shfl_sync(0xffffffffu, base, leader);
+      if (key >= 0) list[base + __popc(peers & lt)] = ((uint32_t)row << 7) | (uint32_t)slot;
+    }
+  }
+}
+
+constexpr int SCAN_THREADS = 1024;
+
+__global__ void __launch_bounds__(SCAN_THREADS)
+inv_scan_kernel(const int *__restrict__ cnt, int nb, int *__restrict__ cursor,
+                TileDesc *__restrict__ tiles, int *__restrict__ ntiles) {
+  __shared__ int warp_tot[SCAN_THREADS / 32 + 1];
+  const int per = (nb + SCAN_THREADS - 1) / SCAN_THREADS;
+  const int b0 = threadIdx.x * per, b1 = min(nb, b0 + per);
+  int sc = 0, st = 0;
+  for (int i = b0; i < b1; i++) {
+    const int c = cnt[i];
+    sc += c;
+    st += (c + TC_N - 1) / TC_N;
+  }
+  int total_c, total_t;
+  int oc = block_exclusive_scan<SCAN_THREADS>(sc, warp_tot, &total_c);
+  int ot = block_exclusive_scan<SCAN_THREADS>(st, warp_tot, &total_t);
+  for (int i = b0; i < b1; i++) {
+    const int c = cnt[i];
+    cursor[i] = oc;
+    for (int t = 0; t * TC_N < c; t++) {
+      TileDesc d;
+      d.list_off = oc + t * TC_N;
+      d.cb = i;
+      d.n = min(TC_N, c - t * TC_N);
+      d.pad = 0;
+      tiles[ot++] = d;
+    }
+    oc += c;
+  }
+  if (threadIdx.x == 0) *ntiles = total_t;
+}
+
+// ---------------------------------------------------------------------------
+// tensor-core scoring
+
+__global__ void __launch_bounds__(TC_THREADS, 1)
+token_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const uint16_t *__restrict__ q,
+                      const uint16_t *__restrict__ k, const int32_t *__restrict__ cu_q,
+                      const int32_t *__restrict__ cu_k, const int32_t *__restrict__ seqlens,
+                      int emax, int m, const TileDesc *__restrict__ tiles,
+                      const int *__restrict__ ntiles_ptr, const uint32_t *__restrict__ list,
+                      uint32_t *__restrict__ scratch, int *status) {
+  extern __shared__ uint8_t tc_smem_raw[];
+  TcSmem &sm = *reinterpret_cast<TcSmem *>((reinterpret_cast<uintptr_t>(tc_smem_raw) + 1023) &
+                                           ~(uintptr_t)1023);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) {
+    mbar_init(&sm.bar_tma, 1);
+    mbar_init(&sm.bar_mma, 1);
+    fence_barrier_init();
+    prefetch_tmap(&kmap);
+  }
+  if (warp == 0) {
+    tmem_alloc(&sm.tmem_base, TC_TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  const uint32_t sa = smem_u32(sm.a), sb = smem_u32(sm.b);
+  const int ntiles = *ntiles_ptr;
+  const size_t row_stride = (size_t)m * BLK;
+  uint32_t phase = 0;
+  for (int t = blockIdx.x; t < ntiles; t += gridDim.x, phase ^= 1u) {
+    const TileDesc td = tiles[t];
+    const int s = td.cb / emax, b = td.cb - (td.cb / emax) * emax;
+    const int kbase = __ldg(cu_k + s);
+    const int len = seqlens ? __ldg(seqlens + s) : __ldg(cu_k + s + 1) - kbase;
+    const int q0 = __ldg(cu_q + s);
+    const int pos_off = len - (__ldg(cu_q + s + 1) - q0) - q0;  // position = row + pos_off
+    const int n = td.n;
+    const int npad = (n + 15) & ~15;
+    for (int i = tid; i < n; i += TC_THREADS) sm.ent[i] = list[td.list_off + i];
+    __syncthreads();
+    // key block
+    const int live = len - b * BLK;
+    if (live >= BLK) {
+      if (tid == 0) {
+        mbar_arrive_expect_tx(&sm.bar_tma, BLK * ROW_BYTES);
+        tma_load_2d(sm.a, &kmap, &sm.bar_tma, 0, kbase + b * BLK);
+      }
+    } else {  // partial last block: load only the rows that exist
+      for (int i = tid; i < BLK * 8; i += TC_THREADS) {
+        const int r = i >> 3, c = i & 7;
+        if (r < live)
+          cp_async_16(sa + sw128_offset(r, c), k + (size_t)(kbase + b * BLK + r) * D + c * 8);
+        else
+          *reinterpret_cast<uint4 *>(sm.a + sw128_offset(r, c)) = make_uint4(0u, 0u, 0u, 0u);
+      }
+      if (tid == 0) mbar_arrive(&sm.bar_tma);
+    }
+    // the queries that selected the block
+    for (int i = tid; i < npad * 8; i += TC_THREADS) {
+      const int r = i >> 3, c = i & 7;
+      if (r < n)
+        cp_async_16(sb + sw128_offset(r, c), q + (size_t)(sm.ent[r] >> 7) * D + c * 8);
+      else
+        *reinterpret_cast<uint4 *>(sm.b + sw128_offset(r, c)) = make_uint4(0u, 0u, 0u, 0u);
+    }
+    cp_async_wait_all();
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (tid == 0) {
+      mbar_wait(&sm.bar_tma, phase, status);
+      tc_fence_after();
+      const uint32_t id = idesc_bf16_f32(BLK, npad);
+#pragma unroll
+      for (int kk = 0; kk < 4; kk++)
+        umma_bf16(tmem, sdesc_k_sw128(sa + kk * 32), sdesc_k_sw128(sb + kk * 32), id, kk > 0);
+      umma_commit(&sm.bar_mma);
+    }
+    __syncwarp();
+    mbar_wait(&sm.bar_mma, phase, status);
+    tc_fence_after();
+    // epilogue: this thread owns key row r of the block
+    const int r = warp * 32 + lane;
+    const int j = b * BLK + r;
+    for (int c0 = 0; c0 < npad; c0 += 16) {
+      uint32_t v[16];
+      tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, v);
+      tmem_wait_ld();
+#pragma unroll
+      for (int u = 0; u < 16; u++) {
+        if (c0 + u < n) {
+          const uint32_t e = sm.ent[c0 + u];
+          const int row = (int)(e >> 7), slot = (int)(e & 127u);
+          const uint32_t key = (j <= row + pos_off) ? score_key(__uint_as_float(v[u])) : 0u;
+          scratch[(size_t)row * row_stride + (size_t)slot * BLK + r] = key;
+        }
+      }
+    }
+    tc_fence_before();
+    __syncthreads();
+  }
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, TC_TMEM_COLS);
+}
+
+// ---------------------------------------------------------------------------
+// host side
+
+static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult qr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &qr) ==
+            cudaSuccess &&
+        qr == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 2-D map over the key rows (64 bf16 = 128 bytes each), boxes of 128 rows, 128-byte
+// swizzle.  The row extent is left open: the kernel only asks for whole blocks that
+// lie inside a sequence's live keys.
+bool make_key_tensor_map(CUtensorMap *map, const uint16_t *k) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)1 << 31};
+  cuuint64_t strides[1] = {(cuuint64_t)ROW_BYTES};
+  cuuint32_t box[2] = {(cuuint32_t)D, (cuuint32_t)BLK};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t *>(k), dims,
+                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+struct TcPlan {
+  size_t off_cnt, off_cursor, off_ntiles, off_tiles, off_list, off_scores, total;
+  int nb, max_tiles;
+};
+
+static size_t a256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+TcPlan tc_plan(int total_q, int num_seqs, int max_seqlen_k, int m) {
+  TcPlan p;
+  const int emax = (max_seqlen_k + BLK - 1) / BLK;
+  p.nb = (num_seqs > 0 ? num_seqs : 1) * (emax > 0 ? emax : 1);
+  const long long pairs = (long long)total_q * m;
+  p.max_tiles = (int)(pairs / TC_N + p.nb + 1);
+  size_t off = 0;
+  p.off_cnt = off;
+  off = a256(off + (size_t)p.nb * 4);
+  p.off_cursor = off;
+  off = a256(off + (size_t)p.nb * 4);
+  p.off_ntiles = off;
+  off = a256(off + 4);
+  p.off_tiles = off;
+  off = a256(off + (size_t)p.max_tiles * sizeof(TileDesc));
+  p.off_list = off;
+  off = a256(off + (size_t)pairs * 4);
+  p.off_scores = off;
+  off = a256(off + (size_t)pairs * BLK * 4);
+  p.total = off;
+  return p;
+}
+
+size_t tc_workspace_bytes(int total_q, int num_seqs, int max_seqlen_k, int m) {
+  return tc_plan(total_q, num_seqs, max_seqlen_k, m).total;
+}
+
+// Scores every selected (query, block) pair into ws's score rows
+// ([total_q][m * 128] order-preserving keys), ready for the select kernel.
+cudaError_t launch_token_score_tc(const uint16_t *q, const uint16_t *k, const int32_t *cu_q,
+                                  const int32_t *cu_k, const int32_t *seqlens, int S,
+                                  int total_q, int max_seqlen_k, int m, const int32_t *blk,
+                                  uint8_t *ws, uint32_t **scores_out, int num_sms, int *status,
+                                  cudaStream_t st) {
+  const TcPlan p = tc_plan(total_q, S, max_seqlen_k, m);
+  const int emax = (max_seqlen_k + BLK - 1) / BLK;
+  int *cnt = reinterpret_cast<int *>(ws + p.off_cnt);
+  int *cursor = reinterpret_cast<int *>(ws + p.off_cursor);
+  int *ntiles = reinterpret_cast<int *>(ws + p.off_ntiles);
+  TileDesc *tiles = reinterpret_cast<TileDesc *>(ws + p.off_tiles);
+  uint32_t *list = reinterpret_cast<uint32_t *>(ws + p.off_list);
+  uint32_t *scores = reinterpret_cast<uint32_t *>(ws + p.off_scores);
+  *scores_out = scores;
+  CUtensorMap kmap;
+  if (!make_key_tensor_map(&kmap, k)) return cudaErrorInvalidValue;
+  cudaError_t e = cudaMemsetAsync(cnt, 0, (size_t)p.nb * 4, st);
+  if (e != cudaSuccess) return e;
+  const int warps = (total_q + 31) / 32;
+  const int grid = (warps + 7) / 8;
+  {
+    ProfScope ps(K_INV_LISTS, st);
+    inv_lists_kernel<<<grid, 256, 0, st>>>(blk, total_q, m, cu_q, S, emax, 0, cnt, cursor, list);
+  }
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  {
+    ProfScope ps(K_INV_SCAN, st);
+    inv_scan_kernel<<<1, SCAN_THREADS, 0, st>>>(cnt, p.nb, cursor, tiles, ntiles);
+  }
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  {
+    ProfScope ps(K_INV_LISTS, st);
+    inv_lists_kernel<<<grid, 256, 0, st>>>(blk, total_q, m, cu_q, S, emax, 1, cnt, cursor, list);
+  }
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  static int attr[64];
+  if ((e = set_smem_once((const void *)token_score_tc_kernel, TC_SMEM_BYTES, attr)) != cudaSuccess)
+    return e;
+  {
+    ProfScope ps(K_TOKEN_SCORE_TC, st);
+    token_score_tc_kernel<<<2 * num_sms, TC_THREADS, TC_SMEM_BYTES, st>>>(
+        kmap, q, k, cu_q, cu_k, seqlens, emax, m, tiles, ntiles, list, scores, status);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace hisa
