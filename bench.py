@@ -55,6 +55,8 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-extras", action="store_true", help="skip the details measurements")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
+    ap.add_argument("--config", type=int, default=4, choices=[1, 3, 4, 5],
+                    help="prefill workload of the timed step (profiling runs; default 4 = 128K)")
     return ap.parse_args()
 
 
@@ -178,12 +180,44 @@ def to_dev_i32(a):
     return torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).cuda()
 
 
-def candidates_per_query(pos: np.ndarray, B: int, m: int) -> np.ndarray:
-    """Stage-2 candidates of a query at position p (single sequence): every token of the
-    selected blocks up to p; m blocks are selected, all full except the own block."""
-    full = pos + 1
-    capped = (m - 1) * B + (pos % B) + 1
-    return np.minimum(full, capped)
+ALU_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+ALU_PEAK_SOURCE = "148 SMs x 128 FP32 lanes x 2 flop x 1965 MHz (max SM clock)"
+
+
+def query_positions(w) -> np.ndarray:
+    """Sequence-local position of every query row (the last q_len positions)."""
+    out = np.empty(w.total_q, np.int64)
+    for s in range(w.num_seqs):
+        a, b = int(w.cu_q[s]), int(w.cu_q[s + 1])
+        L = int(w.seqlens[s])
+        out[a:b] = np.arange(L - (b - a), L)
+    return out
+
+
+def algorithmic(w) -> dict:
+    """Algorithmic work per step of every kernel on the prefill path (bytes that must
+    move, or flops that must be done, counting nothing the method avoids)."""
+    B, m, K, d = w.B, w.m, w.topk, 64
+    pos = query_positions(w)
+    own = pos // B
+    nsel = np.minimum(m, own + 1)
+    pairs = float(nsel.sum())
+    scored_blocks = float(np.where(own + 1 > m, own + 1, 0).sum())
+    live_rows = float(w.seqlens.sum())
+    nblocks = float(((w.seqlens + B - 1) // B).sum())
+    nq = float(w.total_q)
+    return {
+        "pool_blocks": {"bound": "hbm", "per_step": live_rows * 2 * d + nblocks * 4 * d,
+                        "what": "keys read once + fp32 representatives written"},
+        "block_select": {"bound": "alu", "per_step": scored_blocks * d * 2,
+                         "what": "q.rep dot products of every eligible block (2 flop/MAC)"},
+        "inv_lists": {"bound": "hbm", "per_step": pairs * 4 * 2 + pairs * 4,
+                      "what": "block lists read twice + (query, slot) lists written"},
+        "token_score_tc": {"bound": "hbm", "per_step": pairs * B * 4 + nq * 2 * d + live_rows * 2 * d,
+                           "what": "score rows written (m*128 fp32 per query) + q, k read once"},
+        "token_select_scratch": {"bound": "hbm", "per_step": pairs * B * 4 + nq * K * 4 + nq * m * 4,
+                                 "what": "score rows read + k int32 indices written + block lists"},
+    }
 
 
 def iou_rows(a: np.ndarray, b: np.ndarray) -> float:
@@ -221,14 +255,14 @@ def run_ours(args, world, rank):
     stream = torch.cuda.current_stream()
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
 
-    w = config_workload(4)
+    w = config_workload(args.config)
     B, m, K = w.B, w.m, w.topk
     nq = w.total_q
     q, k = to_dev_bf16(w.q), to_dev_bf16(w.k)
     cu_q, cu_k, sl = to_dev_i32(w.cu_q), to_dev_i32(w.cu_k), to_dev_i32(w.seqlens)
     out = torch.empty(nq, K, dtype=torch.int32, device="cuda")
     reps = torch.zeros(w.rep_rows, 64, dtype=torch.float32, device="cuda")
-    ws = torch.empty(max(H.hisa_select_workspace_size(nq, 1, w.max_seqlen_k, m, K), 256),
+    ws = torch.empty(max(H.hisa_select_workspace_size(nq, w.num_seqs, w.max_seqlen_k, m, K), 256),
                      dtype=torch.uint8, device="cuda")
 
     def step():
@@ -296,35 +330,37 @@ def run_ours(args, world, rank):
     d2h = hout.numel() * hout.element_size()
 
     # ---- roofline of the dominant kernel -------------------------------------------
-    dom = max(kt.items(), key=lambda kv: kv[1]["ms"])
-    dname, dstat = dom[0], dom[1]
-    per_launch_ms = dstat["ms"] / max(dstat["timed"], 1)
-    pos = np.arange(nq)
-    if dname == "token_fused":
-        cands = float(candidates_per_query(pos, B, m).sum())
-        flops = cands * 64 * 2
-        alu_peak = 148 * 128 * 2 * 1.965e9 / 1e12  # FP32 lanes x 2 flop x max SM clock, TFLOP/s
-        achieved = flops / (per_launch_ms / 1e3) / 1e12
-        roof = {"kernel": dname, "bound": "alu", "achieved": round(achieved, 3),
-                "peak": round(alu_peak, 2), "unit": "TFLOP/s", "frac": round(achieved / alu_peak, 4),
-                "peak_source": "148 SMs x 128 FP32 lanes x 2 x 1965 MHz",
-                "algorithmic": f"{cands:.4g} candidates x 64 FMA",
-                "launch_ms": round(per_launch_ms, 4)}
-    else:
-        nbytes = {"pool_blocks": nq * 128 + w.rep_rows * 256,
-                  "block_select": nq * 128 + nq * m * 4}.get(dname, 0)
-        achieved = nbytes / (per_launch_ms / 1e3) / 1e9
-        roof = {"kernel": dname, "bound": "hbm", "achieved": round(achieved, 1),
-                "peak": hbm_peak, "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
-                "launch_ms": round(per_launch_ms, 4)}
+    alg = algorithmic(w)
+    per_kernel = {}
+    for name, v in kt.items():
+        if not v["timed"] or name not in alg:
+            continue
+        a = alg[name]
+        launch_ms = v["ms"] / v["timed"]
+        launches_per_step = v["timed"] / args.steps
+        amount = a["per_step"] / launches_per_step  # per launch
+        if a["bound"] == "hbm":
+            ach, peak, unit = amount / (launch_ms / 1e3) / 1e9, hbm_peak, "GB/s"
+        elif a["bound"] == "tensor":
+            ach, peak, unit = amount / (launch_ms / 1e3) / 1e12, tc_peak, "TFLOP/s"
+        else:
+            ach, peak, unit = amount / (launch_ms / 1e3) / 1e12, ALU_PEAK_TFLOPS, "TFLOP/s"
+        per_kernel[name] = {"bound": a["bound"], "achieved": round(ach, 3), "peak": peak,
+                            "unit": unit, "frac": round(ach / peak, 4),
+                            "launch_ms": round(launch_ms, 4), "algorithmic": a["what"]}
+    dname = max((n for n in per_kernel), key=lambda n: kt[n]["ms"])
+    roof = dict(per_kernel[dname])
+    roof["kernel"] = dname
     t = TRAFFIC.get(dname)
     roof["traffic"] = t[0] if t and t[1] == source_sha(t[2]) else None
-    roof["peak_source"] = roof.get("peak_source", f"MEASURED_PEAKS.json ({peak_src})")
+    roof["peak_source"] = (ALU_PEAK_SOURCE if roof["bound"] == "alu" else
+                           f"MEASURED_PEAKS.json ({peak_src})")
 
-    details = {"hisa_128k": {"ms": round(ms, 4), "queries_per_s": round(nq / (ms / 1e3), 1),
+    details = {"hisa_step": {"ms": round(ms, 4), "queries_per_s": round(nq / (ms / 1e3), 1),
                              "kernels": {n: {"ms_per_step": round(v["ms"] / args.steps, 4),
                                              "launches": v["launches"]}
-                                         for n, v in kt.items() if v["launches"]}}}
+                                         for n, v in kt.items() if v["launches"]},
+                             "roofline_per_kernel": per_kernel}}
     if rank == 0 and not args.no_extras:
         details.update(extras(args, w, q, k, cu_q, cu_k, sl, out, flush, stream, hbm_peak))
 

@@ -27,6 +27,7 @@ constexpr int DSA_Q = 128;   // queries per filter CTA
 constexpr int DSA_NB = 128;  // score buckets
 constexpr int DSA_KT = 64;   // keys per staged tile
 constexpr int DSA_SEL_THREADS = 256;
+constexpr int DSA_SEL_KPT = 16;  // candidate lists hold at most 256 * 16 keys
 constexpr int DSA_FB_CTAS = 16;
 
 __global__ void __launch_bounds__(256)
@@ -205,8 +206,8 @@ struct DsaPad {
   }
 };
 
-__host__ __device__ inline size_t dsa_select_smem(int cap, int topk) {
-  return (size_t)cap * 4 + (size_t)16 * topk + sizeof(SelectShared);
+__host__ __device__ inline size_t dsa_select_smem(int topk) {
+  return (size_t)16 * topk + sizeof(LinShared);
 }
 
 __global__ void __launch_bounds__(DSA_SEL_THREADS)
@@ -217,20 +218,13 @@ dsa_select_kernel(int row0, int topk, int cap, const uint32_t *__restrict__ buf_
   const int local = blockIdx.x, row = row0 + local;
   const int n = cnt[local];
   if (n > cap) return;  // the fallback kernel owns this row
-  uint32_t *keys = reinterpret_cast<uint32_t *>(smem);
-  uint8_t *rest = smem + (size_t)cap * 4;
-  uint32_t *sel_key = reinterpret_cast<uint32_t *>(rest);
-  int *sel_c = reinterpret_cast<int *>(rest + (size_t)4 * topk);
-  uint32_t *tmp_key = reinterpret_cast<uint32_t *>(rest + (size_t)8 * topk);
-  int *tmp_c = reinterpret_cast<int *>(rest + (size_t)12 * topk);
-  SelectShared &sh = *reinterpret_cast<SelectShared *>(rest + (size_t)16 * topk);
-  const uint32_t *src = buf_key + (size_t)local * cap;
-  for (int i = threadIdx.x; i < n; i += DSA_SEL_THREADS) keys[i] = src[i];
-  __syncthreads();
+  uint32_t *work = reinterpret_cast<uint32_t *>(smem);
+  LinShared &sh = *reinterpret_cast<LinShared *>(smem + (size_t)16 * topk);
   int32_t *oi = out_idx + (size_t)row * topk;
   float *os = out_scores ? out_scores + (size_t)row * topk : nullptr;
-  select_topk<DSA_SEL_THREADS>(keys, n, topk, sh, sel_key, sel_c, tmp_key, tmp_c,
-                               DsaOut{oi, os, buf_j + (size_t)local * cap}, DsaPad{oi, os});
+  select_topk_reg<DSA_SEL_THREADS, DSA_SEL_KPT>(buf_key + (size_t)local * cap, n, topk, sh, work,
+                                                DsaOut{oi, os, buf_j + (size_t)local * cap},
+                                                DsaPad{oi, os});
 }
 
 __global__ void __launch_bounds__(DSA_SEL_THREADS)
@@ -286,7 +280,7 @@ static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 DsaPlan dsa_plan(int total_q, int num_seqs, int max_seqlen_k, int topk) {
   DsaPlan p;
-  p.cap = topk + 2048;
+  p.cap = (topk + 2048 + 3) & ~3;  // rows stay 16-byte aligned; at most 4096 entries
   // keep the candidate lists to about 512 MiB
   long long chunk = (512ll << 20) / ((long long)p.cap * 8);
   chunk = chunk < DSA_Q ? DSA_Q : chunk;
@@ -326,7 +320,7 @@ cudaError_t launch_dsa(const uint16_t *q, const uint16_t *k, const int32_t *cu_q
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   const size_t fsm = sizeof(DsaShared);
-  const size_t ssm = dsa_select_smem(p.cap, topk);
+  const size_t ssm = dsa_select_smem(topk);
   const size_t bsm = (size_t)16 * topk + sizeof(SelectShared);
   static int attr_f[64], attr_s[64], attr_b[64];
   if ((e = set_smem_once((const void *)dsa_filter_kernel, fsm, attr_f)) != cudaSuccess) return e;

@@ -226,3 +226,215 @@ __device__ void select_topk(const uint32_t *key, int n, int k, SelectShared &sh,
 }
 
 }  // namespace hisa
+
+namespace hisa {
+
+// ---------------------------------------------------------------------------
+// Exact top-k through linear score buckets, candidates held in registers.
+//
+// Each of the NT threads loads KPT of the n <= NT*KPT candidate keys once
+// (coalesced 16-byte loads; candidate c = ((i/4)*NT + thread)*4 + i%4) and keeps
+// them in registers.  Then:
+// 1. min/max and count of the candidate scores;
+// 2. histogram over LIN_BINS buckets linear in the score between max and min
+//    (bucket 0 holds the highest scores).  The bucket map is monotone in the score,
+//    so bucket order is score order;
+// 3. one scan gives every bucket its output offset and finds the bucket b* that
+//    holds the k-th best score;
+// 4. candidates in buckets before b* are scattered to their bucket's output range,
+//    those in b* are gathered apart;
+// 5. the b* candidates are ranked exactly by (score desc, index asc) and the best
+//    k - |buckets before b*| of them fill the end of the output;
+// 6. every other survivor is ranked within its own bucket (a handful of elements
+//    for continuous scores) and written to its final slot.
+// A boundary bucket with more than k members (heavy ties) sends the query through
+// the radix routine above instead, reading the keys again from `key`.
+
+constexpr int LIN_BINS = 2048;
+
+struct LinShared {
+  union {
+    SelectShared radix;
+    struct {
+      uint32_t cnt[LIN_BINS];
+      uint32_t off[LIN_BINS];
+      int warp_tot[33];
+      int wn[32];
+      uint32_t wmx[32], wmn[32];
+      uint32_t misc[8];
+    } lin;
+  };
+};
+
+__device__ __forceinline__ int lin_bucket(uint32_t u, float smax, float inv) {
+  const int b = __float2int_rz((smax - key_score(u)) * inv);
+  return min(max(b, 0), LIN_BINS - 1);
+}
+
+// key: the n candidate keys (global or shared memory), candidate (= token) order,
+// 16-byte aligned.  work: 4*k words of shared scratch.
+template <int NT, int KPT, class Out, class Pad>
+__device__ void select_topk_reg(const uint32_t *key, int n, int k, LinShared &sh, uint32_t *work,
+                                Out out, Pad pad) {
+  static_assert(KPT % 4 == 0, "keys are loaded four at a time");
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  constexpr int NW = NT / 32;
+  uint32_t *tmp_key = work;
+  int *tmp_c = reinterpret_cast<int *>(work + k);
+  uint32_t *bnd_key = work + 2 * k;
+  int *bnd_c = reinterpret_cast<int *>(work + 3 * k);
+
+  uint32_t u[KPT];
+#pragma unroll
+  for (int j = 0; j < KPT / 4; j++) {
+    const int c0 = (j * NT + tid) * 4;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (c0 + 3 < n) {
+      v = *reinterpret_cast<const uint4 *>(key + c0);
+    } else if (c0 < n) {
+      v.x = key[c0];
+      if (c0 + 1 < n) v.y = key[c0 + 1];
+      if (c0 + 2 < n) v.z = key[c0 + 2];
+    }
+    u[4 * j] = v.x;
+    u[4 * j + 1] = v.y;
+    u[4 * j + 2] = v.z;
+    u[4 * j + 3] = v.w;
+  }
+  auto cand = [&](int i) { return ((i >> 2) * NT + tid) * 4 + (i & 3); };
+
+  // 1. range and count
+  uint32_t mx = 0u, mn = 0xffffffffu;
+  int nv = 0;
+#pragma unroll
+  for (int i = 0; i < KPT; i++) {
+    if (u[i]) {
+      mx = max(mx, u[i]);
+      mn = min(mn, u[i]);
+      nv++;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    nv += __shfl_xor_sync(0xffffffffu, nv, o);
+  }
+  if (lane == 0) {
+    sh.lin.wmx[warp] = mx;
+    sh.lin.wmn[warp] = mn;
+    sh.lin.wn[warp] = nv;
+  }
+  for (int i = tid; i < LIN_BINS; i += NT) sh.lin.cnt[i] = 0u;
+  __syncthreads();
+  mx = 0u;
+  mn = 0xffffffffu;
+  nv = 0;
+#pragma unroll
+  for (int w = 0; w < NW; w++) {
+    mx = max(mx, sh.lin.wmx[w]);
+    mn = min(mn, sh.lin.wmn[w]);
+    nv += sh.lin.wn[w];
+  }
+  const int nvalid = nv;
+  const float smax = key_score(mx), smin = key_score(mn);
+  const float range = smax - smin;
+  const float inv = (nvalid > 0 && range > 0.f) ? (float)LIN_BINS / range : 0.f;
+
+  // 2. histogram
+#pragma unroll
+  for (int i = 0; i < KPT; i++)
+    if (u[i]) atomicAdd(&sh.lin.cnt[lin_bucket(u[i], smax, inv)], 1u);
+  __syncthreads();
+
+  // 3. offsets and the boundary bucket
+  const int kp = min(k, nvalid);
+  {
+    constexpr int per = LIN_BINS / NT;
+    int local = 0;
+#pragma unroll
+    for (int i = 0; i < per; i++) local += (int)sh.lin.cnt[tid * per + i];
+    int total;
+    int run = block_exclusive_scan<NT>(local, sh.lin.warp_tot, &total);
+    if (tid == 0) {
+      sh.lin.misc[3] = LIN_BINS;  // no boundary bucket when every candidate survives
+      sh.lin.misc[4] = (uint32_t)kp;
+      sh.lin.misc[5] = 0u;        // boundary fill counter
+    }
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < per; i++) {
+      const int b = tid * per + i;
+      const int h = (int)sh.lin.cnt[b];
+      if (nvalid > k && run < k && run + h >= k) {
+        sh.lin.misc[3] = (uint32_t)b;
+        sh.lin.misc[4] = (uint32_t)run;
+      }
+      sh.lin.off[b] = (uint32_t)run;
+      sh.lin.cnt[b] = (uint32_t)run;  // becomes the scatter cursor
+      run += h;
+    }
+  }
+  __syncthreads();
+  const int bstar = (int)sh.lin.misc[3];
+  const int above = (int)sh.lin.misc[4];  // survivors in buckets before b*
+  const int need = kp - above;             // survivors taken from b*
+
+  // 4. scatter
+#pragma unroll
+  for (int i = 0; i < KPT; i++) {
+    if (u[i]) {
+      const int b = lin_bucket(u[i], smax, inv);
+      if (b < bstar) {
+        const uint32_t slot = atomicAdd(&sh.lin.cnt[b], 1u);
+        tmp_key[slot] = u[i];
+        tmp_c[slot] = cand(i);
+      } else if (b == bstar) {
+        const uint32_t e = atomicAdd(&sh.lin.misc[5], 1u);
+        if (e < (uint32_t)k) {
+          bnd_key[e] = u[i];
+          bnd_c[e] = cand(i);
+        }
+      }
+    }
+  }
+  __syncthreads();
+  const int nbnd = (int)sh.lin.misc[5];
+  if (nbnd > k) {  // heavy ties at the boundary: exact radix route
+    __syncthreads();
+    select_topk<NT>(key, n, k, sh.radix, work, reinterpret_cast<int *>(work + k), work + 2 * k,
+                    reinterpret_cast<int *>(work + 3 * k), out, pad);
+    return;
+  }
+
+  // 5. the boundary bucket, ranked exactly
+  if (need > 0) {
+    for (int e = tid; e < nbnd; e += NT) {
+      const uint32_t ue = bnd_key[e];
+      const int c = bnd_c[e];
+      int rank = 0;
+      for (int t = 0; t < nbnd; t++) {
+        const uint32_t u2 = bnd_key[t];
+        rank += (u2 > ue) || (u2 == ue && bnd_c[t] < c);
+      }
+      if (rank < need) out(above + rank, c, ue);
+    }
+  }
+  // 6. everything above the boundary, ranked within its bucket
+  for (int s = tid; s < above; s += NT) {
+    const uint32_t us = tmp_key[s];
+    const int c = tmp_c[s];
+    const int b = lin_bucket(us, smax, inv);
+    const int st = (int)sh.lin.off[b], en = (int)sh.lin.cnt[b];
+    int rank = 0;
+    for (int t = st; t < en; t++) {
+      const uint32_t u2 = tmp_key[t];
+      rank += (u2 > us) || (u2 == us && tmp_c[t] < c);
+    }
+    out(st + rank, c, us);
+  }
+  for (int r = kp + tid; r < k; r += NT) pad(r);
+  __syncthreads();
+}
+
+}  // namespace hisa

@@ -91,13 +91,9 @@ struct RowPad {
   }
 };
 
-// shared-memory layout of the selecting kernels
-__host__ __device__ inline size_t stage_bytes(int topk) {
-  size_t a = (size_t)STAGE_ROWS * ROW_BYTES, b = (size_t)16 * topk;
-  return a > b ? a : b;
-}
+// shared memory of the selecting kernel: work (4k words) | LinShared | the block list
 __host__ __device__ inline size_t token_smem_bytes(int m, int topk) {
-  return (size_t)m * BLK * 4 + stage_bytes(topk) + sizeof(SelectShared);
+  return (size_t)16 * topk + sizeof(LinShared) + (size_t)m * 4;
 }
 
 __global__ void __launch_bounds__(TS_THREADS)
@@ -121,34 +117,31 @@ token_score_split_kernel(const uint16_t *__restrict__ q, const uint16_t *__restr
               [&](int c, uint32_t key) { dst[c] = key; });
 }
 
-__global__ void __launch_bounds__(TS_THREADS)
+// One CTA per query: exact top-k of the query's score row.  NT threads hold KPT
+// candidates each (NT * KPT >= m * 128).
+template <int NT, int KPT>
+__global__ void __launch_bounds__(NT, 1024 / NT)
 token_select_scratch_kernel(const int32_t *__restrict__ cu_q, const int32_t *__restrict__ cu_k,
                             const int32_t *__restrict__ seqlens, int S, int m, int topk,
                             const int32_t *__restrict__ blk, const uint32_t *__restrict__ scratch,
                             int32_t *__restrict__ out_idx, float *__restrict__ out_scores) {
   extern __shared__ __align__(16) uint8_t smem[];
-  uint32_t *keys = reinterpret_cast<uint32_t *>(smem);
-  uint8_t *stage = smem + (size_t)m * BLK * 4;
-  SelectShared &sh = *reinterpret_cast<SelectShared *>(stage + stage_bytes(topk));
+  uint32_t *work = reinterpret_cast<uint32_t *>(smem);
+  LinShared &sh = *reinterpret_cast<LinShared *>(smem + (size_t)16 * topk);
+  int32_t *sblk = reinterpret_cast<int32_t *>(smem + (size_t)16 * topk + sizeof(LinShared));
   const int row = blockIdx.x;
   RowPad pad{out_idx + (size_t)row * topk, out_scores ? out_scores + (size_t)row * topk : nullptr};
   const QueryInfo qi = locate(cu_q, cu_k, seqlens, S, row, nullptr);
   if (!qi.ok) {
-    for (int r = threadIdx.x; r < topk; r += TS_THREADS) pad(r);
+    for (int r = threadIdx.x; r < topk; r += NT) pad(r);
     return;
   }
-  const int32_t *blkrow = blk + (size_t)row * m;
-  const int nsel = count_selected(blkrow, m);
-  const uint4 *src = reinterpret_cast<const uint4 *>(scratch + (size_t)row * m * BLK);
-  for (int i = threadIdx.x; i < nsel * BLK / 4; i += TS_THREADS)
-    reinterpret_cast<uint4 *>(keys)[i] = src[i];
+  // the block stage keeps exactly min(m, own block + 1) blocks of a valid query
+  const int nsel = min(m, qi.pos / BLK + 1);
+  for (int i = threadIdx.x; i < nsel; i += NT) sblk[i] = blk[(size_t)row * m + i];
   __syncthreads();
-  uint32_t *sel_key = reinterpret_cast<uint32_t *>(stage);
-  int *sel_c = reinterpret_cast<int *>(stage + (size_t)4 * topk);
-  uint32_t *tmp_key = reinterpret_cast<uint32_t *>(stage + (size_t)8 * topk);
-  int *tmp_c = reinterpret_cast<int *>(stage + (size_t)12 * topk);
-  TokenOut out{pad.idx, pad.scores, blkrow};
-  select_topk<TS_THREADS>(keys, nsel * BLK, topk, sh, sel_key, sel_c, tmp_key, tmp_c, out, pad);
+  TokenOut out{pad.idx, pad.scores, sblk};
+  select_topk_reg<NT, KPT>(scratch + (size_t)row * m * BLK, nsel * BLK, topk, sh, work, out, pad);
 }
 
 // Split schedule when there are too few queries to fill the GPU with tensor-core tiles.
@@ -193,13 +186,20 @@ cudaError_t launch_token_select(const uint16_t *q, const uint16_t *k, const int3
     if (e != cudaSuccess) return e;
   }
   const size_t smem = token_smem_bytes(m, topk);
-  static int attr_sel[64];
-  if ((e = set_smem_once((const void *)token_select_scratch_kernel, smem, attr_sel)) != cudaSuccess)
-    return e;
-  {
+  if (m * BLK <= 256 * 32) {
+    static int attr_a[64];
+    auto kern = token_select_scratch_kernel<256, 32>;
+    if ((e = set_smem_once((const void *)kern, smem, attr_a)) != cudaSuccess) return e;
     ProfScope ps(K_TOKEN_SELECT_SCRATCH, st);
-    token_select_scratch_kernel<<<total_q, TS_THREADS, smem, st>>>(
-        cu_q, cu_k, seqlens, S, m, topk, blk, scores, out_idx, out_scores);
+    kern<<<total_q, 256, smem, st>>>(cu_q, cu_k, seqlens, S, m, topk, blk, scores, out_idx,
+                                     out_scores);
+  } else {
+    static int attr_b[64];
+    auto kern = token_select_scratch_kernel<512, 32>;
+    if ((e = set_smem_once((const void *)kern, smem, attr_b)) != cudaSuccess) return e;
+    ProfScope ps(K_TOKEN_SELECT_SCRATCH, st);
+    kern<<<total_q, 512, smem, st>>>(cu_q, cu_k, seqlens, S, m, topk, blk, scores, out_idx,
+                                     out_scores);
   }
   return cudaGetLastError();
 }
