@@ -209,8 +209,10 @@ def algorithmic(w) -> dict:
     return {
         "pool_blocks": {"bound": "hbm", "per_step": live_rows * 2 * d + nblocks * 4 * d,
                         "what": "keys read once + fp32 representatives written"},
-        "block_select": {"bound": "alu", "per_step": scored_blocks * d * 2,
-                         "what": "q.rep dot products of every eligible block (2 flop/MAC)"},
+        "block_score_tc": {"bound": "tensor", "per_step": scored_blocks * d * 2 * 2,
+                           "what": "q.rep_hi + q.rep_lo products of every eligible block (bf16 MMA)"},
+        "block_select": {"bound": "hbm", "per_step": scored_blocks * 4 + nq * m * 4,
+                         "what": "block-score keys read + selected block lists written"},
         "inv_lists": {"bound": "hbm", "per_step": pairs * 4 * 2 + pairs * 4,
                       "what": "block lists read twice + (query, slot) lists written"},
         "token_score_tc": {"bound": "hbm", "per_step": pairs * B * 4 + nq * 2 * d + live_rows * 2 * d,

@@ -19,7 +19,8 @@ cudaError_t launch_append(uint16_t *kc, float *reps, const int32_t *cu_k, int32_
 cudaError_t launch_block_select(const uint16_t *q, const float *reps, const int32_t *cu_q,
                                 const int32_t *cu_k, const int32_t *seqlens, int S,
                                 int total_q, int max_seqlen_k, int m, int32_t *blk,
-                                int32_t *out_blocks, int *status, cudaStream_t st);
+                                int32_t *out_blocks, uint8_t *ws, int num_sms, int *status,
+                                cudaStream_t st);
 cudaError_t launch_token_select(const uint16_t *q, const uint16_t *k, const int32_t *cu_q,
                                 const int32_t *cu_k, const int32_t *seqlens, int S, int total_q,
                                 int max_seqlen_k, int m, int topk, const int32_t *blk,
@@ -43,7 +44,7 @@ const char *kKindNames[K_NUM_KINDS] = {
     "pool_blocks",        "append_keys",         "block_select",   "token_fused",
     "token_score_split",  "token_select_scratch", "key_norm",      "dsa_filter",
     "dsa_select",         "dsa_fallback",         "inv_lists",      "inv_scan",
-    "token_score_tc"};
+    "token_score_tc",     "reps_split",          "block_score_tc"};
 long long g_launches[K_NUM_KINDS];
 double g_ms[K_NUM_KINDS];
 long long g_timed[K_NUM_KINDS];
@@ -229,7 +230,8 @@ hisa_status hisa_select(const hisa_bf16 *q_idx, const hisa_bf16 *k_idx, const fl
   uint8_t *w = static_cast<uint8_t *>(ws);
   int32_t *blk = reinterpret_cast<int32_t *>(w + p.off_blk);
   cudaError_t e = launch_block_select(q_idx, reps, cu_seqlens_q, cu_seqlens_k, seqlens_k,
-                                      num_seqs, total_q, max_seqlen_k, m, blk, out_blocks, st, s);
+                                      num_seqs, total_q, max_seqlen_k, m, blk, out_blocks,
+                                      w + p.off_scratch, num_sms(), st, s);
   if (e != cudaSuccess) return HISA_ERR_CUDA;
   e = launch_token_select(q_idx, k_idx, cu_seqlens_q, cu_seqlens_k, seqlens_k, num_seqs, total_q,
                           max_seqlen_k, m, k, blk, w + p.off_scratch, num_sms(), out_idx,
@@ -380,7 +382,8 @@ extern "C" hisa_status hisa_select_noalloc(const hisa_bf16 *q_idx, const hisa_bf
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int32_t *blk = reinterpret_cast<int32_t *>(w + p.off_blk);
   cudaError_t e = launch_block_select(q_idx, reps, cu_seqlens_q, cu_seqlens_k, seqlens_k,
-                                      num_seqs, total_q, max_seqlen_k, m, blk, out_blocks, st, s);
+                                      num_seqs, total_q, max_seqlen_k, m, blk, out_blocks,
+                                      w + p.off_scratch, num_sms(), st, s);
   if (e != cudaSuccess) return HISA_ERR_CUDA;
   e = launch_token_select(q_idx, k_idx, cu_seqlens_q, cu_seqlens_k, seqlens_k, num_seqs, total_q,
                           max_seqlen_k, m, k, blk, w + p.off_scratch, num_sms(), out_idx,

@@ -41,6 +41,7 @@ __global__ void __launch_bounds__(BS_WARPS * 32)
 block_select_kernel(const uint16_t *__restrict__ q, const float *__restrict__ reps,
                     const int32_t *__restrict__ cu_q, const int32_t *__restrict__ cu_k,
                     const int32_t *__restrict__ seqlens, int S, int total_q, int m, int emax,
+                    const uint32_t *__restrict__ tc_keys, int tc_stride,
                     int32_t *__restrict__ blk, int32_t *__restrict__ out_blocks,
                     int *status) {
   extern __shared__ uint32_t bs_smem[];
@@ -82,11 +83,16 @@ block_select_kernel(const uint16_t *__restrict__ q, const float *__restrict__ re
     return b == own || (nf >= 2 && b == own - 1) || (nf >= 3 && b == 0);
   };
 
-  QRegs qr;
-  load_q(qr, q + (size_t)row * D);
-  const float *rbase = reps + (size_t)(qi.kbase / BLK) * D;
-  for (int b = lane; b < E; b += 32)
-    keys[b] = forced(b) ? 0u : score_key(rep_score(qr, rbase + (size_t)b * D));
+  if (tc_keys) {  // scores already computed on the tensor cores (forced blocks hold 0)
+    const uint32_t *src = tc_keys + (size_t)row * tc_stride;
+    for (int b = lane; b < E; b += 32) keys[b] = __ldg(src + b);
+  } else {
+    QRegs qr;
+    load_q(qr, q + (size_t)row * D);
+    const float *rbase = reps + (size_t)(qi.kbase / BLK) * D;
+    for (int b = lane; b < E; b += 32)
+      keys[b] = forced(b) ? 0u : score_key(rep_score(qr, rbase + (size_t)b * D));
+  }
   __syncwarp();
 
   // T = key of the mfree-th best free block (0 if none are needed)
@@ -130,11 +136,31 @@ block_select_kernel(const uint16_t *__restrict__ q, const float *__restrict__ re
   }
 }
 
+bool use_tc_path(int total_q, int num_sms);
+cudaError_t launch_block_score_tc(const uint16_t *q, const float *reps, const int32_t *cu_q,
+                                  const int32_t *cu_k, const int32_t *seqlens, int S,
+                                  int total_q, int max_seqlen_k, int m, uint8_t *ws,
+                                  uint32_t **scores_out, int *status, cudaStream_t st);
+int block_score_stride(int max_seqlen_k);
+
+// Many queries: scores on the tensor cores (block_tc.cu), then one warp per query
+// selects.  Few queries (decode): one warp per query scores on the CUDA cores too.
 cudaError_t launch_block_select(const uint16_t *q, const float *reps, const int32_t *cu_q,
                                 const int32_t *cu_k, const int32_t *seqlens, int S,
                                 int total_q, int max_seqlen_k, int m, int32_t *blk,
-                                int32_t *out_blocks, int *status, cudaStream_t st) {
+                                int32_t *out_blocks, uint8_t *ws, int num_sms, int *status,
+                                cudaStream_t st) {
   if (total_q == 0) return cudaSuccess;
+  const uint32_t *tc_keys = nullptr;
+  int tc_stride = 0;
+  if (use_tc_path(total_q, num_sms)) {
+    uint32_t *sc = nullptr;
+    cudaError_t e = launch_block_score_tc(q, reps, cu_q, cu_k, seqlens, S, total_q, max_seqlen_k,
+                                          m, ws, &sc, status, st);
+    if (e != cudaSuccess) return e;
+    tc_keys = sc;
+    tc_stride = block_score_stride(max_seqlen_k);
+  }
   const int emax = (max_seqlen_k + BLK - 1) / BLK;
   const size_t smem = (size_t)BS_WARPS * (emax > 0 ? emax : 1) * sizeof(uint32_t);
   static int attr[64];
@@ -146,8 +172,9 @@ cudaError_t launch_block_select(const uint16_t *q, const float *reps, const int3
   {
     ProfScope ps(K_BLOCK_SELECT, st);
     block_select_kernel<<<grid, BS_WARPS * 32, smem, st>>>(q, reps, cu_q, cu_k, seqlens, S,
-                                                         total_q, m, emax > 0 ? emax : 1, blk,
-                                                         out_blocks, status);
+                                                         total_q, m, emax > 0 ? emax : 1,
+                                                         tc_keys, tc_stride, blk, out_blocks,
+                                                         status);
   }
   return cudaGetLastError();
 }

@@ -21,6 +21,8 @@ enum KernelKind {
   K_INV_LISTS,
   K_INV_SCAN,
   K_TOKEN_SCORE_TC,
+  K_REPS_SPLIT,
+  K_BLOCK_SCORE_TC,
   K_NUM_KINDS
 };
 

@@ -144,10 +144,13 @@ token_select_scratch_kernel(const int32_t *__restrict__ cu_q, const int32_t *__r
   select_topk_reg<NT, KPT>(scratch + (size_t)row * m * BLK, nsel * BLK, topk, sh, work, out, pad);
 }
 
-// Split schedule when there are too few queries to fill the GPU with tensor-core tiles.
-bool token_use_split(int total_q, int num_sms) { return total_q < 2 * num_sms; }
+// Tensor-core schedule when there are enough queries to fill the GPU with tiles;
+// otherwise (decode) the split CUDA-core schedule.
+bool use_tc_path(int total_q, int num_sms) { return total_q >= 2 * num_sms; }
+static bool token_use_split(int total_q, int num_sms) { return !use_tc_path(total_q, num_sms); }
 
 size_t tc_workspace_bytes(int total_q, int num_seqs, int max_seqlen_k, int m);
+size_t block_tc_workspace_bytes(int total_q, int num_seqs, int max_seqlen_k);
 cudaError_t launch_token_score_tc(const uint16_t *q, const uint16_t *k, const int32_t *cu_q,
                                   const int32_t *cu_k, const int32_t *seqlens, int S,
                                   int total_q, int max_seqlen_k, int m, const int32_t *blk,
@@ -156,7 +159,10 @@ cudaError_t launch_token_score_tc(const uint16_t *q, const uint16_t *k, const in
 
 size_t token_scratch_bytes(int total_q, int num_seqs, int max_seqlen_k, int m, int num_sms) {
   if (token_use_split(total_q, num_sms)) return (size_t)total_q * m * BLK * 4;
-  return tc_workspace_bytes(total_q, num_seqs, max_seqlen_k, m);
+  // the block-score matrix is dead before the token stage writes its lists and rows
+  const size_t a = tc_workspace_bytes(total_q, num_seqs, max_seqlen_k, m);
+  const size_t b = block_tc_workspace_bytes(total_q, num_seqs, max_seqlen_k);
+  return a > b ? a : b;
 }
 
 cudaError_t launch_token_select(const uint16_t *q, const uint16_t *k, const int32_t *cu_q,

@@ -234,20 +234,26 @@ static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// 2-D map over the key rows (64 bf16 = 128 bytes each), boxes of 128 rows, 128-byte
-// swizzle.  The row extent is left open: the kernel only asks for whole blocks that
-// lie inside a sequence's live keys.
-bool make_key_tensor_map(CUtensorMap *map, const uint16_t *k) {
+// 2-D map over rows of 64 bf16 (128 bytes each), boxes of box_rows rows, 128-byte
+// swizzle (the K-major SW128 operand layout); rows past `rows` read as zero.
+bool make_rows_tensor_map(CUtensorMap *map, const void *base, uint64_t rows, uint32_t box_rows) {
   auto enc = tensor_map_encoder();
-  if (!enc) return false;
-  cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)1 << 31};
+  if (!enc || rows == 0) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)ROW_BYTES};
-  cuuint32_t box[2] = {(cuuint32_t)D, (cuuint32_t)BLK};
+  cuuint32_t box[2] = {(cuuint32_t)D, box_rows};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t *>(k), dims,
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims,
                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+// Map over the key rows.  Their count is not passed to hisa_select, so the extent is
+// left open (2^31 rows): the kernel only asks for whole blocks that lie inside a
+// sequence's live keys.
+bool make_key_tensor_map(CUtensorMap *map, const uint16_t *k) {
+  return make_rows_tensor_map(map, k, (uint64_t)1 << 31, BLK);
 }
 
 struct TcPlan {
