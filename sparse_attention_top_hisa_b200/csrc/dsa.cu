@@ -8,13 +8,13 @@
 // Schedule (the score matrix is never materialised):
 //   1. key_norm_kernel: per sequence the largest key norm |k|max, so that every
 //      score of query q lies in [-R, R] with R = |q| |k|max (Cauchy-Schwarz).
-//   2. dsa_filter_kernel: one thread per query, 128 queries per CTA share key
-//      tiles staged in shared memory.  Pass 1 histograms the scores into 128
-//      linear buckets over [-R, R] (bucket 0 = highest); the bucket holding the
-//      k-th best score is b*.  Pass 2 recomputes the scores and appends every
-//      candidate in buckets <= b* (a superset of the top-k, in token order) to
-//      the query's candidate list.  Bucketing is monotone in the score, so the
-//      superset property holds exactly whatever the rounding.
+//   2. dsa_filter_tc_kernel (dsa_tc.cu): one thread per query, 128 queries per
+//      CTA, scores on the tensor cores.  Pass 1 histograms the scores into linear
+//      buckets over [-R, R] (bucket 0 = highest); the bucket holding the k-th best
+//      score is b*.  Pass 2 recomputes the scores and appends every candidate in
+//      buckets <= b* (a superset of the top-k, in token order) to the query's
+//      candidate list.  Bucketing is monotone in the score, so the superset
+//      property holds exactly whatever the rounding.
 //   3. dsa_select_kernel: exact top-k of each candidate list (shared routine).
 //   4. dsa_fallback_kernel: a row whose list overflowed its capacity (many equal
 //      scores) is redone exactly from a full score row in scratch memory.
@@ -24,8 +24,6 @@
 namespace hisa {
 
 constexpr int DSA_Q = 128;   // queries per filter CTA
-constexpr int DSA_NB = 128;  // score buckets
-constexpr int DSA_KT = 64;   // keys per staged tile
 constexpr int DSA_SEL_THREADS = 256;
 constexpr int DSA_SEL_KPT = 16;  // candidate lists hold at most 256 * 16 keys
 constexpr int DSA_FB_CTAS = 16;
@@ -58,124 +56,6 @@ key_norm_kernel(const uint16_t *__restrict__ k, const int32_t *__restrict__ cu_k
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) nrm = fmaxf(nrm, __shfl_xor_sync(0xffffffffu, nrm, o));
   if ((threadIdx.x & 31) == 0 && nrm > 0.f) atomicMax(reinterpret_cast<int *>(kmax + s), __float_as_int(nrm));
-}
-
-__device__ __forceinline__ int score_bucket(float s, float R, float inv) {
-  int b = __float2int_rz((R - s) * inv);
-  return min(max(b, 0), DSA_NB - 1);
-}
-
-struct DsaShared {
-  uint32_t hist[DSA_Q * (DSA_NB + 1)];
-  uint4 tile[DSA_KT * 8];
-  int jmax;
-  int srange[2];
-};
-
-__global__ void __launch_bounds__(DSA_Q)
-dsa_filter_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ k,
-                  const int32_t *__restrict__ cu_q, const int32_t *__restrict__ cu_k,
-                  const int32_t *__restrict__ seqlens, int S, int row0, int nrows, int topk,
-                  int cap, const float *__restrict__ kmax, uint32_t *__restrict__ buf_key,
-                  int32_t *__restrict__ buf_j, int32_t *__restrict__ cnt_out, int *status) {
-  extern __shared__ __align__(16) uint8_t dsa_smem[];
-  DsaShared &sh = *reinterpret_cast<DsaShared *>(dsa_smem);
-  const int tid = threadIdx.x;
-  const int local = blockIdx.x * DSA_Q + tid;  // row within the chunk
-  const int row = row0 + local;
-  const bool in_range = local < nrows;
-  QueryInfo qi;
-  qi.ok = false;
-  qi.seq = -1;
-  if (in_range) qi = locate(cu_q, cu_k, seqlens, S, row, status);
-  uint32_t *hist = sh.hist + tid * (DSA_NB + 1);
-  int count = 0;
-
-  QRegs qr;
-  float R = 0.f, inv = 0.f;
-  if (in_range && qi.ok) {
-    load_q(qr, q + (size_t)row * D);
-    float qq = 0.f;
-#pragma unroll
-    for (int c = 0; c < D; c++) qq = fmaf(qr.v[c], qr.v[c], qq);
-    R = sqrtf(qq) * kmax[qi.seq] * (1.0f + 1.0f / 1024.0f);
-    inv = R > 0.f ? (float)DSA_NB / (2.0f * R) : 0.f;
-  }
-  if (tid == 0) {
-    sh.srange[0] = in_range ? find_seq(cu_q, S, row) : 0;
-    int last = min(row0 + nrows, row0 + (int)(blockIdx.x + 1) * DSA_Q) - 1;
-    sh.srange[1] = find_seq(cu_q, S, last);
-  }
-  __syncthreads();
-  const int s_lo = sh.srange[0], s_hi = sh.srange[1];
-
-  for (int s = s_lo; s <= s_hi; s++) {
-    const bool active = in_range && qi.ok && qi.seq == s;
-    if (tid == 0) sh.jmax = -1;
-    __syncthreads();
-    if (active) atomicMax(&sh.jmax, qi.pos);
-    __syncthreads();
-    const int jmax = sh.jmax;
-    if (jmax < 0) continue;  // block-uniform
-    const uint4 *kseq = reinterpret_cast<const uint4 *>(k + (size_t)__ldg(cu_k + s) * D);
-
-    // pass 1: histogram
-    if (active)
-      for (int b = 0; b <= DSA_NB; b++) hist[b] = 0u;
-    for (int j0 = 0; j0 <= jmax; j0 += DSA_KT) {
-      const int nk = min(DSA_KT, jmax + 1 - j0);
-      __syncthreads();
-      for (int i = tid; i < nk * 8; i += DSA_Q) sh.tile[i] = __ldg(kseq + (size_t)j0 * 8 + i);
-      __syncthreads();
-      if (active) {
-        const int jend = min(nk, qi.pos + 1 - j0);
-        for (int jj = 0; jj < jend; jj++) {
-          uint4 w[8];
-#pragma unroll
-          for (int c = 0; c < 8; c++) w[c] = sh.tile[jj * 8 + c];
-          hist[score_bucket(token_score(qr, w), R, inv)]++;
-        }
-      }
-    }
-    // bucket of the k-th best score
-    int bstar = DSA_NB - 1;
-    if (active) {
-      int cum = 0;
-      for (int b = 0; b < DSA_NB; b++) {
-        cum += (int)hist[b];
-        if (cum >= topk) {
-          bstar = b;
-          break;
-        }
-      }
-    }
-    // pass 2: collect candidates in buckets <= b*
-    uint32_t *bk = buf_key + (size_t)local * cap;
-    int32_t *bj = buf_j + (size_t)local * cap;
-    for (int j0 = 0; j0 <= jmax; j0 += DSA_KT) {
-      const int nk = min(DSA_KT, jmax + 1 - j0);
-      __syncthreads();
-      for (int i = tid; i < nk * 8; i += DSA_Q) sh.tile[i] = __ldg(kseq + (size_t)j0 * 8 + i);
-      __syncthreads();
-      if (active) {
-        const int jend = min(nk, qi.pos + 1 - j0);
-        for (int jj = 0; jj < jend; jj++) {
-          uint4 w[8];
-#pragma unroll
-          for (int c = 0; c < 8; c++) w[c] = sh.tile[jj * 8 + c];
-          const float sc = token_score(qr, w);
-          if (score_bucket(sc, R, inv) <= bstar) {
-            if (count < cap) {
-              bk[count] = score_key(sc);
-              bj[count] = j0 + jj;
-            }
-            count++;
-          }
-        }
-      }
-    }
-  }
-  if (in_range) cnt_out[local] = count;
 }
 
 struct DsaOut {
@@ -281,8 +161,8 @@ static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 DsaPlan dsa_plan(int total_q, int num_seqs, int max_seqlen_k, int topk) {
   DsaPlan p;
   p.cap = (topk + 2048 + 3) & ~3;  // rows stay 16-byte aligned; at most 4096 entries
-  // keep the candidate lists to about 512 MiB
-  long long chunk = (512ll << 20) / ((long long)p.cap * 8);
+  // keep the candidate lists to about 8 GiB (one round covers 262144 queries at k = 2048)
+  long long chunk = (8ll << 30) / ((long long)p.cap * 8);
   chunk = chunk < DSA_Q ? DSA_Q : chunk;
   chunk = chunk > total_q ? total_q : chunk;
   p.chunk = (int)(chunk < 1 ? 1 : chunk);
@@ -300,6 +180,12 @@ DsaPlan dsa_plan(int total_q, int num_seqs, int max_seqlen_k, int topk) {
   p.total = off;
   return p;
 }
+
+cudaError_t launch_dsa_filter_tc(const uint16_t *q, const uint16_t *k, const int32_t *cu_q,
+                                 const int32_t *cu_k, const int32_t *seqlens, int S, int total_q,
+                                 int row0, int nrows, int topk, int cap, const float *kmax,
+                                 uint32_t *buf_key, int32_t *buf_j, int32_t *cnt, int *status,
+                                 cudaStream_t st);
 
 cudaError_t launch_dsa(const uint16_t *q, const uint16_t *k, const int32_t *cu_q,
                        const int32_t *cu_k, const int32_t *seqlens, int S, int total_q,
@@ -319,21 +205,16 @@ cudaError_t launch_dsa(const uint16_t *q, const uint16_t *k, const int32_t *cu_q
     key_norm_kernel<<<dim3((max_seqlen_k + 255) / 256, S), 256, 0, st>>>(k, cu_k, seqlens, kmax);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  const size_t fsm = sizeof(DsaShared);
   const size_t ssm = dsa_select_smem(topk);
   const size_t bsm = (size_t)16 * topk + sizeof(SelectShared);
-  static int attr_f[64], attr_s[64], attr_b[64];
-  if ((e = set_smem_once((const void *)dsa_filter_kernel, fsm, attr_f)) != cudaSuccess) return e;
+  static int attr_s[64], attr_b[64];
   if ((e = set_smem_once((const void *)dsa_select_kernel, ssm, attr_s)) != cudaSuccess) return e;
   if ((e = set_smem_once((const void *)dsa_fallback_kernel, bsm, attr_b)) != cudaSuccess) return e;
   for (int row0 = 0; row0 < total_q; row0 += p.chunk) {
     const int nrows = min(p.chunk, total_q - row0);
-    {
-      ProfScope ps(K_DSA_FILTER, st);
-      dsa_filter_kernel<<<(nrows + DSA_Q - 1) / DSA_Q, DSA_Q, fsm, st>>>(
-          q, k, cu_q, cu_k, seqlens, S, row0, nrows, topk, p.cap, kmax, bkey, bj, cnt, status);
-    }
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    e = launch_dsa_filter_tc(q, k, cu_q, cu_k, seqlens, S, total_q, row0, nrows, topk, p.cap, kmax,
+                             bkey, bj, cnt, status, st);
+    if (e != cudaSuccess) return e;
     {
       ProfScope ps(K_DSA_SELECT, st);
       dsa_select_kernel<<<nrows, DSA_SEL_THREADS, ssm, st>>>(row0, topk, p.cap, bkey, bj, cnt,

@@ -151,8 +151,6 @@ def test_equal_keys_degenerate():
     assert np.array_equal(h_idx, o_h)
 
 
-@pytest.mark.xfail(reason="the flat scan still scores on the CUDA cores; the identity needs "
-                          "both paths on the same tcgen05 arithmetic", strict=False)
 def test_hisa_equals_dsa_when_every_block_is_selected():
     """m >= number of blocks: HISA is the flat scan, bit for bit, on Gaussian inputs too."""
     w = gaussian_prefill(4096 + 77, 5, m=64, topk=512)
