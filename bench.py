@@ -516,9 +516,17 @@ def decode_bench(flush, stream, hbm_peak, n_states=4, steps=256):
         for kc, lens, reps, out in states:
             lens.copy_(lens0)
 
-    # warm-up (sets kernel attributes), then capture
+    # warm-up (sets kernel attributes), then a timed pass for the per-kernel breakdown,
+    # then capture
     run_steps()
     torch.cuda.synchronize()
+    reset()
+    H.hisa_timing_collect(reset=True)
+    H.hisa_timing_enable(True)
+    run_steps()
+    H.hisa_timing_enable(False)
+    breakdown = {n: round(v["ms"] / steps * 1e3, 2)
+                 for n, v in H.hisa_timing_collect(reset=True).items() if v["timed"]}
     reset()
     H.hisa_timing_collect(reset=True)
     g = torch.cuda.CUDAGraph()
@@ -552,7 +560,7 @@ def decode_bench(flush, stream, hbm_peak, n_states=4, steps=256):
             "launches_per_step": launches_per_graph / steps,
             "algorithmic_MB_per_step": round(per_seq * S / 1e6, 2),
             "GBs": round(gbs, 1), "frac_of_hbm_peak": round(gbs / hbm_peak, 4),
-            "states": n_states}
+            "states": n_states, "kernel_us_per_step_eager": breakdown}
 
 
 def cpu_baseline(w, budget_s: float = 15.0):

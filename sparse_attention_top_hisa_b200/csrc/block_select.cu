@@ -7,10 +7,11 @@
 // blocks survive.  The forced blocks count inside m; a query that sees at most
 // m blocks keeps all of them; ties between block scores go to the lower block.
 //
-// One warp per query.  The scores of the eligible, non-forced blocks are
-// turned into order-preserving keys in shared memory; a 32-step bitwise search
-// finds the key of the (m - |forced|)-th best block; ballots over ascending
-// block numbers resolve ties and emit the selected blocks in ascending order.
+// The scores of the eligible, non-forced blocks become order-preserving keys in
+// shared memory (computed on the tensor cores for many queries, on the CUDA cores
+// by one CTA per query for few); one warp per query then finds the key of the
+// (m - |forced|)-th best block with a 32-step bitwise search, and ballots over
+// ascending block numbers resolve ties and emit the selected blocks in order.
 #include "common.cuh"
 #include "prof.cuh"
 
@@ -37,64 +38,17 @@ __device__ __forceinline__ float rep_score(const QRegs &q, const float *rep) {
   return a + b;
 }
 
-__global__ void __launch_bounds__(BS_WARPS * 32)
-block_select_kernel(const uint16_t *__restrict__ q, const float *__restrict__ reps,
-                    const int32_t *__restrict__ cu_q, const int32_t *__restrict__ cu_k,
-                    const int32_t *__restrict__ seqlens, int S, int total_q, int m, int emax,
-                    const uint32_t *__restrict__ tc_keys, int tc_stride,
-                    int32_t *__restrict__ blk, int32_t *__restrict__ out_blocks,
-                    int *status) {
-  extern __shared__ uint32_t bs_smem[];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int row = blockIdx.x * BS_WARPS + warp;
-  if (row >= total_q) return;
-  uint32_t *keys = bs_smem + (size_t)warp * emax;
-  int32_t *dst = blk + (size_t)row * m;
-  int32_t *dst2 = out_blocks ? out_blocks + (size_t)row * m : nullptr;
-
-  const QueryInfo qi = locate(cu_q, cu_k, seqlens, S, row, status);
-  if (!qi.ok) {
-    for (int i = lane; i < m; i += 32) {
-      dst[i] = -1;
-      if (dst2) dst2[i] = -1;
-    }
-    return;
-  }
-  const int own = qi.pos / BLK, E = own + 1;
-  if (E > emax) {  // max_seqlen_k understated by the caller
-    if (lane == 0) raise_status(status, HISA_ERR_INVALID_ARG);
-    for (int i = lane; i < m; i += 32) {
-      dst[i] = -1;
-      if (dst2) dst2[i] = -1;
-    }
-    return;
-  }
-  if (E <= m) {  // every eligible block is kept
-    for (int i = lane; i < m; i += 32) {
-      int v = i < E ? i : -1;
-      dst[i] = v;
-      if (dst2) dst2[i] = v;
-    }
-    return;
-  }
+// Top-(m - |forced|) of the keys[0..E) of one query (forced blocks and blocks after
+// the query hold key 0), written in ascending block order with the forced blocks.
+// Executed by one full warp.
+__device__ void warp_select_blocks(const uint32_t *keys, int E, int own, int m,
+                                   int32_t *dst, int32_t *dst2) {
+  const int lane = threadIdx.x & 31;
   const int nf = min(m, 3);  // forced: own, previous, first (E > m >= 3 makes them distinct)
   const int mfree = m - nf;
   auto forced = [&](int b) {
     return b == own || (nf >= 2 && b == own - 1) || (nf >= 3 && b == 0);
   };
-
-  if (tc_keys) {  // scores already computed on the tensor cores (forced blocks hold 0)
-    const uint32_t *src = tc_keys + (size_t)row * tc_stride;
-    for (int b = lane; b < E; b += 32) keys[b] = __ldg(src + b);
-  } else {
-    QRegs qr;
-    load_q(qr, q + (size_t)row * D);
-    const float *rbase = reps + (size_t)(qi.kbase / BLK) * D;
-    for (int b = lane; b < E; b += 32)
-      keys[b] = forced(b) ? 0u : score_key(rep_score(qr, rbase + (size_t)b * D));
-  }
-  __syncwarp();
-
   // T = key of the mfree-th best free block (0 if none are needed)
   uint32_t T = 0u;
   if (mfree > 0) {
@@ -136,6 +90,99 @@ block_select_kernel(const uint16_t *__restrict__ q, const float *__restrict__ re
   }
 }
 
+// Common front part of both kernels: locate the query, handle invalid rows and the
+// take-all case.  Returns false when the row is finished.
+__device__ __forceinline__ bool block_row_setup(const int32_t *cu_q, const int32_t *cu_k,
+                                                const int32_t *seqlens, int S, int row, int m,
+                                                int emax, int32_t *dst, int32_t *dst2,
+                                                int *status, QueryInfo &qi, int &own, int &E,
+                                                int lane_id, int nthreads) {
+  qi = locate(cu_q, cu_k, seqlens, S, row, lane_id == 0 ? status : nullptr);
+  if (!qi.ok) {
+    for (int i = lane_id; i < m; i += nthreads) {
+      dst[i] = -1;
+      if (dst2) dst2[i] = -1;
+    }
+    return false;
+  }
+  own = qi.pos / BLK;
+  E = own + 1;
+  if (E > emax) {  // max_seqlen_k understated by the caller
+    if (lane_id == 0) raise_status(status, HISA_ERR_INVALID_ARG);
+    for (int i = lane_id; i < m; i += nthreads) {
+      dst[i] = -1;
+      if (dst2) dst2[i] = -1;
+    }
+    return false;
+  }
+  if (E <= m) {  // every eligible block is kept
+    for (int i = lane_id; i < m; i += nthreads) {
+      const int v = i < E ? i : -1;
+      dst[i] = v;
+      if (dst2) dst2[i] = v;
+    }
+    return false;
+  }
+  return true;
+}
+
+// Many queries: one warp per query reads the keys computed on the tensor cores.
+__global__ void __launch_bounds__(BS_WARPS * 32)
+block_select_kernel(const int32_t *__restrict__ cu_q, const int32_t *__restrict__ cu_k,
+                    const int32_t *__restrict__ seqlens, int S, int total_q, int m, int emax,
+                    const uint32_t *__restrict__ tc_keys, int tc_stride,
+                    int32_t *__restrict__ blk, int32_t *__restrict__ out_blocks,
+                    int *status) {
+  extern __shared__ uint32_t bs_smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.x * BS_WARPS + warp;
+  if (row >= total_q) return;
+  uint32_t *keys = bs_smem + (size_t)warp * emax;
+  int32_t *dst = blk + (size_t)row * m;
+  int32_t *dst2 = out_blocks ? out_blocks + (size_t)row * m : nullptr;
+  QueryInfo qi;
+  int own, E;
+  if (!block_row_setup(cu_q, cu_k, seqlens, S, row, m, emax, dst, dst2, status, qi, own, E, lane,
+                       32))
+    return;
+  const uint32_t *src = tc_keys + (size_t)row * tc_stride;
+  for (int b = lane; b < E; b += 32) keys[b] = __ldg(src + b);
+  __syncwarp();
+  warp_select_blocks(keys, E, own, m, dst, dst2);
+}
+
+// Few queries (decode): one CTA per query scores every eligible block on the CUDA
+// cores (one thread per block, all representative rows in flight at once), then warp
+// 0 selects.
+constexpr int BS_CTA_THREADS = 256;
+
+__global__ void __launch_bounds__(BS_CTA_THREADS)
+block_select_cta_kernel(const uint16_t *__restrict__ q, const float *__restrict__ reps,
+                        const int32_t *__restrict__ cu_q, const int32_t *__restrict__ cu_k,
+                        const int32_t *__restrict__ seqlens, int S, int m, int emax,
+                        int32_t *__restrict__ blk, int32_t *__restrict__ out_blocks,
+                        int *status) {
+  extern __shared__ uint32_t bsc_smem[];
+  const int row = blockIdx.x, tid = threadIdx.x;
+  int32_t *dst = blk + (size_t)row * m;
+  int32_t *dst2 = out_blocks ? out_blocks + (size_t)row * m : nullptr;
+  QueryInfo qi;
+  int own, E;
+  if (!block_row_setup(cu_q, cu_k, seqlens, S, row, m, emax, dst, dst2, status, qi, own, E, tid,
+                       BS_CTA_THREADS))
+    return;
+  const int nf = min(m, 3);
+  QRegs qr;
+  load_q(qr, q + (size_t)row * D);
+  const float *rbase = reps + (size_t)(qi.kbase / BLK) * D;
+  for (int b = tid; b < E; b += BS_CTA_THREADS) {
+    const bool forced = b == own || (nf >= 2 && b == own - 1) || (nf >= 3 && b == 0);
+    bsc_smem[b] = forced ? 0u : score_key(rep_score(qr, rbase + (size_t)b * D));
+  }
+  __syncthreads();
+  if (tid < 32) warp_select_blocks(bsc_smem, E, own, m, dst, dst2);
+}
+
 bool use_tc_path(int total_q, int num_sms);
 cudaError_t launch_block_score_tc(const uint16_t *q, const float *reps, const int32_t *cu_q,
                                   const int32_t *cu_k, const int32_t *seqlens, int S,
@@ -162,19 +209,28 @@ cudaError_t launch_block_select(const uint16_t *q, const float *reps, const int3
     tc_stride = block_score_stride(max_seqlen_k);
   }
   const int emax = (max_seqlen_k + BLK - 1) / BLK;
-  const size_t smem = (size_t)BS_WARPS * (emax > 0 ? emax : 1) * sizeof(uint32_t);
-  static int attr[64];
-  if (smem > 48 * 1024) {
-    cudaError_t e = set_smem_once((const void *)block_select_kernel, smem, attr);
-    if (e != cudaSuccess) return e;
-  }
-  dim3 grid((total_q + BS_WARPS - 1) / BS_WARPS);
-  {
+  if (tc_keys) {
+    const size_t smem = (size_t)BS_WARPS * (emax > 0 ? emax : 1) * sizeof(uint32_t);
+    static int attr[64];
+    if (smem > 48 * 1024) {
+      cudaError_t e = set_smem_once((const void *)block_select_kernel, smem, attr);
+      if (e != cudaSuccess) return e;
+    }
+    dim3 grid((total_q + BS_WARPS - 1) / BS_WARPS);
     ProfScope ps(K_BLOCK_SELECT, st);
-    block_select_kernel<<<grid, BS_WARPS * 32, smem, st>>>(q, reps, cu_q, cu_k, seqlens, S,
-                                                         total_q, m, emax > 0 ? emax : 1,
-                                                         tc_keys, tc_stride, blk, out_blocks,
-                                                         status);
+    block_select_kernel<<<grid, BS_WARPS * 32, smem, st>>>(cu_q, cu_k, seqlens, S, total_q, m,
+                                                         emax > 0 ? emax : 1, tc_keys, tc_stride,
+                                                         blk, out_blocks, status);
+  } else {
+    const size_t smem = (size_t)(emax > 0 ? emax : 1) * sizeof(uint32_t);
+    static int attr_cta[64];
+    if (smem > 48 * 1024) {
+      cudaError_t e = set_smem_once((const void *)block_select_cta_kernel, smem, attr_cta);
+      if (e != cudaSuccess) return e;
+    }
+    ProfScope ps(K_BLOCK_SELECT, st);
+    block_select_cta_kernel<<<total_q, BS_CTA_THREADS, smem, st>>>(
+        q, reps, cu_q, cu_k, seqlens, S, m, emax > 0 ? emax : 1, blk, out_blocks, status);
   }
   return cudaGetLastError();
 }

@@ -91,7 +91,7 @@ __host__ __device__ inline size_t dsa_select_smem(int topk) {
 }
 
 __global__ void __launch_bounds__(DSA_SEL_THREADS)
-dsa_select_kernel(int row0, int topk, int cap, const uint32_t *__restrict__ buf_key,
+dsa_select_kernel(int row0, int topk, int cap, const float *__restrict__ buf_key,
                   const int32_t *__restrict__ buf_j, const int32_t *__restrict__ cnt,
                   int32_t *__restrict__ out_idx, float *__restrict__ out_scores) {
   extern __shared__ __align__(16) uint8_t smem[];
@@ -142,7 +142,8 @@ dsa_fallback_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__
     __syncthreads();
     int32_t *oi = out_idx + (size_t)row * topk;
     float *os = out_scores ? out_scores + (size_t)row * topk : nullptr;
-    select_topk<DSA_SEL_THREADS>(keys, qi.pos + 1, topk, sh, sel_key, sel_c, tmp_key, tmp_c,
+    select_topk<DSA_SEL_THREADS>([&](int c) { return keys[c]; }, qi.pos + 1, topk, sh, sel_key,
+                                 sel_c, tmp_key, tmp_c,
                                  DirectOut{oi, os}, DsaPad{oi, os});
   }
 }
@@ -184,7 +185,7 @@ DsaPlan dsa_plan(int total_q, int num_seqs, int max_seqlen_k, int topk) {
 cudaError_t launch_dsa_filter_tc(const uint16_t *q, const uint16_t *k, const int32_t *cu_q,
                                  const int32_t *cu_k, const int32_t *seqlens, int S, int total_q,
                                  int row0, int nrows, int topk, int cap, const float *kmax,
-                                 uint32_t *buf_key, int32_t *buf_j, int32_t *cnt, int *status,
+                                 float *buf_key, int32_t *buf_j, int32_t *cnt, int *status,
                                  cudaStream_t st);
 
 cudaError_t launch_dsa(const uint16_t *q, const uint16_t *k, const int32_t *cu_q,
@@ -195,7 +196,7 @@ cudaError_t launch_dsa(const uint16_t *q, const uint16_t *k, const int32_t *cu_q
   const DsaPlan p = dsa_plan(total_q, S, max_seqlen_k, topk);
   float *kmax = reinterpret_cast<float *>(ws + p.off_kmax);
   int32_t *cnt = reinterpret_cast<int32_t *>(ws + p.off_cnt);
-  uint32_t *bkey = reinterpret_cast<uint32_t *>(ws + p.off_key);
+  float *bkey = reinterpret_cast<float *>(ws + p.off_key);
   int32_t *bj = reinterpret_cast<int32_t *>(ws + p.off_j);
   uint32_t *fb = reinterpret_cast<uint32_t *>(ws + p.off_fb);
   cudaError_t e = cudaMemsetAsync(kmax, 0, (size_t)S * 4, st);

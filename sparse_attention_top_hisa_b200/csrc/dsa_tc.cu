@@ -47,7 +47,7 @@ dsa_filter_tc_kernel(const __grid_constant__ CUtensorMap qmap,
                      const __grid_constant__ CUtensorMap kmap, const uint16_t *__restrict__ k,
                      const int32_t *__restrict__ cu_q, const int32_t *__restrict__ cu_k,
                      const int32_t *__restrict__ seqlens, int S, int row0, int nrows, int topk,
-                     int cap, const float *__restrict__ kmax, uint32_t *__restrict__ buf_key,
+                     int cap, const float *__restrict__ kmax, float *__restrict__ buf_key,
                      int32_t *__restrict__ buf_j, int32_t *__restrict__ cnt_out, int *status) {
   extern __shared__ uint8_t dsa_tc_raw[];
   DsaTcSmem &sm = *reinterpret_cast<DsaTcSmem *>((reinterpret_cast<uintptr_t>(dsa_tc_raw) + 1023) &
@@ -183,7 +183,7 @@ dsa_filter_tc_kernel(const __grid_constant__ CUtensorMap qmap,
     }
     const int pos = len - qlen + (row - q0);
     int bstar = DSA_TC_NB - 1, count = 0;
-    uint32_t *bk = buf_key + (size_t)(row - row0) * cap;
+    float *bk = buf_key + (size_t)(row - row0) * cap;
     int32_t *bj = buf_j + (size_t)(row - row0) * cap;
     for (int it = 0; it < steps; it++) {
       const int st = it & 1;
@@ -216,7 +216,7 @@ dsa_filter_tc_kernel(const __grid_constant__ CUtensorMap qmap,
               const float sc = __uint_as_float(v[u]);
               if (dsa_bucket(sc, R, inv) <= bstar) {
                 if (count < cap) {
-                  bk[count] = score_key(sc);
+                  bk[count] = sc;
                   bj[count] = b * BLK + c0 + u;
                 }
                 count++;
@@ -233,7 +233,7 @@ dsa_filter_tc_kernel(const __grid_constant__ CUtensorMap qmap,
                 atomicAdd(&hist[bb], 1u);
               } else if (bb <= bstar) {
                 if (count < cap) {
-                  bk[count] = score_key(sc);
+                  bk[count] = sc;
                   bj[count] = b * BLK + c0 + u;
                 }
                 count++;
@@ -260,7 +260,7 @@ bool make_key_tensor_map(CUtensorMap *map, const uint16_t *k);
 cudaError_t launch_dsa_filter_tc(const uint16_t *q, const uint16_t *k, const int32_t *cu_q,
                                  const int32_t *cu_k, const int32_t *seqlens, int S, int total_q,
                                  int row0, int nrows, int topk, int cap, const float *kmax,
-                                 uint32_t *buf_key, int32_t *buf_j, int32_t *cnt, int *status,
+                                 float *buf_key, int32_t *buf_j, int32_t *cnt, int *status,
                                  cudaStream_t st) {
   CUtensorMap qmap, kmap;
   if (!make_rows_tensor_map(&qmap, q, (uint64_t)total_q, BLK) || !make_key_tensor_map(&kmap, k))

@@ -61,11 +61,18 @@ pool_blocks_kernel(const uint16_t *__restrict__ k, const int32_t *__restrict__ c
                   reps + (size_t)(row0 / BLK) * D);
 }
 
-__global__ void __launch_bounds__(128)
+// Append: one CTA per sequence.  The block that receives the new rows is staged in
+// shared memory by all threads at once (one memory round trip), then summed row by
+// row in increasing order exactly like pool_block_warp, so the result is
+// bit-identical to pooling the grown block from scratch.
+constexpr int APPEND_THREADS = 256;
+
+__global__ void __launch_bounds__(APPEND_THREADS)
 append_keys_kernel(uint16_t *__restrict__ kc, float *__restrict__ reps,
                    const int32_t *__restrict__ cu_k, int32_t *__restrict__ seqlens,
                    const uint16_t *__restrict__ new_keys, int n_new, int *status) {
-  const int s = blockIdx.x, tid = threadIdx.x, warp = tid >> 5;
+  __shared__ __align__(16) uint4 blockrows[BLK * 8];
+  const int s = blockIdx.x, tid = threadIdx.x;
   const int start = cu_k[s], cap = cu_k[s + 1] - start;
   const int len = seqlens[s];
   if (start % BLK != 0) {
@@ -80,20 +87,35 @@ append_keys_kernel(uint16_t *__restrict__ kc, float *__restrict__ reps,
     if (tid == 0) raise_status(status, HISA_ERR_CAPACITY);
     return;
   }
-  // copy the new rows (16-byte chunks)
   const uint4 *src = reinterpret_cast<const uint4 *>(new_keys + (size_t)s * n_new * D);
-  uint4 *dst = reinterpret_cast<uint4 *>(kc + (size_t)(start + len) * D);
-  for (int i = tid; i < n_new * (ROW_BYTES / 16); i += blockDim.x) dst[i] = src[i];
-  __syncthreads();
-  // re-pool every block the new rows touched
+  uint4 *rows = reinterpret_cast<uint4 *>(kc + (size_t)start * D);
   const int nlen = len + n_new;
+  // copy the new rows to the cache
+  for (int i = tid; i < n_new * 8; i += APPEND_THREADS) rows[(size_t)len * 8 + i] = src[i];
+  // re-pool every touched block from shared memory
   const int first = len / BLK, last = (nlen - 1) / BLK;
-  for (int b = first + warp; b <= last; b += blockDim.x / 32) {
-    const int row0 = start + b * BLK;
-    pool_block_warp(reinterpret_cast<const uint32_t *>(kc + (size_t)row0 * D),
-                    min(BLK, nlen - b * BLK), reps + (size_t)(row0 / BLK) * D);
+  for (int b = first; b <= last; b++) {
+    const int count = min(BLK, nlen - b * BLK);
+    for (int i = tid; i < count * 8; i += APPEND_THREADS) {
+      const int r = b * BLK + (i >> 3);  // row within the sequence
+      blockrows[i] = r < len ? rows[(size_t)r * 8 + (i & 7)]
+                             : src[(size_t)(r - len) * 8 + (i & 7)];
+    }
+    __syncthreads();
+    if (tid < 32) {
+      const uint32_t *w = reinterpret_cast<const uint32_t *>(blockrows);
+      float a = 0.f, c = 0.f;
+      for (int t = 0; t < count; t++) {
+        const uint32_t x = w[t * 32 + tid];
+        a += bf_lo(x);
+        c += bf_hi(x);
+      }
+      const float cnt = (float)count;
+      reinterpret_cast<float2 *>(reps + (size_t)(start / BLK + b) * D)[tid] =
+          make_float2(__fdiv_rn(a, cnt), __fdiv_rn(c, cnt));
+    }
+    __syncthreads();
   }
-  __syncthreads();
   if (tid == 0) seqlens[s] = nlen;
 }
 
@@ -116,8 +138,8 @@ cudaError_t launch_append(uint16_t *kc, float *reps, const int32_t *cu_k, int32_
   if (num_seqs == 0 || n_new == 0) return cudaSuccess;
   {
     ProfScope ps(K_APPEND, st);
-    append_keys_kernel<<<num_seqs, 128, 0, st>>>(kc, reps, cu_k, seqlens, new_keys, n_new,
-                                                 status);
+    append_keys_kernel<<<num_seqs, APPEND_THREADS, 0, st>>>(kc, reps, cu_k, seqlens, new_keys,
+                                                            n_new, status);
   }
   return cudaGetLastError();
 }

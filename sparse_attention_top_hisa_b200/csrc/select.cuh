@@ -58,13 +58,12 @@ __device__ __forceinline__ void block_minmax(uint32_t &mx, uint32_t &mn, SelectS
   __syncthreads();
 }
 
-// key: n candidate keys (shared or global memory), token order.
+// key(c): the order-preserving key of candidate c (0 = not a candidate), token order.
 // sel_key/sel_c/tmp_key/tmp_c: shared arrays of at least k entries.
 // out(rank, c, key) writes one output slot; pad(rank) fills a slot past the survivors.
-template <int NT, class Out, class Pad>
-__device__ void select_topk(const uint32_t *key, int n, int k, SelectShared &sh,
-                            uint32_t *sel_key, int *sel_c, uint32_t *tmp_key, int *tmp_c,
-                            Out out, Pad pad) {
+template <int NT, class Key, class Out, class Pad>
+__device__ void select_topk(Key key, int n, int k, SelectShared &sh, uint32_t *sel_key,
+                            int *sel_c, uint32_t *tmp_key, int *tmp_c, Out out, Pad pad) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   constexpr int NW = NT / 32;
 
@@ -79,7 +78,7 @@ __device__ void select_topk(const uint32_t *key, int n, int k, SelectShared &sh,
     for (int i = tid; i < nb; i += NT) sh.hist[i] = 0;
     __syncthreads();
     for (int c = tid; c < n; c += NT) {
-      uint32_t u = key[c];
+      uint32_t u = key(c);
       if (u != 0u && (u & pmask) == prefix) atomicAdd(&sh.hist[(u >> shift) & (nb - 1)], 1u);
     }
     __syncthreads();
@@ -131,7 +130,7 @@ __device__ void select_topk(const uint32_t *key, int n, int k, SelectShared &sh,
   int ngt = 0, neq = 0;
   for (int base = c0; base < c1; base += 32) {
     int c = base + lane;
-    uint32_t u = c < c1 ? key[c] : 0u;
+    uint32_t u = c < c1 ? key(c) : 0u;
     ngt += __popc(__ballot_sync(0xffffffffu, u > T));
     neq += __popc(__ballot_sync(0xffffffffu, eq_live && u == T));
   }
@@ -158,7 +157,7 @@ __device__ void select_topk(const uint32_t *key, int n, int k, SelectShared &sh,
     const unsigned lt = (1u << lane) - 1u;
     for (int base = c0; base < c1; base += 32) {
       int c = base + lane;
-      uint32_t u = c < c1 ? key[c] : 0u;
+      uint32_t u = c < c1 ? key(c) : 0u;
       bool is_eq = eq_live && u == T;
       unsigned beq = __ballot_sync(0xffffffffu, is_eq);
       bool sel = (u > T) || (is_eq && eqr + __popc(beq & lt) < need_eq);
@@ -232,23 +231,25 @@ namespace hisa {
 // ---------------------------------------------------------------------------
 // Exact top-k through linear score buckets, candidates held in registers.
 //
-// Each of the NT threads loads KPT of the n <= NT*KPT candidate keys once
-// (coalesced 16-byte loads; candidate c = ((i/4)*NT + thread)*4 + i%4) and keeps
-// them in registers.  Then:
-// 1. min/max and count of the candidate scores;
+// Input: n raw fp32 scores in candidate (= token) order, -inf marking a position
+// that is not a candidate (finite scores are the contract).  Each of the NT threads
+// loads KPT of them once (coalesced 16-byte loads; candidate c = ((i/4)*NT +
+// thread)*4 + i%4) and keeps them in registers.  Then:
+// 1. max/min and count of the candidate scores (fused with the load);
 // 2. histogram over LIN_BINS buckets linear in the score between max and min
 //    (bucket 0 holds the highest scores).  The bucket map is monotone in the score,
 //    so bucket order is score order;
 // 3. one scan gives every bucket its output offset and finds the bucket b* that
 //    holds the k-th best score;
 // 4. candidates in buckets before b* are scattered to their bucket's output range,
-//    those in b* are gathered apart;
-// 5. the b* candidates are ranked exactly by (score desc, index asc) and the best
-//    k - |buckets before b*| of them fill the end of the output;
-// 6. every other survivor is ranked within its own bucket (a handful of elements
-//    for continuous scores) and written to its final slot.
+//    those in b* are gathered apart, each as a 64-bit (key, ~index) composite whose
+//    unsigned order is the output order (score desc, index asc);
+// 5. the b* candidates are ranked exactly and the best k - |buckets before b*| of
+//    them fill the end of the output;
+// 6. every other survivor is ranked within its own bucket (a handful of elements for
+//    continuous scores) and written to its final slot.
 // A boundary bucket with more than k members (heavy ties) sends the query through
-// the radix routine above instead, reading the keys again from `key`.
+// the radix routine above instead, reading the scores again.
 
 constexpr int LIN_BINS = 2048;
 
@@ -260,64 +261,66 @@ struct LinShared {
       uint32_t off[LIN_BINS];
       int warp_tot[33];
       int wn[32];
-      uint32_t wmx[32], wmn[32];
+      float wmx[32], wmn[32];
       uint32_t misc[8];
     } lin;
   };
 };
 
-__device__ __forceinline__ int lin_bucket(uint32_t u, float smax, float inv) {
-  const int b = __float2int_rz((smax - key_score(u)) * inv);
+__device__ __forceinline__ int lin_bucket(float s, float smax, float inv) {
+  const int b = __float2int_rz((smax - s) * inv);
   return min(max(b, 0), LIN_BINS - 1);
 }
 
-// key: the n candidate keys (global or shared memory), candidate (= token) order,
-// 16-byte aligned.  work: 4*k words of shared scratch.
+__device__ __forceinline__ uint64_t rank_key(float s, int c) {
+  return ((uint64_t)score_key(s) << 32) | (uint32_t)(~(uint32_t)c);
+}
+
+// sc: the n raw scores (global or shared memory, 16-byte aligned).
+// work: 4*k words (2*k uint64) of shared scratch.
 template <int NT, int KPT, class Out, class Pad>
-__device__ void select_topk_reg(const uint32_t *key, int n, int k, LinShared &sh, uint32_t *work,
+__device__ void select_topk_reg(const float *sc, int n, int k, LinShared &sh, uint32_t *work,
                                 Out out, Pad pad) {
-  static_assert(KPT % 4 == 0, "keys are loaded four at a time");
+  static_assert(KPT % 4 == 0, "scores are loaded four at a time");
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   constexpr int NW = NT / 32;
-  uint32_t *tmp_key = work;
-  int *tmp_c = reinterpret_cast<int *>(work + k);
-  uint32_t *bnd_key = work + 2 * k;
-  int *bnd_c = reinterpret_cast<int *>(work + 3 * k);
+  uint64_t *surv = reinterpret_cast<uint64_t *>(work);      // k survivors
+  uint64_t *bnd = reinterpret_cast<uint64_t *>(work) + k;   // up to k boundary members
+  const float NEG = -__int_as_float(0x7f800000);             // -inf
 
-  uint32_t u[KPT];
+  float f[KPT];
+  float mx = NEG, mn = -NEG;
+  int nv = 0;
 #pragma unroll
   for (int j = 0; j < KPT / 4; j++) {
     const int c0 = (j * NT + tid) * 4;
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    float4 v = make_float4(NEG, NEG, NEG, NEG);
     if (c0 + 3 < n) {
-      v = *reinterpret_cast<const uint4 *>(key + c0);
+      v = *reinterpret_cast<const float4 *>(sc + c0);
     } else if (c0 < n) {
-      v.x = key[c0];
-      if (c0 + 1 < n) v.y = key[c0 + 1];
-      if (c0 + 2 < n) v.z = key[c0 + 2];
+      v.x = sc[c0];
+      if (c0 + 1 < n) v.y = sc[c0 + 1];
+      if (c0 + 2 < n) v.z = sc[c0 + 2];
     }
-    u[4 * j] = v.x;
-    u[4 * j + 1] = v.y;
-    u[4 * j + 2] = v.z;
-    u[4 * j + 3] = v.w;
+    f[4 * j] = v.x;
+    f[4 * j + 1] = v.y;
+    f[4 * j + 2] = v.z;
+    f[4 * j + 3] = v.w;
+#pragma unroll
+    for (int e = 0; e < 4; e++) {
+      const float x = f[4 * j + e];
+      if (x != NEG) {
+        mx = fmaxf(mx, x);
+        mn = fminf(mn, x);
+        nv++;
+      }
+    }
   }
   auto cand = [&](int i) { return ((i >> 2) * NT + tid) * 4 + (i & 3); };
-
-  // 1. range and count
-  uint32_t mx = 0u, mn = 0xffffffffu;
-  int nv = 0;
-#pragma unroll
-  for (int i = 0; i < KPT; i++) {
-    if (u[i]) {
-      mx = max(mx, u[i]);
-      mn = min(mn, u[i]);
-      nv++;
-    }
-  }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
-    mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
     nv += __shfl_xor_sync(0xffffffffu, nv, o);
   }
   if (lane == 0) {
@@ -327,24 +330,24 @@ __device__ void select_topk_reg(const uint32_t *key, int n, int k, LinShared &sh
   }
   for (int i = tid; i < LIN_BINS; i += NT) sh.lin.cnt[i] = 0u;
   __syncthreads();
-  mx = 0u;
-  mn = 0xffffffffu;
+  mx = NEG;
+  mn = -NEG;
   nv = 0;
 #pragma unroll
   for (int w = 0; w < NW; w++) {
-    mx = max(mx, sh.lin.wmx[w]);
-    mn = min(mn, sh.lin.wmn[w]);
+    mx = fmaxf(mx, sh.lin.wmx[w]);
+    mn = fminf(mn, sh.lin.wmn[w]);
     nv += sh.lin.wn[w];
   }
   const int nvalid = nv;
-  const float smax = key_score(mx), smin = key_score(mn);
-  const float range = smax - smin;
+  const float smax = mx;
+  const float range = mx - mn;
   const float inv = (nvalid > 0 && range > 0.f) ? (float)LIN_BINS / range : 0.f;
 
   // 2. histogram
 #pragma unroll
   for (int i = 0; i < KPT; i++)
-    if (u[i]) atomicAdd(&sh.lin.cnt[lin_bucket(u[i], smax, inv)], 1u);
+    if (f[i] != NEG) atomicAdd(&sh.lin.cnt[lin_bucket(f[i], smax, inv)], 1u);
   __syncthreads();
 
   // 3. offsets and the boundary bucket
@@ -383,18 +386,14 @@ __device__ void select_topk_reg(const uint32_t *key, int n, int k, LinShared &sh
   // 4. scatter
 #pragma unroll
   for (int i = 0; i < KPT; i++) {
-    if (u[i]) {
-      const int b = lin_bucket(u[i], smax, inv);
+    if (f[i] != NEG) {
+      const int b = lin_bucket(f[i], smax, inv);
       if (b < bstar) {
         const uint32_t slot = atomicAdd(&sh.lin.cnt[b], 1u);
-        tmp_key[slot] = u[i];
-        tmp_c[slot] = cand(i);
+        surv[slot] = rank_key(f[i], cand(i));
       } else if (b == bstar) {
         const uint32_t e = atomicAdd(&sh.lin.misc[5], 1u);
-        if (e < (uint32_t)k) {
-          bnd_key[e] = u[i];
-          bnd_c[e] = cand(i);
-        }
+        if (e < (uint32_t)k) bnd[e] = rank_key(f[i], cand(i));
       }
     }
   }
@@ -402,6 +401,10 @@ __device__ void select_topk_reg(const uint32_t *key, int n, int k, LinShared &sh
   const int nbnd = (int)sh.lin.misc[5];
   if (nbnd > k) {  // heavy ties at the boundary: exact radix route
     __syncthreads();
+    auto key = [&](int c) -> uint32_t {
+      const float x = sc[c];
+      return x != NEG ? score_key(x) : 0u;
+    };
     select_topk<NT>(key, n, k, sh.radix, work, reinterpret_cast<int *>(work + k), work + 2 * k,
                     reinterpret_cast<int *>(work + 3 * k), out, pad);
     return;
@@ -410,28 +413,20 @@ __device__ void select_topk_reg(const uint32_t *key, int n, int k, LinShared &sh
   // 5. the boundary bucket, ranked exactly
   if (need > 0) {
     for (int e = tid; e < nbnd; e += NT) {
-      const uint32_t ue = bnd_key[e];
-      const int c = bnd_c[e];
+      const uint64_t me = bnd[e];
       int rank = 0;
-      for (int t = 0; t < nbnd; t++) {
-        const uint32_t u2 = bnd_key[t];
-        rank += (u2 > ue) || (u2 == ue && bnd_c[t] < c);
-      }
-      if (rank < need) out(above + rank, c, ue);
+      for (int t = 0; t < nbnd; t++) rank += bnd[t] > me;
+      if (rank < need) out(above + rank, (int)~(uint32_t)me, (uint32_t)(me >> 32));
     }
   }
-  // 6. everything above the boundary, ranked within its bucket
+  // 6. everything above the boundary, ranked within its own bucket
   for (int s = tid; s < above; s += NT) {
-    const uint32_t us = tmp_key[s];
-    const int c = tmp_c[s];
-    const int b = lin_bucket(us, smax, inv);
+    const uint64_t me = surv[s];
+    const int b = lin_bucket(key_score((uint32_t)(me >> 32)), smax, inv);
     const int st = (int)sh.lin.off[b], en = (int)sh.lin.cnt[b];
     int rank = 0;
-    for (int t = st; t < en; t++) {
-      const uint32_t u2 = tmp_key[t];
-      rank += (u2 > us) || (u2 == us && tmp_c[t] < c);
-    }
-    out(st + rank, c, us);
+    for (int t = st; t < en; t++) rank += surv[t] > me;
+    out(st + rank, (int)~(uint32_t)me, (uint32_t)(me >> 32));
   }
   for (int r = kp + tid; r < k; r += NT) pad(r);
   __syncthreads();

@@ -33,7 +33,8 @@ __device__ __forceinline__ void cp_async_commit_wait() {
   asm volatile("cp.async.wait_all;\n" ::: "memory");
 }
 
-// Scores selected-block slots [s0, s1) of one query; dst(candidate, key).
+// Scores selected-block slots [s0, s1) of one query; dst(candidate, raw score), -inf
+// for a key after the query.
 template <class Dst>
 __device__ __forceinline__ void score_slots(const QRegs &q, const uint16_t *kseq, int pos,
                                             const int32_t *blkrow, int s0, int s1,
@@ -52,24 +53,18 @@ __device__ __forceinline__ void score_slots(const QRegs &q, const uint16_t *kseq
     if (tid < nb2 * BLK) {
       const int r = tid;
       const int j = blkrow[p + (r >> 7)] * BLK + (r & 127);
-      uint32_t key = 0u;
+      float sc = -__int_as_float(0x7f800000);
       if (j <= pos) {
         uint4 w[8];
 #pragma unroll
         for (int c = 0; c < 8; c++)
           w[c] = *reinterpret_cast<const uint4 *>(stage + r * ROW_BYTES + ((c ^ (r & 7)) << 4));
-        key = score_key(token_score(q, w));
+        sc = token_score(q, w);
       }
-      dst((p << 7) + r, key);
+      dst((p << 7) + r, sc);
     }
     __syncthreads();
   }
-}
-
-__device__ __forceinline__ int count_selected(const int32_t *blkrow, int m) {
-  int n = 0;
-  while (n < m && blkrow[n] >= 0) n++;
-  return n;
 }
 
 struct TokenOut {
@@ -101,20 +96,20 @@ token_score_split_kernel(const uint16_t *__restrict__ q, const uint16_t *__restr
                          const int32_t *__restrict__ cu_q, const int32_t *__restrict__ cu_k,
                          const int32_t *__restrict__ seqlens, int S, int m,
                          const int32_t *__restrict__ blk, int slots_per_cta,
-                         uint32_t *__restrict__ scratch) {
+                         float *__restrict__ scratch) {
   __shared__ __align__(16) uint8_t stage[STAGE_ROWS * ROW_BYTES];
   const int row = blockIdx.x;
   const QueryInfo qi = locate(cu_q, cu_k, seqlens, S, row, nullptr);
   if (!qi.ok) return;
   const int32_t *blkrow = blk + (size_t)row * m;
-  const int nsel = count_selected(blkrow, m);
+  const int nsel = min(m, qi.pos / BLK + 1);  // the block stage keeps exactly this many
   const int s0 = blockIdx.y * slots_per_cta, s1 = min(nsel, s0 + slots_per_cta);
   if (s0 >= s1) return;
   QRegs qr;
   load_q(qr, q + (size_t)row * D);
-  uint32_t *dst = scratch + (size_t)row * m * BLK;
+  float *dst = scratch + (size_t)row * m * BLK;
   score_slots(qr, k + (size_t)qi.kbase * D, qi.pos, blkrow, s0, s1, stage,
-              [&](int c, uint32_t key) { dst[c] = key; });
+              [&](int c, float sc) { dst[c] = sc; });
 }
 
 // One CTA per query: exact top-k of the query's score row.  NT threads hold KPT
@@ -123,7 +118,7 @@ template <int NT, int KPT>
 __global__ void __launch_bounds__(NT, 1024 / NT)
 token_select_scratch_kernel(const int32_t *__restrict__ cu_q, const int32_t *__restrict__ cu_k,
                             const int32_t *__restrict__ seqlens, int S, int m, int topk,
-                            const int32_t *__restrict__ blk, const uint32_t *__restrict__ scratch,
+                            const int32_t *__restrict__ blk, const float *__restrict__ scratch,
                             int32_t *__restrict__ out_idx, float *__restrict__ out_scores) {
   extern __shared__ __align__(16) uint8_t smem[];
   uint32_t *work = reinterpret_cast<uint32_t *>(smem);
@@ -154,7 +149,7 @@ size_t block_tc_workspace_bytes(int total_q, int num_seqs, int max_seqlen_k);
 cudaError_t launch_token_score_tc(const uint16_t *q, const uint16_t *k, const int32_t *cu_q,
                                   const int32_t *cu_k, const int32_t *seqlens, int S,
                                   int total_q, int max_seqlen_k, int m, const int32_t *blk,
-                                  uint8_t *ws, uint32_t **scores_out, int num_sms, int *status,
+                                  uint8_t *ws, float **scores_out, int num_sms, int *status,
                                   cudaStream_t st);
 
 size_t token_scratch_bytes(int total_q, int num_seqs, int max_seqlen_k, int m, int num_sms) {
@@ -172,7 +167,7 @@ cudaError_t launch_token_select(const uint16_t *q, const uint16_t *k, const int3
                                 int *status, cudaStream_t st) {
   if (total_q == 0) return cudaSuccess;
   cudaError_t e;
-  uint32_t *scores = reinterpret_cast<uint32_t *>(ws);
+  float *scores = reinterpret_cast<float *>(ws);
   if (token_use_split(total_q, num_sms)) {
     // spread each query's blocks over enough CTAs to cover the SMs about twice
     int splits = (2 * num_sms + total_q - 1) / total_q;
@@ -192,7 +187,23 @@ cudaError_t launch_token_select(const uint16_t *q, const uint16_t *k, const int3
     if (e != cudaSuccess) return e;
   }
   const size_t smem = token_smem_bytes(m, topk);
-  if (m * BLK <= 256 * 32) {
+  if (token_use_split(total_q, num_sms)) {
+    // few queries: a wider CTA per query shortens each selection
+    static int attr_c[64], attr_d[64];
+    if (m * BLK <= 1024 * 8) {
+      auto kern = token_select_scratch_kernel<1024, 8>;
+      if ((e = set_smem_once((const void *)kern, smem, attr_c)) != cudaSuccess) return e;
+      ProfScope ps(K_TOKEN_SELECT_SCRATCH, st);
+      kern<<<total_q, 1024, smem, st>>>(cu_q, cu_k, seqlens, S, m, topk, blk, scores, out_idx,
+                                        out_scores);
+    } else {
+      auto kern = token_select_scratch_kernel<1024, 16>;
+      if ((e = set_smem_once((const void *)kern, smem, attr_d)) != cudaSuccess) return e;
+      ProfScope ps(K_TOKEN_SELECT_SCRATCH, st);
+      kern<<<total_q, 1024, smem, st>>>(cu_q, cu_k, seqlens, S, m, topk, blk, scores, out_idx,
+                                        out_scores);
+    }
+  } else if (m * BLK <= 256 * 32) {
     static int attr_a[64];
     auto kern = token_select_scratch_kernel<256, 32>;
     if ((e = set_smem_once((const void *)kern, smem, attr_a)) != cudaSuccess) return e;

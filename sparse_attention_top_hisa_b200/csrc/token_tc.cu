@@ -120,7 +120,7 @@ token_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const uint16_t *
                       const int32_t *__restrict__ cu_k, const int32_t *__restrict__ seqlens,
                       int emax, int m, const TileDesc *__restrict__ tiles,
                       const int *__restrict__ ntiles_ptr, const uint32_t *__restrict__ list,
-                      uint32_t *__restrict__ scratch, int *status) {
+                      float *__restrict__ scratch, int *status) {
   extern __shared__ uint8_t tc_smem_raw[];
   TcSmem &sm = *reinterpret_cast<TcSmem *>((reinterpret_cast<uintptr_t>(tc_smem_raw) + 1023) &
                                            ~(uintptr_t)1023);
@@ -206,8 +206,9 @@ token_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const uint16_t *
         if (c0 + u < n) {
           const uint32_t e = sm.ent[c0 + u];
           const int row = (int)(e >> 7), slot = (int)(e & 127u);
-          const uint32_t key = (j <= row + pos_off) ? score_key(__uint_as_float(v[u])) : 0u;
-          scratch[(size_t)row * row_stride + (size_t)slot * BLK + r] = key;
+          // raw score; -inf marks a key after the query
+          scratch[(size_t)row * row_stride + (size_t)slot * BLK + r] =
+              (j <= row + pos_off) ? __uint_as_float(v[u]) : -__int_as_float(0x7f800000);
         }
       }
     }
@@ -295,7 +296,7 @@ size_t tc_workspace_bytes(int total_q, int num_seqs, int max_seqlen_k, int m) {
 cudaError_t launch_token_score_tc(const uint16_t *q, const uint16_t *k, const int32_t *cu_q,
                                   const int32_t *cu_k, const int32_t *seqlens, int S,
                                   int total_q, int max_seqlen_k, int m, const int32_t *blk,
-                                  uint8_t *ws, uint32_t **scores_out, int num_sms, int *status,
+                                  uint8_t *ws, float **scores_out, int num_sms, int *status,
                                   cudaStream_t st) {
   const TcPlan p = tc_plan(total_q, S, max_seqlen_k, m);
   const int emax = (max_seqlen_k + BLK - 1) / BLK;
@@ -304,7 +305,7 @@ cudaError_t launch_token_score_tc(const uint16_t *q, const uint16_t *k, const in
   int *ntiles = reinterpret_cast<int *>(ws + p.off_ntiles);
   TileDesc *tiles = reinterpret_cast<TileDesc *>(ws + p.off_tiles);
   uint32_t *list = reinterpret_cast<uint32_t *>(ws + p.off_list);
-  uint32_t *scores = reinterpret_cast<uint32_t *>(ws + p.off_scores);
+  float *scores = reinterpret_cast<float *>(ws + p.off_scores);
   *scores_out = scores;
   CUtensorMap kmap;
   if (!make_key_tensor_map(&kmap, k)) return cudaErrorInvalidValue;
