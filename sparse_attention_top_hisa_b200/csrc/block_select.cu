@@ -38,42 +38,98 @@ __device__ __forceinline__ float rep_score(const QRegs &q, const float *rep) {
   return a + b;
 }
 
+// Key T of the mfree-th best free block and how many blocks with key == T are
+// still needed, by a radix select over 8-bit digits (most significant first) with a
+// per-warp histogram of 256 bins in shared memory.  keys[b] == 0 marks a block that
+// is not free (forced, or after the query).  Executed by one full warp; `hist0`, if
+// not null, already holds the histogram of the top digit of keys[0..E).
+__device__ void warp_radix_threshold(const uint32_t *keys, int E, int mfree, uint32_t *hist,
+                                     bool hist0_ready, uint32_t &T_out, int &need_eq_out) {
+  const int lane = threadIdx.x & 31;
+  uint32_t prefix = 0u, pmask = 0u;
+  int remaining = mfree;
+#pragma unroll 1
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    if (!(shift == 24 && hist0_ready)) {
+#pragma unroll
+      for (int i = 0; i < 8; i++) hist[lane * 8 + i] = 0u;
+      __syncwarp();
+      for (int b = lane; b < E; b += 32) {
+        const uint32_t u = keys[b];
+        if (u != 0u && (u & pmask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], 1u);
+      }
+      __syncwarp();
+    }
+    // lane l owns bins 255 - 8l .. 248 - 8l (highest digits first)
+    int h[8], local = 0;
+#pragma unroll
+    for (int i = 0; i < 8; i++) {
+      h[i] = (int)hist[255 - lane * 8 - i];
+      local += h[i];
+    }
+    int incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const int excl = incl - local;
+    // the lane whose range holds the remaining-th key
+    const unsigned who = __ballot_sync(0xffffffffu, excl < remaining && incl >= remaining);
+    const int src = __ffs(who) - 1;
+    int digit = 0, above = 0, inbin = 0;
+    if (lane == src) {
+      int run = excl;
+#pragma unroll
+      for (int i = 0; i < 8; i++) {
+        if (run < remaining && run + h[i] >= remaining) {
+          digit = 255 - lane * 8 - i;
+          above = run;
+          inbin = h[i];
+        }
+        run += h[i];
+      }
+    }
+    digit = __shfl_sync(0xffffffffu, digit, src);
+    above = __shfl_sync(0xffffffffu, above, src);
+    inbin = __shfl_sync(0xffffffffu, inbin, src);
+    __syncwarp();
+    remaining -= above;
+    prefix |= (uint32_t)digit << shift;
+    pmask |= 255u << shift;
+    if (inbin == remaining) {  // the whole bin is selected
+      T_out = prefix ? prefix - 1u : 0u;
+      need_eq_out = 0;
+      return;
+    }
+  }
+  T_out = prefix;
+  need_eq_out = remaining;
+}
+
 // Top-(m - |forced|) of the keys[0..E) of one query (forced blocks and blocks after
 // the query hold key 0), written in ascending block order with the forced blocks.
 // Executed by one full warp.
 __device__ void warp_select_blocks(const uint32_t *keys, int E, int own, int m,
-                                   int32_t *dst, int32_t *dst2) {
+                                   int32_t *dst, int32_t *dst2, uint32_t *hist,
+                                   bool hist0_ready) {
   const int lane = threadIdx.x & 31;
   const int nf = min(m, 3);  // forced: own, previous, first (E > m >= 3 makes them distinct)
   const int mfree = m - nf;
   auto forced = [&](int b) {
     return b == own || (nf >= 2 && b == own - 1) || (nf >= 3 && b == 0);
   };
-  // T = key of the mfree-th best free block (0 if none are needed)
-  uint32_t T = 0u;
-  if (mfree > 0) {
-    for (int bit = 31; bit >= 0; bit--) {
-      const uint32_t cand = T | (1u << bit);
-      int cnt = 0;
-      for (int b = lane; b < E; b += 32) cnt += keys[b] >= cand;
-      cnt = __reduce_add_sync(0xffffffffu, cnt);
-      if (cnt >= mfree) T = cand;
-    }
-  }
-  int ngt = 0;
-  if (mfree > 0) {
-    for (int b = lane; b < E; b += 32) ngt += keys[b] > T;
-    ngt = __reduce_add_sync(0xffffffffu, ngt);
-  }
-  const int need_eq = mfree - ngt;
+  uint32_t T = 0xffffffffu;  // nothing free is taken when mfree == 0
+  int need_eq = 0;
+  if (mfree > 0) warp_radix_threshold(keys, E, mfree, hist, hist0_ready, T, need_eq);
   const unsigned lt = (1u << lane) - 1u;
   int eqr = 0, outp = 0;
   for (int b0 = 0; b0 < E; b0 += 32) {
     const int b = b0 + lane;
     const uint32_t u = b < E ? keys[b] : 0u;
-    const bool is_eq = mfree > 0 && u != 0u && u == T;
+    const bool is_eq = need_eq > 0 && u != 0u && u == T;
     const unsigned beq = __ballot_sync(0xffffffffu, is_eq);
-    const bool sel = (b < E && forced(b)) || (mfree > 0 && u > T) ||
+    const bool sel = (b < E && forced(b)) || (mfree > 0 && u != 0u && u > T) ||
                      (is_eq && eqr + __popc(beq & lt) < need_eq);
     const unsigned bsel = __ballot_sync(0xffffffffu, sel);
     if (sel) {
@@ -137,7 +193,8 @@ block_select_kernel(const int32_t *__restrict__ cu_q, const int32_t *__restrict_
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * BS_WARPS + warp;
   if (row >= total_q) return;
-  uint32_t *keys = bs_smem + (size_t)warp * emax;
+  uint32_t *hist = bs_smem + (size_t)warp * 256;
+  uint32_t *keys = bs_smem + BS_WARPS * 256 + (size_t)warp * emax;
   int32_t *dst = blk + (size_t)row * m;
   int32_t *dst2 = out_blocks ? out_blocks + (size_t)row * m : nullptr;
   QueryInfo qi;
@@ -146,9 +203,16 @@ block_select_kernel(const int32_t *__restrict__ cu_q, const int32_t *__restrict_
                        32))
     return;
   const uint32_t *src = tc_keys + (size_t)row * tc_stride;
-  for (int b = lane; b < E; b += 32) keys[b] = __ldg(src + b);
+#pragma unroll
+  for (int i = 0; i < 8; i++) hist[lane * 8 + i] = 0u;
   __syncwarp();
-  warp_select_blocks(keys, E, own, m, dst, dst2);
+  for (int b = lane; b < E; b += 32) {
+    const uint32_t u = __ldg(src + b);
+    keys[b] = u;
+    if (u != 0u) atomicAdd(&hist[u >> 24], 1u);
+  }
+  __syncwarp();
+  warp_select_blocks(keys, E, own, m, dst, dst2, hist, true);
 }
 
 // Few queries (decode): one CTA per query scores every eligible block on the CUDA
@@ -177,10 +241,10 @@ block_select_cta_kernel(const uint16_t *__restrict__ q, const float *__restrict_
   const float *rbase = reps + (size_t)(qi.kbase / BLK) * D;
   for (int b = tid; b < E; b += BS_CTA_THREADS) {
     const bool forced = b == own || (nf >= 2 && b == own - 1) || (nf >= 3 && b == 0);
-    bsc_smem[b] = forced ? 0u : score_key(rep_score(qr, rbase + (size_t)b * D));
+    bsc_smem[256 + b] = forced ? 0u : score_key(rep_score(qr, rbase + (size_t)b * D));
   }
   __syncthreads();
-  if (tid < 32) warp_select_blocks(bsc_smem, E, own, m, dst, dst2);
+  if (tid < 32) warp_select_blocks(bsc_smem + 256, E, own, m, dst, dst2, bsc_smem, false);
 }
 
 bool use_tc_path(int total_q, int num_sms);
@@ -210,7 +274,7 @@ cudaError_t launch_block_select(const uint16_t *q, const float *reps, const int3
   }
   const int emax = (max_seqlen_k + BLK - 1) / BLK;
   if (tc_keys) {
-    const size_t smem = (size_t)BS_WARPS * (emax > 0 ? emax : 1) * sizeof(uint32_t);
+    const size_t smem = (size_t)BS_WARPS * (256 + (emax > 0 ? emax : 1)) * sizeof(uint32_t);
     static int attr[64];
     if (smem > 48 * 1024) {
       cudaError_t e = set_smem_once((const void *)block_select_kernel, smem, attr);
@@ -222,7 +286,7 @@ cudaError_t launch_block_select(const uint16_t *q, const float *reps, const int3
                                                          emax > 0 ? emax : 1, tc_keys, tc_stride,
                                                          blk, out_blocks, status);
   } else {
-    const size_t smem = (size_t)(emax > 0 ? emax : 1) * sizeof(uint32_t);
+    const size_t smem = (size_t)(256 + (emax > 0 ? emax : 1)) * sizeof(uint32_t);
     static int attr_cta[64];
     if (smem > 48 * 1024) {
       cudaError_t e = set_smem_once((const void *)block_select_cta_kernel, smem, attr_cta);

@@ -52,30 +52,70 @@ static_assert(sizeof(TcSmem) + 1024 <= TC_SMEM_BYTES, "tile does not fit");
 // ---------------------------------------------------------------------------
 // inverted lists
 
-// mode 0: count pairs per compact key block; mode 1: write them into the lists.
-__global__ void __launch_bounds__(256)
+// The (query, slot) pairs of a range of INV_ROWS consecutive query rows are first
+// aggregated per compact key block in shared memory, so that global atomics are
+// issued once per (CTA, key block) instead of once per pair.  A CTA whose rows span
+// more compact blocks than fit in shared memory uses global atomics directly.
+//   mode 0: add the pair counts of every key block to cnt;
+//   mode 1: reserve each key block's share of its list (cursor holds the list
+//           starts) and write the entries row << 7 | slot.
+constexpr int INV_THREADS = 256;
+constexpr int INV_ROWS = 256;
+constexpr int INV_LOCAL_BINS = 8192;
+
+__global__ void __launch_bounds__(INV_THREADS)
 inv_lists_kernel(const int32_t *__restrict__ blk, int total_q, int m,
                  const int32_t *__restrict__ cu_q, int S, int emax, int mode,
                  int *__restrict__ cnt, int *__restrict__ cursor, uint32_t *__restrict__ list) {
-  const int lane = threadIdx.x & 31;
-  const int row = ((blockIdx.x * blockDim.x + threadIdx.x) >> 5) * 32 + lane;
-  const bool valid = row < total_q;
-  const int s = valid ? find_seq(cu_q, S, row) : 0;
-  const unsigned lt = (1u << lane) - 1u;
-  for (int slot = 0; slot < m; slot++) {
-    const int b = valid ? __ldg(blk + (size_t)row * m + slot) : -1;
-    const int key = b >= 0 ? s * emax + b : -1;
-    const unsigned peers = __match_any_sync(0xffffffffu, key);
-    const int leader = __ffs(peers) - 1;
-    if (mode == 0) {
-      if (key >= 0 && lane == leader) atomicAdd(cnt + key, __popc(peers));
-    } else {
-      int base = 0;
-      if (key >= 0 && lane == leader) base = atomicAdd(cursor + key, __popc(peers));
-      base = __shfl_sync(0xffffffffu, base, leader);
-      if (key >= 0) list[base + __popc(peers & lt)] = ((uint32_t)row << 7) | (uint32_t)slot;
-    }
+  __shared__ int loc[INV_LOCAL_BINS];
+  __shared__ int seq_range[2];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  constexpr int NW = INV_THREADS / 32;
+  const int r0 = blockIdx.x * INV_ROWS, r1 = min(total_q, r0 + INV_ROWS);
+  if (tid == 0) {
+    seq_range[0] = find_seq(cu_q, S, r0);
+    seq_range[1] = find_seq(cu_q, S, r1 - 1);
   }
+  __syncthreads();
+  const int s0 = seq_range[0], s1 = seq_range[1];
+  const int base = s0 * emax;
+  const int nbl = (s1 - s0 + 1) * emax;
+  const bool local = nbl <= INV_LOCAL_BINS;
+  // walk the pairs: warp w takes rows r0 + w, r0 + w + NW, ...; lane = slot
+  auto walk = [&](auto &&fn) {
+    int s = s0;
+    for (int row = r0 + warp; row < r1; row += NW) {
+      while (s < s1 && __ldg(cu_q + s + 1) <= row) s++;
+      for (int slot = lane; slot < m; slot += 32) {
+        const int b = __ldg(blk + (size_t)row * m + slot);
+        if (b >= 0) fn(row, slot, s * emax + b);
+      }
+    }
+  };
+  if (!local) {  // wide row range: global atomics per pair
+    if (mode == 0)
+      walk([&](int, int, int cb) { atomicAdd(cnt + cb, 1); });
+    else
+      walk([&](int row, int slot, int cb) {
+        list[atomicAdd(cursor + cb, 1)] = ((uint32_t)row << 7) | (uint32_t)slot;
+      });
+    return;
+  }
+  for (int i = tid; i < nbl; i += INV_THREADS) loc[i] = 0;
+  __syncthreads();
+  walk([&](int, int, int cb) { atomicAdd(&loc[cb - base], 1); });
+  __syncthreads();
+  if (mode == 0) {
+    for (int i = tid; i < nbl; i += INV_THREADS)
+      if (loc[i]) atomicAdd(cnt + base + i, loc[i]);
+    return;
+  }
+  for (int i = tid; i < nbl; i += INV_THREADS)
+    if (loc[i]) loc[i] = atomicAdd(cursor + base + i, loc[i]);
+  __syncthreads();
+  walk([&](int row, int slot, int cb) {
+    list[atomicAdd(&loc[cb - base], 1)] = ((uint32_t)row << 7) | (uint32_t)slot;
+  });
 }
 
 constexpr int SCAN_THREADS = 1024;
@@ -311,11 +351,10 @@ cudaError_t launch_token_score_tc(const uint16_t *q, const uint16_t *k, const in
   if (!make_key_tensor_map(&kmap, k)) return cudaErrorInvalidValue;
   cudaError_t e = cudaMemsetAsync(cnt, 0, (size_t)p.nb * 4, st);
   if (e != cudaSuccess) return e;
-  const int warps = (total_q + 31) / 32;
-  const int grid = (warps + 7) / 8;
+  const int grid = (total_q + INV_ROWS - 1) / INV_ROWS;
   {
     ProfScope ps(K_INV_LISTS, st);
-    inv_lists_kernel<<<grid, 256, 0, st>>>(blk, total_q, m, cu_q, S, emax, 0, cnt, cursor, list);
+    inv_lists_kernel<<<grid, INV_THREADS, 0, st>>>(blk, total_q, m, cu_q, S, emax, 0, cnt, cursor, list);
   }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   {
@@ -325,7 +364,7 @@ cudaError_t launch_token_score_tc(const uint16_t *q, const uint16_t *k, const in
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   {
     ProfScope ps(K_INV_LISTS, st);
-    inv_lists_kernel<<<grid, 256, 0, st>>>(blk, total_q, m, cu_q, S, emax, 1, cnt, cursor, list);
+    inv_lists_kernel<<<grid, INV_THREADS, 0, st>>>(blk, total_q, m, cu_q, S, emax, 1, cnt, cursor, list);
   }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   static int attr[64];
