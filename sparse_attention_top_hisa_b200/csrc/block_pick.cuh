@@ -1,0 +1,122 @@
+// Top-m block choice of HISA stage 1 for one query, executed by one warp.
+//
+// HISA summary page (aitrends.kr), paragraph on stage 1: the first block and the
+// last two blocks (read as the query's own block and the one before it) are always
+// kept and count inside m; the rest of the m slots go to the best-scoring eligible
+// blocks, ties to the lower block.  The scores arrive as order-preserving keys
+// (0 = forced or not eligible).
+#pragma once
+
+#include "common.cuh"
+
+namespace hisa {
+
+// Key T of the mfree-th best free block and how many blocks with key == T are
+// still needed, by a radix select over 8-bit digits (most significant first) with a
+// per-warp histogram of 256 bins in shared memory.  keys[b] == 0 marks a block that
+// is not free (forced, or after the query).  Executed by one full warp; `hist0`, if
+// not null, already holds the histogram of the top digit of keys[0..E).
+__device__ __forceinline__ void warp_radix_threshold(const uint32_t *keys, int E, int mfree, uint32_t *hist,
+                                     bool hist0_ready, uint32_t &T_out, int &need_eq_out) {
+  const int lane = threadIdx.x & 31;
+  uint32_t prefix = 0u, pmask = 0u;
+  int remaining = mfree;
+#pragma unroll 1
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    if (!(shift == 24 && hist0_ready)) {
+#pragma unroll
+      for (int i = 0; i < 8; i++) hist[lane * 8 + i] = 0u;
+      __syncwarp();
+      for (int b = lane; b < E; b += 32) {
+        const uint32_t u = keys[b];
+        if (u != 0u && (u & pmask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], 1u);
+      }
+      __syncwarp();
+    }
+    // lane l owns bins 255 - 8l .. 248 - 8l (highest digits first)
+    int h[8], local = 0;
+#pragma unroll
+    for (int i = 0; i < 8; i++) {
+      h[i] = (int)hist[255 - lane * 8 - i];
+      local += h[i];
+    }
+    int incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const int excl = incl - local;
+    // the lane whose range holds the remaining-th key
+    const unsigned who = __ballot_sync(0xffffffffu, excl < remaining && incl >= remaining);
+    const int src = __ffs(who) - 1;
+    int digit = 0, above = 0, inbin = 0;
+    if (lane == src) {
+      int run = excl;
+#pragma unroll
+      for (int i = 0; i < 8; i++) {
+        if (run < remaining && run + h[i] >= remaining) {
+          digit = 255 - lane * 8 - i;
+          above = run;
+          inbin = h[i];
+        }
+        run += h[i];
+      }
+    }
+    digit = __shfl_sync(0xffffffffu, digit, src);
+    above = __shfl_sync(0xffffffffu, above, src);
+    inbin = __shfl_sync(0xffffffffu, inbin, src);
+    __syncwarp();
+    remaining -= above;
+    prefix |= (uint32_t)digit << shift;
+    pmask |= 255u << shift;
+    if (inbin == remaining) {  // the whole bin is selected
+      T_out = prefix ? prefix - 1u : 0u;
+      need_eq_out = 0;
+      return;
+    }
+  }
+  T_out = prefix;
+  need_eq_out = remaining;
+}
+
+// Top-(m - |forced|) of the keys[0..E) of one query (forced blocks and blocks after
+// the query hold key 0), written in ascending block order with the forced blocks.
+// Executed by one full warp.
+__device__ __forceinline__ void warp_select_blocks(const uint32_t *keys, int E, int own, int m,
+                                   int32_t *dst, int32_t *dst2, uint32_t *hist,
+                                   bool hist0_ready) {
+  const int lane = threadIdx.x & 31;
+  const int nf = min(m, 3);  // forced: own, previous, first (E > m >= 3 makes them distinct)
+  const int mfree = m - nf;
+  auto forced = [&](int b) {
+    return b == own || (nf >= 2 && b == own - 1) || (nf >= 3 && b == 0);
+  };
+  uint32_t T = 0xffffffffu;  // nothing free is taken when mfree == 0
+  int need_eq = 0;
+  if (mfree > 0) warp_radix_threshold(keys, E, mfree, hist, hist0_ready, T, need_eq);
+  const unsigned lt = (1u << lane) - 1u;
+  int eqr = 0, outp = 0;
+  for (int b0 = 0; b0 < E; b0 += 32) {
+    const int b = b0 + lane;
+    const uint32_t u = b < E ? keys[b] : 0u;
+    const bool is_eq = need_eq > 0 && u != 0u && u == T;
+    const unsigned beq = __ballot_sync(0xffffffffu, is_eq);
+    const bool sel = (b < E && forced(b)) || (mfree > 0 && u != 0u && u > T) ||
+                     (is_eq && eqr + __popc(beq & lt) < need_eq);
+    const unsigned bsel = __ballot_sync(0xffffffffu, sel);
+    if (sel) {
+      const int p = outp + __popc(bsel & lt);
+      dst[p] = b;
+      if (dst2) dst2[p] = b;
+    }
+    eqr += __popc(beq);
+    outp += __popc(bsel);
+  }
+  for (int i = outp + lane; i < m; i += 32) {  // only reachable if fewer than m exist
+    dst[i] = -1;
+    if (dst2) dst2[i] = -1;
+  }
+}
+
+}  // namespace hisa

@@ -252,13 +252,17 @@ namespace hisa {
 // the radix routine above instead, reading the scores again.
 
 constexpr int LIN_BINS = 2048;
+// Bucket b lives at word b + b / 32 of the count arrays: a thread scanning eight
+// consecutive buckets then touches 32 distinct banks across its warp.
+constexpr int LIN_WORDS = LIN_BINS + LIN_BINS / 32;
+__device__ __forceinline__ int lin_slot(int b) { return b + (b >> 5); }
 
 struct LinShared {
   union {
     SelectShared radix;
     struct {
-      uint32_t cnt[LIN_BINS];
-      uint32_t off[LIN_BINS];
+      uint32_t cnt[LIN_WORDS];
+      uint32_t off[LIN_WORDS];
       int warp_tot[33];
       int wn[32];
       float wmx[32], wmn[32];
@@ -328,7 +332,7 @@ __device__ void select_topk_reg(const float *sc, int n, int k, LinShared &sh, ui
     sh.lin.wmn[warp] = mn;
     sh.lin.wn[warp] = nv;
   }
-  for (int i = tid; i < LIN_BINS; i += NT) sh.lin.cnt[i] = 0u;
+  for (int i = tid; i < LIN_WORDS; i += NT) sh.lin.cnt[i] = 0u;
   __syncthreads();
   mx = NEG;
   mn = -NEG;
@@ -347,16 +351,20 @@ __device__ void select_topk_reg(const float *sc, int n, int k, LinShared &sh, ui
   // 2. histogram
 #pragma unroll
   for (int i = 0; i < KPT; i++)
-    if (f[i] != NEG) atomicAdd(&sh.lin.cnt[lin_bucket(f[i], smax, inv)], 1u);
+    if (f[i] != NEG) atomicAdd(&sh.lin.cnt[lin_slot(lin_bucket(f[i], smax, inv))], 1u);
   __syncthreads();
 
   // 3. offsets and the boundary bucket
   const int kp = min(k, nvalid);
   {
     constexpr int per = LIN_BINS / NT;
+    uint32_t h[per];
     int local = 0;
 #pragma unroll
-    for (int i = 0; i < per; i++) local += (int)sh.lin.cnt[tid * per + i];
+    for (int i = 0; i < per; i++) {
+      h[i] = sh.lin.cnt[lin_slot(tid * per + i)];
+      local += (int)h[i];
+    }
     int total;
     int run = block_exclusive_scan<NT>(local, sh.lin.warp_tot, &total);
     if (tid == 0) {
@@ -368,14 +376,13 @@ __device__ void select_topk_reg(const float *sc, int n, int k, LinShared &sh, ui
 #pragma unroll
     for (int i = 0; i < per; i++) {
       const int b = tid * per + i;
-      const int h = (int)sh.lin.cnt[b];
-      if (nvalid > k && run < k && run + h >= k) {
+      if (nvalid > k && run < k && run + (int)h[i] >= k) {
         sh.lin.misc[3] = (uint32_t)b;
         sh.lin.misc[4] = (uint32_t)run;
       }
-      sh.lin.off[b] = (uint32_t)run;
-      sh.lin.cnt[b] = (uint32_t)run;  // becomes the scatter cursor
-      run += h;
+      sh.lin.off[lin_slot(b)] = (uint32_t)run;
+      sh.lin.cnt[lin_slot(b)] = (uint32_t)run;  // becomes the scatter cursor
+      run += (int)h[i];
     }
   }
   __syncthreads();
@@ -389,7 +396,7 @@ __device__ void select_topk_reg(const float *sc, int n, int k, LinShared &sh, ui
     if (f[i] != NEG) {
       const int b = lin_bucket(f[i], smax, inv);
       if (b < bstar) {
-        const uint32_t slot = atomicAdd(&sh.lin.cnt[b], 1u);
+        const uint32_t slot = atomicAdd(&sh.lin.cnt[lin_slot(b)], 1u);
         surv[slot] = rank_key(f[i], cand(i));
       } else if (b == bstar) {
         const uint32_t e = atomicAdd(&sh.lin.misc[5], 1u);
@@ -423,7 +430,7 @@ __device__ void select_topk_reg(const float *sc, int n, int k, LinShared &sh, ui
   for (int s = tid; s < above; s += NT) {
     const uint64_t me = surv[s];
     const int b = lin_bucket(key_score((uint32_t)(me >> 32)), smax, inv);
-    const int st = (int)sh.lin.off[b], en = (int)sh.lin.cnt[b];
+    const int st = (int)sh.lin.off[lin_slot(b)], en = (int)sh.lin.cnt[lin_slot(b)];
     int rank = 0;
     for (int t = st; t < en; t++) rank += surv[t] > me;
     out(st + rank, (int)~(uint32_t)me, (uint32_t)(me >> 32));

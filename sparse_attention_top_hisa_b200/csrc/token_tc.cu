@@ -11,12 +11,17 @@
 //      key block, with warp-aggregated atomics (block 0 is selected by every query);
 //   2. inv_scan_kernel: list offsets per key block and tile descriptors (one tile =
 //      one key block and up to 256 of its selecting queries);
-//   3. token_score_tc_kernel: persistent CTAs; per tile the key block arrives by TMA
-//      (or by guarded cp.async when it is the partial last block of a sequence), the
-//      selecting queries are gathered with cp.async into the 128-byte-swizzled
-//      K-major layout, one thread issues four tcgen05.mma (K = 4 x 16) into a
-//      128 x N fp32 accumulator in TMEM, and four warps move it out (warp w owns
-//      TMEM lanes 32w..32w+31, i.e. key rows) into each query's score row;
+//   3. token_score_tc_kernel: persistent, warp-specialised CTAs (one per SM).  Per
+//      tile the key block arrives by TMA (or by cp.async when it is the partial last
+//      block of a sequence) and the selecting queries are gathered with cp.async into
+//      the 128-byte-swizzled K-major layout, through a three-stage shared-memory ring
+//      filled by three loader warps.  One thread issues the tcgen05.mma chain
+//      S = K_b [128 x 64] . Q_sel^T [64 x N] (K = 4 x 16, N <= 256) into one of two
+//      TMEM accumulators, so that the loads, the MMAs and the epilogue of
+//      consecutive tiles overlap.  The accumulator lane is the key row: each of the
+//      eight epilogue warps owns 32 key rows (TMEM lane quarter w % 4) of half of the
+//      queries (w / 4), and every store instruction writes the 32 consecutive scores
+//      of one query (one 128-byte line of its score row);
 //   4. the exact select of token_select.cu reads the score rows.
 // Key j of block b is admitted for a query at position i only when j <= i.
 #include <cudaTypedefs.h>
@@ -26,9 +31,7 @@
 
 namespace hisa {
 
-constexpr int TC_N = 256;          // selecting queries per tile (MMA N, at most)
-constexpr int TC_THREADS = 128;    // four warps, one TMEM lane quarter each
-constexpr uint32_t TC_TMEM_COLS = 256;
+constexpr int TC_N = 256;  // selecting queries per tile (two MMA chains of M = 128, at most)
 
 struct TileDesc {
   int list_off;  // first list entry of the tile
@@ -37,17 +40,23 @@ struct TileDesc {
   int pad;
 };
 
+constexpr int TC_STAGES = 3;       // shared-memory ring depth
+constexpr int TC_EPI_WARPS = 8;    // epilogue: warp w owns TMEM lanes 32 (w % 4).., queries half w / 4
+constexpr int TC_MMA_WARP = TC_EPI_WARPS;
+constexpr int TC_LOAD_WARP0 = TC_EPI_WARPS + 1;
+constexpr int TC_LOAD_WARPS = 3;
+constexpr int TC_LOADERS = TC_LOAD_WARPS * 32;
+constexpr int TC_THREADS = (TC_EPI_WARPS + 1 + TC_LOAD_WARPS) * 32;
+constexpr uint32_t TC_TMEM_COLS = 512;  // two accumulators of 256 columns
+
 struct TcSmem {
-  uint8_t a[BLK * ROW_BYTES];   // key block, 1024-byte aligned
-  uint8_t b[TC_N * ROW_BYTES];  // gathered queries, 1024-byte aligned
-  uint32_t ent[TC_N];
-  uint64_t bar_tma;
-  uint64_t bar_mma;
+  uint8_t q[TC_STAGES][TC_N * ROW_BYTES];  // gathered queries (MMA B), 1024-byte aligned
+  uint8_t k[TC_STAGES][BLK * ROW_BYTES];   // key block (MMA A)
+  uint64_t full[TC_STAGES], empty[TC_STAGES], acc_full[2], acc_empty[2];
   uint32_t tmem_base;
+  int abort;
 };
-// request enough shared memory that at most two CTAs share an SM (2 x 256 TMEM columns)
-constexpr size_t TC_SMEM_BYTES = 110 * 1024;
-static_assert(sizeof(TcSmem) + 1024 <= TC_SMEM_BYTES, "tile does not fit");
+constexpr size_t TC_SMEM_BYTES = sizeof(TcSmem) + 1024;
 
 // ---------------------------------------------------------------------------
 // inverted lists
@@ -154,6 +163,22 @@ inv_scan_kernel(const int *__restrict__ cnt, int nb, int *__restrict__ cursor,
 // ---------------------------------------------------------------------------
 // tensor-core scoring
 
+struct TileSeq {
+  int b, kbase, len, pos_off;  // key block, region start, live keys, position = row + pos_off
+};
+
+__device__ __forceinline__ TileSeq tile_seq(const TileDesc &td, int emax, const int32_t *cu_q,
+                                            const int32_t *cu_k, const int32_t *seqlens) {
+  TileSeq r;
+  const int s = td.cb / emax;
+  r.b = td.cb - s * emax;
+  r.kbase = __ldg(cu_k + s);
+  r.len = seqlens ? __ldg(seqlens + s) : __ldg(cu_k + s + 1) - r.kbase;
+  const int q0 = __ldg(cu_q + s);
+  r.pos_off = r.len - (__ldg(cu_q + s + 1) - q0) - q0;
+  return r;
+}
+
 __global__ void __launch_bounds__(TC_THREADS, 1)
 token_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const uint16_t *__restrict__ q,
                       const uint16_t *__restrict__ k, const int32_t *__restrict__ cu_q,
@@ -166,8 +191,15 @@ token_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const uint16_t *
                                            ~(uintptr_t)1023);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
-    mbar_init(&sm.bar_tma, 1);
-    mbar_init(&sm.bar_mma, 1);
+    for (int i = 0; i < TC_STAGES; i++) {
+      mbar_init(&sm.full[i], TC_LOADERS + 1);  // every loader thread + the key TMA issuer
+      mbar_init(&sm.empty[i], 1);
+    }
+    for (int i = 0; i < 2; i++) {
+      mbar_init(&sm.acc_full[i], 1);
+      mbar_init(&sm.acc_empty[i], TC_EPI_WARPS * 32);
+    }
+    sm.abort = 0;
     fence_barrier_init();
     prefetch_tmap(&kmap);
   }
@@ -179,81 +211,145 @@ token_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const uint16_t *
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
-  const uint32_t sa = smem_u32(sm.a), sb = smem_u32(sm.b);
   const int ntiles = *ntiles_ptr;
-  const size_t row_stride = (size_t)m * BLK;
-  uint32_t phase = 0;
-  for (int t = blockIdx.x; t < ntiles; t += gridDim.x, phase ^= 1u) {
-    const TileDesc td = tiles[t];
-    const int s = td.cb / emax, b = td.cb - (td.cb / emax) * emax;
-    const int kbase = __ldg(cu_k + s);
-    const int len = seqlens ? __ldg(seqlens + s) : __ldg(cu_k + s + 1) - kbase;
-    const int q0 = __ldg(cu_q + s);
-    const int pos_off = len - (__ldg(cu_q + s + 1) - q0) - q0;  // position = row + pos_off
-    const int n = td.n;
-    const int npad = (n + 15) & ~15;
-    for (int i = tid; i < n; i += TC_THREADS) sm.ent[i] = list[td.list_off + i];
-    __syncthreads();
-    // key block
-    const int live = len - b * BLK;
-    if (live >= BLK) {
-      if (tid == 0) {
-        mbar_arrive_expect_tx(&sm.bar_tma, BLK * ROW_BYTES);
-        tma_load_2d(sm.a, &kmap, &sm.bar_tma, 0, kbase + b * BLK);
+  volatile int *abort_flag = &sm.abort;
+
+  if (warp >= TC_LOAD_WARP0) {
+    // ---------------- loaders: key block (TMA or cp.async) and query gather ----------------
+    const int lt = tid - TC_LOAD_WARP0 * 32;
+    int i = 0;
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x, i++) {
+      const int s = i % TC_STAGES;
+      const TileDesc td = tiles[t];  // fetched while the stage drains
+      const TileSeq ts = tile_seq(td, emax, cu_q, cu_k, seqlens);
+      if (i >= TC_STAGES && !mbar_wait(&sm.empty[s], (uint32_t)(((i / TC_STAGES) & 1) ^ 1), status)) {
+        *abort_flag = 1;
+        break;
       }
-    } else {  // partial last block: load only the rows that exist
-      for (int i = tid; i < BLK * 8; i += TC_THREADS) {
-        const int r = i >> 3, c = i & 7;
-        if (r < live)
-          cp_async_16(sa + sw128_offset(r, c), k + (size_t)(kbase + b * BLK + r) * D + c * 8);
-        else
-          *reinterpret_cast<uint4 *>(sm.a + sw128_offset(r, c)) = make_uint4(0u, 0u, 0u, 0u);
-      }
-      if (tid == 0) mbar_arrive(&sm.bar_tma);
-    }
-    // the queries that selected the block
-    for (int i = tid; i < npad * 8; i += TC_THREADS) {
-      const int r = i >> 3, c = i & 7;
-      if (r < n)
-        cp_async_16(sb + sw128_offset(r, c), q + (size_t)(sm.ent[r] >> 7) * D + c * 8);
-      else
-        *reinterpret_cast<uint4 *>(sm.b + sw128_offset(r, c)) = make_uint4(0u, 0u, 0u, 0u);
-    }
-    cp_async_wait_all();
-    fence_proxy_async_smem();
-    __syncthreads();
-    if (tid == 0) {
-      mbar_wait(&sm.bar_tma, phase, status);
-      tc_fence_after();
-      const uint32_t id = idesc_bf16_f32(BLK, npad);
-#pragma unroll
-      for (int kk = 0; kk < 4; kk++)
-        umma_bf16(tmem, sdesc_k_sw128(sa + kk * 32), sdesc_k_sw128(sb + kk * 32), id, kk > 0);
-      umma_commit(&sm.bar_mma);
-    }
-    __syncwarp();
-    mbar_wait(&sm.bar_mma, phase, status);
-    tc_fence_after();
-    // epilogue: this thread owns key row r of the block
-    const int r = warp * 32 + lane;
-    const int j = b * BLK + r;
-    for (int c0 = 0; c0 < npad; c0 += 16) {
-      uint32_t v[16];
-      tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, v);
-      tmem_wait_ld();
-#pragma unroll
-      for (int u = 0; u < 16; u++) {
-        if (c0 + u < n) {
-          const uint32_t e = sm.ent[c0 + u];
-          const int row = (int)(e >> 7), slot = (int)(e & 127u);
-          // raw score; -inf marks a key after the query
-          scratch[(size_t)row * row_stride + (size_t)slot * BLK + r] =
-              (j <= row + pos_off) ? __uint_as_float(v[u]) : -__int_as_float(0x7f800000);
+      if (*abort_flag) break;
+      const int live = ts.len - ts.b * BLK;
+      const uint32_t sq = smem_u32(sm.q[s]), sk = smem_u32(sm.k[s]);
+      if (lt == 0) {
+        if (live >= BLK) {
+          mbar_arrive_expect_tx(&sm.full[s], BLK * ROW_BYTES);
+          tma_load_2d(sm.k[s], &kmap, &sm.full[s], 0, ts.kbase + ts.b * BLK);
+        } else {
+          mbar_arrive(&sm.full[s]);
         }
       }
+      if (live < BLK) {  // partial last block: only the rows that exist (the rest is masked)
+        for (int x = lt; x < live * 8; x += TC_LOADERS) {
+          const int r = x >> 3, c = x & 7;
+          cp_async_16(sk + sw128_offset(r, c), k + (size_t)(ts.kbase + ts.b * BLK + r) * D + c * 8);
+        }
+      }
+      // the selecting queries, in chunks of 32 rows (chunk c is loaded by loader warp
+      // c % TC_LOAD_WARPS): one coalesced read of the chunk's list entries, then lane l
+      // copies 16-byte piece l % 8 of row 4 i + l / 8 for i = 0..7.  Rows past n stay
+      // stale (their accumulator columns are ignored).
+      {
+        const int lw = lt >> 5;
+        constexpr int MAXC = (TC_N / 32 + TC_LOAD_WARPS - 1) / TC_LOAD_WARPS;
+        uint32_t ent[MAXC];
+#pragma unroll
+        for (int j = 0; j < MAXC; j++) {
+          const int row = (lw + j * TC_LOAD_WARPS) * 32 + lane;
+          ent[j] = row < td.n ? __ldg(list + td.list_off + row) : 0u;
+        }
+#pragma unroll
+        for (int j = 0; j < MAXC; j++) {
+          const int c = lw + j * TC_LOAD_WARPS;
+          if (c * 32 < td.n) {  // warp-uniform
+#pragma unroll
+            for (int i2 = 0; i2 < 8; i2++) {
+              const int rl = i2 * 4 + (lane >> 3), row = c * 32 + rl, piece = lane & 7;
+              const uint32_t e = __shfl_sync(0xffffffffu, ent[j], rl);
+              if (row < td.n)
+                cp_async_16(sq + sw128_offset(row, piece), q + (size_t)(e >> 7) * D + piece * 8);
+            }
+          }
+        }
+      }
+      cp_async_wait_all();
+      fence_proxy_async_smem();
+      mbar_arrive(&sm.full[s]);
     }
-    tc_fence_before();
-    __syncthreads();
+  } else if (warp == TC_MMA_WARP) {
+    // ---------------- MMA issue (one thread) ----------------
+    if (lane == 0) {
+      int i = 0;
+      for (int t = blockIdx.x; t < ntiles; t += gridDim.x, i++) {
+        const int s = i % TC_STAGES, a = i & 1;
+        const int n = tiles[t].n;
+        if (!mbar_wait(&sm.full[s], (uint32_t)((i / TC_STAGES) & 1), status) ||
+            (i >= 2 && !mbar_wait(&sm.acc_empty[a], (uint32_t)(((i >> 1) & 1) ^ 1), status))) {
+          *abort_flag = 1;
+          break;
+        }
+        if (*abort_flag) break;
+        tc_fence_after();
+        const uint32_t sq = smem_u32(sm.q[s]), sk = smem_u32(sm.k[s]);
+        const uint32_t id = idesc_bf16_f32(BLK, (n + 15) & ~15);
+#pragma unroll
+        for (int kk = 0; kk < 4; kk++)
+          umma_bf16(tmem + (uint32_t)(a * 256), sdesc_k_sw128(sk + kk * 32),
+                    sdesc_k_sw128(sq + kk * 32), id, kk > 0);
+        umma_commit(&sm.empty[s]);
+        umma_commit(&sm.acc_full[a]);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ---------------- epilogue: thread = key row of the block ----------------
+    const int h = warp >> 2, quarter = warp & 3;
+    const int r = quarter * 32 + lane;  // key row of the block
+    const size_t row_stride = (size_t)m * BLK;
+    const float NEG = -__int_as_float(0x7f800000);
+    int i = 0;
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x, i++) {
+      const int a = i & 1;
+      const TileDesc td = tiles[t];
+      const int c_beg = h * 128, c_end = min(td.n, c_beg + 128);
+      // the list entries of this warp's queries, fetched while the MMA runs:
+      // entry c_beg + 32 j + lane in ej[j]
+      uint32_t ej[4];
+#pragma unroll
+      for (int j = 0; j < 4; j++) {
+        const int c = c_beg + 32 * j + lane;
+        ej[j] = c < c_end ? __ldg(list + td.list_off + c) : 0u;
+      }
+      if (!mbar_wait(&sm.acc_full[a], (uint32_t)((i >> 1) & 1), status)) {
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      if (c_beg < c_end) {  // warp-uniform
+        const TileSeq ts = tile_seq(td, emax, cu_q, cu_k, seqlens);
+        const int rlim = ts.b * BLK + r - ts.pos_off;  // key row r is causal for rows >= rlim
+        const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(a * 256);
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+          const int c0 = c_beg + 32 * j;
+          if (c0 < c_end) {  // warp-uniform
+            uint32_t v[32];
+            tmem_ld16(taddr + (uint32_t)c0, *reinterpret_cast<uint32_t(*)[16]>(&v[0]));
+            tmem_ld16(taddr + (uint32_t)(c0 + 16), *reinterpret_cast<uint32_t(*)[16]>(&v[16]));
+            tmem_wait_ld();
+#pragma unroll
+            for (int u = 0; u < 32; u++) {
+              const uint32_t e = __shfl_sync(0xffffffffu, ej[j], u);
+              if (c0 + u < c_end) {
+                const int row = (int)(e >> 7), slot = (int)(e & 127u);
+                scratch[(size_t)row * row_stride + (size_t)slot * BLK + r] =
+                    row >= rlim ? __uint_as_float(v[u]) : NEG;
+              }
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&sm.acc_empty[a]);
+    }
   }
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, TC_TMEM_COLS);
@@ -372,7 +468,7 @@ cudaError_t launch_token_score_tc(const uint16_t *q, const uint16_t *k, const in
     return e;
   {
     ProfScope ps(K_TOKEN_SCORE_TC, st);
-    token_score_tc_kernel<<<2 * num_sms, TC_THREADS, TC_SMEM_BYTES, st>>>(
+    token_score_tc_kernel<<<num_sms, TC_THREADS, TC_SMEM_BYTES, st>>>(
         kmap, q, k, cu_q, cu_k, seqlens, emax, m, tiles, ntiles, list, scores, status);
   }
   return cudaGetLastError();
