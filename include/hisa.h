@@ -216,11 +216,12 @@ hisa_status hisa_device_status(int32_t *status, int clear, hisa_stream_t stream)
  *
  *   - The array exists once per device and every device that loads the library
  *     holds it until the process exits.
- *   - Problems whose scratch exceeds HISA_NOALLOC_SCRATCH_BYTES are rejected with
- *     HISA_ERR_WORKSPACE before anything is launched.  The scratch needed equals
- *     hisa_select_workspace_size() for the same arguments (about m * 516 bytes per
- *     query); at m = 64 every batch of up to 500 queries fits, which covers decode
- *     batches.
+ *   - Batches of fewer than twice as many queries as the GPU has SMs (decode) run
+ *     on a path that needs no scratch at all.  Larger batches need the scratch
+ *     hisa_select_workspace_size() reports for the same arguments (about
+ *     m * 516 bytes per query plus the block-score matrix), and problems whose
+ *     scratch exceeds HISA_NOALLOC_SCRATCH_BYTES are rejected with
+ *     HISA_ERR_WORKSPACE before anything is launched.
  *   - Every call shares the array and it keeps the last call's contents; nothing
  *     in it needs to start at zero.  Calls whose kernels overlap on the GPU (on
  *     different streams, or from different host threads) race on the array and

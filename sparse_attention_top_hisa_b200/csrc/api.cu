@@ -32,6 +32,13 @@ cudaError_t launch_dsa(const uint16_t *q, const uint16_t *k, const int32_t *cu_q
                        int max_seqlen_k, int topk, int32_t *out_idx, float *out_scores,
                        uint8_t *ws, int *status, cudaStream_t st);
 size_t dsa_workspace_bytes(int total_q, int num_seqs, int max_seqlen_k, int topk);
+bool use_tc_path(int total_q, int num_sms);
+bool decode_path_fits(int max_seqlen_k);
+cudaError_t launch_decode_select(const uint16_t *q, const uint16_t *k, const float *reps,
+                                 const int32_t *cu_q, const int32_t *cu_k,
+                                 const int32_t *seqlens, int S, int total_q, int max_seqlen_k,
+                                 int m, int topk, int32_t *out_idx, float *out_scores,
+                                 int32_t *out_blocks, int *status, cudaStream_t st);
 }  // namespace hisa
 
 using namespace hisa;
@@ -44,7 +51,7 @@ const char *kKindNames[K_NUM_KINDS] = {
     "pool_blocks",        "append_keys",         "block_select",   "token_fused",
     "token_score_split",  "token_select_scratch", "key_norm",      "dsa_filter",
     "dsa_select",         "dsa_fallback",         "inv_lists",      "inv_scan",
-    "token_score_tc",     "reps_split",          "block_score_tc"};
+    "token_score_tc",     "reps_split",          "block_score_tc",  "decode_select"};
 long long g_launches[K_NUM_KINDS];
 double g_ms[K_NUM_KINDS];
 long long g_timed[K_NUM_KINDS];
@@ -227,6 +234,10 @@ hisa_status hisa_select(const hisa_bf16 *q_idx, const hisa_bf16 *k_idx, const fl
   int *st = status_word();
   if (!st) return HISA_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (!use_tc_path(total_q, num_sms()) && decode_path_fits(max_seqlen_k))
+    return from_cuda(launch_decode_select(q_idx, k_idx, reps, cu_seqlens_q, cu_seqlens_k,
+                                          seqlens_k, num_seqs, total_q, max_seqlen_k, m, k,
+                                          out_idx, out_scores, out_blocks, st, s));
   uint8_t *w = static_cast<uint8_t *>(ws);
   int32_t *blk = reinterpret_cast<int32_t *>(w + p.off_blk);
   cudaError_t e = launch_block_select(q_idx, reps, cu_seqlens_q, cu_seqlens_k, seqlens_k,
@@ -369,14 +380,20 @@ extern "C" hisa_status hisa_select_noalloc(const hisa_bf16 *q_idx, const hisa_bf
       !aligned(cu_seqlens_q, 4) || !aligned(cu_seqlens_k, 4) || !aligned(seqlens_k, 4) ||
       !aligned(out_idx, 4) || !aligned(out_scores, 4) || !aligned(out_blocks, 4))
     return HISA_ERR_UNALIGNED;
-  // the same scratch layout hisa_select carves from its workspace must fit the array
   if (total_q >= (1 << 25)) return HISA_ERR_INVALID_ARG;
+  int *st = status_word();
+  if (!st) return HISA_ERR_CUDA;
+  cudaStream_t s0 = static_cast<cudaStream_t>(stream);
+  // few queries: the cluster kernel, which needs no scratch at all (as in hisa_select)
+  if (!use_tc_path(total_q, num_sms()) && decode_path_fits(max_seqlen_k))
+    return from_cuda(launch_decode_select(q_idx, k_idx, reps, cu_seqlens_q, cu_seqlens_k,
+                                          seqlens_k, num_seqs, total_q, max_seqlen_k, m, k,
+                                          out_idx, out_scores, out_blocks, st, s0));
+  // the same scratch layout hisa_select carves from its workspace must fit the array
   const SelectPlan p = select_plan(total_q, num_seqs, max_seqlen_k, m);
   if (p.total > (size_t)HISA_NOALLOC_SCRATCH_BYTES) return HISA_ERR_WORKSPACE;
   uint8_t *w = noalloc_scratch();
   if (!w) return HISA_ERR_CUDA;
-  int *st = status_word();
-  if (!st) return HISA_ERR_CUDA;
   // Nothing in the scratch has to start at zero: the block lists are written in full by
   // the block stage and every score row is written before it is read.
   cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -120,3 +120,97 @@ __device__ __forceinline__ void warp_select_blocks(const uint32_t *keys, int E, 
 }
 
 }  // namespace hisa
+
+namespace hisa {
+
+// CTA-wide version of the above for NT >= 256 threads: the radix select over 8-bit
+// digits uses one histogram bin per thread, and the selected blocks are emitted in
+// ascending order through block scans (thread t owns a contiguous range of blocks).
+// `hist` holds 256 words, `warp_tot` NT/32 + 1 ints, `bc` 4 ints of shared memory.
+template <int NT>
+__device__ void cta_select_blocks(const uint32_t *keys, int E, int own, int m, int32_t *dst,
+                                  int32_t *dst2, uint32_t *hist, int *warp_tot, int *bc) {
+  static_assert(NT >= 256, "one histogram bin per thread");
+  const int tid = threadIdx.x;
+  const int nf = min(m, 3);
+  const int mfree = m - nf;
+  uint32_t T = 0xffffffffu;  // nothing free is taken when mfree == 0
+  int need_eq = 0;
+  if (mfree > 0) {
+    uint32_t prefix = 0u, pmask = 0u;
+    int remaining = mfree;
+    bool done = false;
+#pragma unroll 1
+    for (int shift = 24; shift >= 0 && !done; shift -= 8) {
+      if (tid < 256) hist[tid] = 0u;
+      __syncthreads();
+      for (int b = tid; b < E; b += NT) {
+        const uint32_t u = keys[b];
+        if (u != 0u && (u & pmask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], 1u);
+      }
+      __syncthreads();
+      const int h = tid < 256 ? (int)hist[255 - tid] : 0;  // highest digit first
+      int total;
+      const int run = block_exclusive_scan<NT>(h, warp_tot, &total);
+      if (tid < 256 && run < remaining && run + h >= remaining) {
+        bc[0] = 255 - tid;
+        bc[1] = run;
+        bc[2] = h;
+      }
+      __syncthreads();
+      const int digit = bc[0], above = bc[1], inbin = bc[2];
+      remaining -= above;
+      prefix |= (uint32_t)digit << shift;
+      pmask |= 255u << shift;
+      if (inbin == remaining) {  // the whole bin is selected
+        T = prefix ? prefix - 1u : 0u;
+        need_eq = 0;
+        done = true;
+      } else if (shift == 0) {
+        T = prefix;
+        need_eq = remaining;
+      }
+    }
+  }
+  auto forced = [&](int b) {
+    return b == own || (nf >= 2 && b == own - 1) || (nf >= 3 && b == 0);
+  };
+  // emission in ascending block order
+  const int per = (E + NT - 1) / NT;
+  const int b0 = min(E, tid * per), b1 = min(E, b0 + per);
+  int neq = 0;
+  for (int b = b0; b < b1; b++) {
+    const uint32_t u = keys[b];
+    neq += (need_eq > 0 && u != 0u && u == T);
+  }
+  int tot;
+  int eqr = block_exclusive_scan<NT>(neq, warp_tot, &tot);
+  int nsel = 0;
+  {
+    int e = eqr;
+    for (int b = b0; b < b1; b++) {
+      const uint32_t u = keys[b];
+      const bool is_eq = need_eq > 0 && u != 0u && u == T;
+      nsel += forced(b) || (mfree > 0 && u != 0u && u > T) || (is_eq && e < need_eq);
+      e += is_eq;
+    }
+  }
+  int outp = block_exclusive_scan<NT>(nsel, warp_tot, &tot);
+  for (int b = b0; b < b1; b++) {
+    const uint32_t u = keys[b];
+    const bool is_eq = need_eq > 0 && u != 0u && u == T;
+    if (forced(b) || (mfree > 0 && u != 0u && u > T) || (is_eq && eqr < need_eq)) {
+      dst[outp] = b;
+      if (dst2) dst2[outp] = b;
+      outp++;
+    }
+    eqr += is_eq;
+  }
+  for (int i = tot + tid; i < m; i += NT) {  // only reachable if fewer than m exist
+    dst[i] = -1;
+    if (dst2) dst2[i] = -1;
+  }
+  __syncthreads();
+}
+
+}  // namespace hisa

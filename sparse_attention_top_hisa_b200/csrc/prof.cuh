@@ -23,6 +23,7 @@ enum KernelKind {
   K_TOKEN_SCORE_TC,
   K_REPS_SPLIT,
   K_BLOCK_SCORE_TC,
+  K_DECODE_SELECT,
   K_NUM_KINDS
 };
 

@@ -46,11 +46,11 @@ def _call_noalloc(L, q, k, reps, cu_q, cu_k, sl, S, total_q, maxlen, m, topk):
 
 
 def _cases():
-    # prefill: one CTA per query, scratch = the block lists
+    # prefill (tensor-core path): scratch = block lists, inverted lists and score rows
     w = gaussian_prefill(3000, 31, m=8, topk=256)
     dw = OnDevice(w)
     yield "prefill", dw.q, dw.k, dw.cu_q, dw.cu_k, dw.seqlens, 1, w.total_q, w.max_seqlen_k, 8, 256
-    # decode: 16 single-query sequences, scratch = block lists + split score rows
+    # decode: 16 single-query sequences (the cluster kernel, which uses no scratch)
     d = decode_workload(16, 5000, 1, 32, m=16, topk=512)
     kc = dev_bf16(d.k_cache)
     cu_k = dev_i32(d.cu_k)
