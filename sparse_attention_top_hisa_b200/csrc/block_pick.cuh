@@ -214,3 +214,156 @@ __device__ void cta_select_blocks(const uint32_t *keys, int E, int own, int m, i
 }
 
 }  // namespace hisa
+
+namespace hisa {
+
+// Top-m by linear score buckets, for NT >= 256 threads: 256 buckets linear in the
+// score between the lowest and the highest free key, one scan for the bucket that
+// holds the mfree-th best block, exact ranking (score desc, block asc) of that
+// bucket's members, and emission in ascending block order by warp ballots over
+// contiguous ranges.  Returns false, with nothing written, when the boundary bucket
+// has more than LIN_BLK_CAP members (heavy ties); the caller then uses
+// cta_select_blocks.  `scratch` must hold lin_blk_scratch_bytes(E) bytes.
+constexpr int LIN_BLK_CAP = 512;
+
+__host__ __device__ inline size_t lin_blk_scratch_bytes(int E) {
+  return (size_t)LIN_BLK_CAP * 8 + (size_t)((E + 15) & ~15);
+}
+
+template <int NT>
+__device__ bool cta_select_blocks_lin(const uint32_t *keys, int E, int own, int m,
+                                      int32_t *dst, int32_t *dst2, uint32_t *hist,
+                                      int *warp_tot, int *bc, uint8_t *scratch) {
+  static_assert(NT >= 256, "one bucket per thread");
+  constexpr int NW = NT / 32;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nf = min(m, 3);
+  const int mfree = m - nf;
+  uint32_t *mem_key = reinterpret_cast<uint32_t *>(scratch);
+  int32_t *mem_blk = reinterpret_cast<int32_t *>(scratch) + LIN_BLK_CAP;
+  uint8_t *selb = scratch + (size_t)LIN_BLK_CAP * 8;
+  auto forced = [&](int b) {
+    return b == own || (nf >= 2 && b == own - 1) || (nf >= 3 && b == 0);
+  };
+  // 1. range of the free scores
+  const float NEG = -__int_as_float(0x7f800000);
+  float mx = NEG, mn = -NEG;
+  for (int b = tid; b < E; b += NT) {
+    const uint32_t u = keys[b];
+    if (u != 0u) {
+      const float s = key_score(u);
+      mx = fmaxf(mx, s);
+      mn = fminf(mn, s);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+  }
+  float *wr = reinterpret_cast<float *>(hist);  // 2 * NW floats, before the histogram
+  if (tid < 256) hist[tid] = 0u;
+  __syncthreads();
+  if (lane == 0) {
+    wr[256 + warp] = mx;  // hist has 256 + 2 * NW words
+    wr[256 + NW + warp] = mn;
+  }
+  __syncthreads();
+  mx = NEG;
+  mn = -NEG;
+#pragma unroll
+  for (int w = 0; w < NW; w++) {
+    mx = fmaxf(mx, wr[256 + w]);
+    mn = fminf(mn, wr[256 + NW + w]);
+  }
+  const float range = mx - mn;
+  const float inv = range > 0.f ? 256.f / range : 0.f;
+  if (mfree > 0 && !(inv > 0.f && isfinite(inv))) return false;  // one distinct score
+  auto bucket = [&](uint32_t u) { return min(__float2int_rz((mx - key_score(u)) * inv), 255); };
+  // 2. histogram, 3. boundary bucket
+  int bstar = 256, above = 0, nb = 0;
+  if (mfree > 0) {
+    for (int b = tid; b < E; b += NT) {
+      const uint32_t u = keys[b];
+      if (u != 0u) atomicAdd(&hist[bucket(u)], 1u);
+    }
+    __syncthreads();
+    const int h = tid < 256 ? (int)hist[tid] : 0;
+    int total;
+    const int run = block_exclusive_scan<NT>(h, warp_tot, &total);
+    if (tid == 0) bc[3] = 0;
+    if (tid < 256 && run < mfree && run + h >= mfree) {
+      bc[0] = tid;
+      bc[1] = run;
+      bc[2] = h;
+    }
+    __syncthreads();
+    bstar = bc[0];
+    above = bc[1];
+    nb = bc[2];
+    if (nb > LIN_BLK_CAP) return false;
+  }
+  const int need = mfree - above;
+  // 4. sure picks and forced blocks flagged, boundary members gathered
+  for (int b = tid; b < E; b += NT) {
+    const uint32_t u = keys[b];
+    bool s = forced(b);
+    if (u != 0u && mfree > 0) {
+      const int bk = bucket(u);
+      s = s || bk < bstar;
+      if (bk == bstar) {
+        const int e = atomicAdd(&bc[3], 1);
+        mem_key[e] = u;
+        mem_blk[e] = b;
+      }
+    }
+    selb[b] = s ? 1 : 0;
+  }
+  __syncthreads();
+  // 5. the best `need` boundary members
+  for (int e = tid; e < nb; e += NT) {
+    const uint32_t mk = mem_key[e];
+    const int mb = mem_blk[e];
+    int rank = 0;
+    for (int t = 0; t < nb; t++) {
+      const uint32_t tk = mem_key[t];
+      rank += (tk > mk) || (tk == mk && mem_blk[t] < mb);
+    }
+    if (rank < need) selb[mb] = 1;
+  }
+  __syncthreads();
+  // 6. emission: warp w walks blocks [w * per, (w + 1) * per) twice (count, write)
+  const int per = ((E + NW - 1) / NW + 31) & ~31;
+  const int w0 = min(E, warp * per), w1 = min(E, w0 + per);
+  int cnt = 0;
+  for (int b0 = w0; b0 < w1; b0 += 32) {
+    const int b = b0 + lane;
+    cnt += __popc(__ballot_sync(0xffffffffu, b < w1 && selb[b]));
+  }
+  if (lane == 0) bc[4 + warp] = cnt;  // bc holds 4 + NW ints
+  __syncthreads();
+  int outp = 0, tot = 0;
+  for (int w = 0; w < NW; w++) {
+    if (w < warp) outp += bc[4 + w];
+    tot += bc[4 + w];
+  }
+  const unsigned lt = (1u << lane) - 1u;
+  for (int b0 = w0; b0 < w1; b0 += 32) {
+    const int b = b0 + lane;
+    const bool s = b < w1 && selb[b];
+    const unsigned mask = __ballot_sync(0xffffffffu, s);
+    if (s) {
+      dst[outp + __popc(mask & lt)] = b;
+      if (dst2) dst2[outp + __popc(mask & lt)] = b;
+    }
+    outp += __popc(mask);
+  }
+  for (int i = tot + tid; i < m; i += NT) {  // only reachable if fewer than m exist
+    dst[i] = -1;
+    if (dst2) dst2[i] = -1;
+  }
+  __syncthreads();
+  return true;
+}
+
+}  // namespace hisa

@@ -167,6 +167,28 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int *warp_tot, int *t
   return excl;
 }
 
+// Launch `func` as a programmatic dependent of the previous kernel on `st` (its
+// launch may overlap that kernel's tail; the kernel itself must execute
+// griddepcontrol.wait before touching memory).  On the legacy default stream the
+// launch is an ordinary one.
+template <typename... Args>
+inline cudaError_t launch_pdl(const void *func, dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t st, Args... args) {
+  void *argv[] = {(void *)&args...};
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  const bool legacy = st == nullptr || st == cudaStreamLegacy || st == cudaStreamPerThread;
+  cfg.attrs = legacy ? nullptr : attr;
+  cfg.numAttrs = legacy ? 0 : 1;
+  return cudaLaunchKernelExC(&cfg, func, argv);
+}
+
 // Raise a kernel's dynamic shared-memory limit once per device; later calls (for
 // example while a CUDA graph is being captured) find it already set.
 inline cudaError_t set_smem_once(const void *func, size_t bytes, int *cache /*[64]*/) {

@@ -9,8 +9,9 @@
 // distributed shared memory:
 //   A. block scores: CTA c scores a contiguous share of the eligible blocks (eight
 //      lanes per representative row, fp32) into order-preserving keys;
-//   B. every CTA gathers all keys from the cluster and runs the same CTA-wide radix
-//      top-m (identical inputs, identical choice), so no broadcast step is needed;
+//   B. every CTA gathers all keys from the cluster and runs the same CTA-wide top-m
+//      (linear score buckets, exact ranking of the boundary bucket; radix select on
+//      heavy ties) on identical inputs, so no broadcast step is needed;
 //   C. CTA c gathers and scores its share of the selected blocks' tokens straight
 //      from HBM (four lanes per key row, 16 dims each, eight rows in flight per lane);
 //   D. exact top-k across the cluster: global max / min / count, per-CTA bucket
@@ -46,6 +47,7 @@ constexpr int DC_BINS = 1024;
 constexpr int DC_BIN_WORDS = DC_BINS + DC_BINS / 32;  // bucket b at word b + b / 32
 constexpr int DC_MAXK = HISA_MAX_TOPK;
 constexpr int DC_LOC_MAX = 1024;  // sequences looked up cooperatively (else by binary search)
+constexpr size_t LIN_BLK_SCRATCH_MAX = (size_t)LIN_BLK_CAP * 8 + DC_MAX_E;
 static_assert(DC_KPT * DC_THREADS == DC_MAX_CAND, "candidates split evenly");
 
 struct DcRed {
@@ -71,10 +73,10 @@ struct __align__(16) DcSmem {
   uint32_t boff[DC_BIN_WORDS];              // D: global bucket offsets
   uint32_t bcnt[DC_BIN_WORDS];              // D: global bucket counts
   uint32_t curs[DC_BIN_WORDS];              // D: this CTA's scatter cursors
-  uint32_t whist[256];                      // B: warp radix histogram
+  uint32_t whist[256 + 2 * DC_WARPS];       // B: top-m histogram and warp partials
   int32_t blocks[HISA_MAX_M];               // B: selected blocks, ascending
   int pos_lo[DC_CTAS];                      // D: first output position ranked by each CTA
-  int bsc[4];                               // B: radix scratch
+  int bsc[4 + DC_WARPS];                    // B: top-m scratch
   int32_t cuq[DC_LOC_MAX + 1];              // cu_seqlens_q, for the sequence lookup
   uint4 qrow[D / 8];                        // the query row
   int seqinfo[4];                           // sequence, region start, region end, live keys
@@ -120,6 +122,11 @@ decode_select_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict_
                      int *status) {
   extern __shared__ __align__(16) uint8_t dc_raw[];
   DcSmem &sm = *reinterpret_cast<DcSmem *>(dc_raw);
+  // Launched as a programmatic dependent of the previous kernel on the stream (when
+  // the stream allows it): nothing is read before that kernel has completed, and the
+  // next kernel may begin launching at once (it waits the same way).
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   cg::cluster_group cl = cg::this_cluster();
   const int me = (int)cl.block_rank();
   const int row = blockIdx.x / DC_CTAS;
@@ -244,8 +251,12 @@ decode_select_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict_
       *reinterpret_cast<uint4 *>(&sm.u1.allkeys[b]) = rk[(b - owner * per) >> 2];
     }
     __syncthreads();
-    cta_select_blocks<DC_THREADS>(sm.u1.allkeys, E, own, m, sm.blocks, me == 0 ? ob : nullptr,
-                                  sm.whist, sm.warp_tot, sm.bsc);
+    static_assert(sizeof(sm.u2) >= LIN_BLK_SCRATCH_MAX, "top-m scratch fits the staging area");
+    if (!cta_select_blocks_lin<DC_THREADS>(sm.u1.allkeys, E, own, m, sm.blocks,
+                                           me == 0 ? ob : nullptr, sm.whist, sm.warp_tot,
+                                           sm.bsc, reinterpret_cast<uint8_t *>(&sm.u2)))
+      cta_select_blocks<DC_THREADS>(sm.u1.allkeys, E, own, m, sm.blocks,
+                                    me == 0 ? ob : nullptr, sm.whist, sm.warp_tot, sm.bsc);
   } else {
     for (int i = tid; i < m; i += DC_THREADS) {
       const int v = i < E ? i : -1;
@@ -534,10 +545,11 @@ cudaError_t launch_decode_select(const uint16_t *q, const uint16_t *k, const flo
   const int emax = (max_seqlen_k + BLK - 1) / BLK;
   {
     ProfScope ps(K_DECODE_SELECT, st);
-    decode_select_kernel<<<total_q * DC_CTAS, DC_THREADS, sizeof(DcSmem), st>>>(
-        q, k, reps, cu_q, cu_k, seqlens, S, m, topk, emax > 0 ? emax : 1, out_idx, out_scores,
-        out_blocks, status);
+    e = launch_pdl((const void *)decode_select_kernel, dim3(total_q * DC_CTAS), dim3(DC_THREADS),
+                   sizeof(DcSmem), st, q, k, reps, cu_q, cu_k, seqlens, S, m, topk,
+                   emax > 0 ? emax : 1, out_idx, out_scores, out_blocks, status);
   }
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

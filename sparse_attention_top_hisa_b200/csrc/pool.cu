@@ -72,6 +72,9 @@ append_keys_kernel(uint16_t *__restrict__ kc, float *__restrict__ reps,
                    const int32_t *__restrict__ cu_k, int32_t *__restrict__ seqlens,
                    const uint16_t *__restrict__ new_keys, int n_new, int *status) {
   __shared__ __align__(16) uint4 blockrows[BLK * 8];
+  // programmatic dependent launch (see launch_append): wait for the previous kernel
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int s = blockIdx.x, tid = threadIdx.x;
   const int start = cu_k[s], cap = cu_k[s + 1] - start;
   const int len = seqlens[s];
@@ -136,11 +139,13 @@ cudaError_t launch_append(uint16_t *kc, float *reps, const int32_t *cu_k, int32_
                           const uint16_t *new_keys, int n_new, int num_seqs, int *status,
                           cudaStream_t st) {
   if (num_seqs == 0 || n_new == 0) return cudaSuccess;
+  cudaError_t e;
   {
     ProfScope ps(K_APPEND, st);
-    append_keys_kernel<<<num_seqs, APPEND_THREADS, 0, st>>>(kc, reps, cu_k, seqlens, new_keys,
-                                                            n_new, status);
+    e = launch_pdl((const void *)append_keys_kernel, dim3(num_seqs), dim3(APPEND_THREADS), 0, st,
+                   kc, reps, cu_k, seqlens, new_keys, n_new, status);
   }
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

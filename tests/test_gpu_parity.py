@@ -281,6 +281,56 @@ def test_decode_steps():
             assert torch.equal(pre[0], idx[s])
 
 
+def test_decode_side_stream_and_graph_match_default_stream():
+    """On a non-default stream the append and decode kernels are launched as
+    programmatic dependents of the previous kernel; eager and graph-captured runs
+    there must reproduce the default-stream rows bit for bit."""
+    h = H()
+    dwl = config_workload(2, steps=4)
+    S, cap = dwl.num_seqs, dwl.capacity
+    cu_k = dev_i32(dwl.cu_k)
+    cu_q = dev_i32(np.arange(S + 1))
+    newk = dev_bf16(dwl.new_keys)
+    qs = dev_bf16(dwl.queries.reshape(-1, 64)).view(dwl.steps, S, 64)
+
+    def fresh():
+        kc = dev_bf16(dwl.k_cache)
+        lens = dev_i32(dwl.seqlens0)
+        reps = h.hisa_pool_blocks(kc, cu_k, lens, cap)
+        outs = [torch.empty(S, dwl.topk, dtype=torch.int32, device="cuda") for _ in range(dwl.steps)]
+        return kc, lens, reps, outs
+
+    def run(state):
+        kc, lens, reps, outs = state
+        for i in range(dwl.steps):
+            h.hisa_append_keys(kc, reps, cu_k, lens, newk[i])
+            h.hisa_select(qs[i], kc, reps, cu_q, cu_k, lens, cap, dwl.m, dwl.topk, out_idx=outs[i])
+
+    ref = fresh()
+    run(ref)
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream()
+    eager = fresh()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(side):
+        run(eager)
+    side.synchronize()
+    graphed = fresh()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(g, stream=side):
+            run(graphed)
+    g.replay()
+    torch.cuda.synchronize()
+    assert h.hisa_device_status() == 0
+    for st in (eager, graphed):
+        assert torch.equal(st[0], ref[0]) and torch.equal(st[1], ref[1]) and torch.equal(st[2], ref[2])
+        for a, b in zip(st[3], ref[3]):
+            assert torch.equal(a, b)
+    del g
+
+
 # ---------------------------------------------------------------------------
 # errors found on the device
 
