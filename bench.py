@@ -42,9 +42,13 @@ UNIT = "queries/s"
 WORKLOAD = "prefill_L131072 (1 seq, q/k bf16 N(0,1), d=64, B=128, m=64, k=2048)"
 L2_FLUSH_BYTES = 256 << 20
 
-# DRAM bytes per launch read from an ncu capture, keyed by kernel kind, with the
-# sha256 of the kernel source the capture was taken on (a changed source voids it).
-TRAFFIC = {}
+# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from an ncu
+# capture, keyed by kernel kind, with the sha256 of the kernel's sources at capture time
+# (a changed source voids the figure).  token_select_scratch: captured on the 32768-token
+# prefill (1.203 GB for 1.84 M selected pairs, 0.987 of its algorithmic bytes) and scaled
+# to the 131072-token launch by selected pairs (8.13 M): see
+# profiles/token_select_scratch_prefill_L32768.md.
+TRAFFIC = {"token_select_scratch": (5203113956, "5ba765819dfc6bf0", ("token_select.cu", "select.cuh"))}
 
 
 def parse_args():
@@ -59,6 +63,9 @@ def parse_args():
                     help="prefill workload of the timed step (profiling runs; default 4 = 128K)")
     ap.add_argument("--dsa-steps", type=int, default=0,
                     help="profiling runs: flat-scan calls on the same workload after the timed steps")
+    ap.add_argument("--decode-profile", type=int, default=0, metavar="N",
+                    help="profiling runs: only N eager decode steps (16 x 32768 keys, append + "
+                         "selection on the default stream), then exit")
     return ap.parse_args()
 
 
@@ -234,10 +241,12 @@ def iou_rows(a: np.ndarray, b: np.ndarray) -> float:
     return float(np.mean(vals))
 
 
-def source_sha(name: str) -> str:
-    path = os.path.join(ROOT, "sparse_attention_top_hisa_b200", "csrc", name)
-    with open(path, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+def source_sha(names) -> str:
+    h = hashlib.sha256()
+    for name in names:
+        with open(os.path.join(ROOT, "sparse_attention_top_hisa_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 # ---------------------------------------------------------------------------
@@ -476,6 +485,28 @@ def extras(args, w4, q4, k4, cu_q4, cu_k4, sl4, out4, flush, stream, hbm_peak):
                           "hisa_queries_per_s": round(w3.total_q / (hm3 / 1e3), 1),
                           "iou_hisa_vs_dsa_4096_rows": round(iou_rows(a3[rows3], b3[rows3]), 4),
                           "needle_recall_hisa": float(rec_h), "needle_recall_dsa": float(rec_d)}
+    # variants on the same inputs: stage 1 alone (all tokens of the best k/B blocks,
+    # i.e. no token refinement) and a fractional block budget (m = M/2)
+    variants = {}
+    M3 = (w3.max_seqlen_k + w3.B - 1) // w3.B
+    for name, mv in (("block_sparse_only_m%d" % (w3.topk // w3.B), w3.topk // w3.B),
+                     ("hisa_half_m%d" % min(128, (M3 + 1) // 2), min(128, (M3 + 1) // 2))):
+        ov = torch.empty_like(o3)
+        wsv = torch.empty(H.hisa_select_workspace_size(w3.total_q, 1, w3.max_seqlen_k, mv, w3.topk),
+                          dtype=torch.uint8, device="cuda")
+
+        def hv():
+            H.hisa_pool_blocks(k3, ck3, sl3, w3.max_seqlen_k, reps=reps3)
+            H.hisa_select(q3, k3, reps3, cq3, ck3, sl3, w3.max_seqlen_k, mv, w3.topk, out_idx=ov,
+                          workspace=wsv)
+        hv()
+        msv = statistics.median(time_events(hv, 3, flush, stream))
+        av = ov.cpu().numpy()
+        variants[name] = {"m": mv, "ms": round(msv, 3),
+                          "iou_vs_dsa_4096_rows": round(iou_rows(av[rows3], b3[rows3]), 4),
+                          "needle_recall": float(np.mean([j in av[i] for i, j in w3.needles]))}
+        del ov, wsv
+    det["prefill_32k"]["variants"] = variants
     det["dsa_128k"]["hisa_speedup_over_dsa"] = None  # filled by the caller
     del q3, k3, o3, d3, ws3, dws3
     torch.cuda.empty_cache()
@@ -616,8 +647,33 @@ def run_reference(args, world, rank):
                     "d2h_bytes_per_step": 0}}
 
 
+def decode_profile(steps):
+    """Eager decode steps for a profiler: the decode workload of decode_bench, one state."""
+    import torch
+    import sparse_attention_top_hisa_b200 as H
+    from synth import config_workload
+    dw = config_workload(2, steps=steps)
+    S, cap, m, K = dw.num_seqs, dw.capacity, dw.m, dw.topk
+    cu_k, cu_q = to_dev_i32(dw.cu_k), to_dev_i32(np.arange(S + 1))
+    kc, lens = to_dev_bf16(dw.k_cache), to_dev_i32(dw.seqlens0)
+    reps = H.hisa_pool_blocks(kc, cu_k, lens, cap)
+    out = torch.empty(S, K, dtype=torch.int32, device="cuda")
+    ws = torch.empty(H.hisa_select_workspace_size(S, S, cap, m, K), dtype=torch.uint8, device="cuda")
+    newk = to_dev_bf16(dw.new_keys)
+    qs = to_dev_bf16(dw.queries.reshape(steps * S, 64)).view(steps, S, 64)
+    for i in range(steps):
+        H.hisa_append_keys(kc, reps, cu_k, lens, newk[i])
+        H.hisa_select(qs[i], kc, reps, cu_q, cu_k, lens, cap, m, K, out_idx=out, workspace=ws)
+    torch.cuda.synchronize()
+    assert H.hisa_device_status() == 0
+
+
 def main():
     args = parse_args()
+    if args.decode_profile > 0:
+        dist_setup(args)
+        decode_profile(args.decode_profile)
+        return
     if args.impl == "reference":
         world = int(os.environ.get("WORLD_SIZE", "1"))
         rank = int(os.environ.get("RANK", "0"))
