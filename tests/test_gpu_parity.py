@@ -13,8 +13,8 @@ import torch
 import oracle
 from parity import (OnDevice, check_block_band, check_token_band, dev_bf16, dev_i32,
                     exact_scores, sample_rows)
-from synth import (bf16_from_f32, config_workload, gaussian_prefill, integer_prefill,
-                   varlen_prefill)
+from synth import (bf16_from_f32, config_workload, decode_workload, gaussian_prefill,
+                   integer_prefill, varlen_prefill)
 
 pytestmark = pytest.mark.gpu
 
@@ -129,6 +129,82 @@ def test_dsa_exact_integer(lengths, k):
     assert np.array_equal(idx, o_idx)
     valid = o_idx >= 0
     assert np.array_equal(sc[valid].astype(np.float64), o_sc[valid])
+
+
+# Few queries (fewer than two per SM) take the cluster path: decode-shaped states with
+# long key caches, exact on integer inputs.
+DECODE_INT_CASES = [
+    # (num_seqs, live keys, m, k)
+    (16, 5000, 16, 512),     # a decode batch; ties at the block and token boundaries
+    (3, 40000, 64, 2048),    # long caches: 313 eligible blocks
+    (5, 300, 8, 256),        # at most m blocks: every block is selected
+    (4, 2000, 1, 64),        # m < 3: only the own block is forced
+    (4, 2000, 2, 64),        # m < 3: own and previous
+    (2, 9000, 128, 2048),    # the largest m
+]
+
+
+@pytest.mark.parametrize("S,L,m,k", DECODE_INT_CASES, ids=[str(c) for c in DECODE_INT_CASES])
+def test_decode_exact_integer(S, L, m, k):
+    h = H()
+    d = decode_workload(S, L, 1, 700 + m, m=m, topk=k, integer=True)
+    kc, cu_k, lens = dev_bf16(d.k_cache), dev_i32(d.cu_k), dev_i32(d.seqlens0)
+    cu_q = dev_i32(np.arange(S + 1))
+    q = dev_bf16(d.queries[0])
+    reps = h.hisa_pool_blocks(kc, cu_k, lens, L)
+    sc = torch.empty(S, k, dtype=torch.float32, device="cuda")
+    bl = torch.empty(S, m, dtype=torch.int32, device="cuda")
+    idx = h.hisa_select(q, kc, reps, cu_q, cu_k, lens, L, m, k, out_scores=sc, out_blocks=bl)
+    torch.cuda.synchronize()
+    assert h.hisa_device_status() == 0
+    o_idx, o_sc, o_bl, _ = oracle.hisa(d.queries[0], d.k_cache, np.arange(S + 1, dtype=np.int32),
+                                       d.cu_k, d.seqlens0, d.B, m, k)
+    assert np.array_equal(bl.cpu().numpy(), o_bl)
+    assert np.array_equal(idx.cpu().numpy(), o_idx)
+    scn = sc.cpu().numpy()
+    valid = o_idx >= 0
+    assert np.array_equal(scn[valid].astype(np.float64), o_sc[valid])
+    assert np.all(scn[~valid] == 0)
+
+
+def test_few_queries_several_per_sequence_exact():
+    """The cluster path with several query rows per sequence (the last 40 positions of
+    each of two sequences), exact on integer inputs."""
+    h = H()
+    w = varlen_prefill([3000, 1500], 41, m=8, topk=256, integer=True)
+    tail = 40
+    rows = np.concatenate([np.arange(int(w.cu_q[s + 1]) - tail, int(w.cu_q[s + 1]))
+                           for s in range(w.num_seqs)])
+    qsel = w.q[rows]
+    cu_q = np.arange(w.num_seqs + 1, dtype=np.int32) * tail
+    dq, dk = dev_bf16(qsel), dev_bf16(w.k)
+    dcu_q, dcu_k, dsl = dev_i32(cu_q), dev_i32(w.cu_k), dev_i32(w.seqlens)
+    reps = h.hisa_pool_blocks(dk, dcu_k, dsl, w.max_seqlen_k)
+    idx = h.hisa_select(dq, dk, reps, dcu_q, dcu_k, dsl, w.max_seqlen_k, 8, 256)
+    torch.cuda.synchronize()
+    assert h.hisa_device_status() == 0
+    o_idx, _, _, _ = oracle.hisa(qsel, w.k, cu_q, w.cu_k, w.seqlens, w.B, 8, 256)
+    assert np.array_equal(idx.cpu().numpy(), o_idx)
+
+
+def test_few_queries_all_scores_equal():
+    """Every score equal on the cluster path: the distributed select takes its radix
+    route and every row is its lowest-index candidates."""
+    h = H()
+    S, L, m, k = 3, 3000, 8, 512
+    d = decode_workload(S, L, 1, 9, m=m, topk=k, integer=True)
+    ones = bf16_from_f32(np.ones((1, 64), np.float32))[0]
+    d.k_cache[:] = ones
+    d.queries[:] = ones
+    kc, cu_k, lens = dev_bf16(d.k_cache), dev_i32(d.cu_k), dev_i32(d.seqlens0)
+    reps = h.hisa_pool_blocks(kc, cu_k, lens, L)
+    idx = h.hisa_select(dev_bf16(d.queries[0]), kc, reps, dev_i32(np.arange(S + 1)), cu_k, lens,
+                        L, m, k)
+    torch.cuda.synchronize()
+    assert h.hisa_device_status() == 0
+    o_idx, _, _, _ = oracle.hisa(d.queries[0], d.k_cache, np.arange(S + 1, dtype=np.int32),
+                                 d.cu_k, d.seqlens0, d.B, m, k)
+    assert np.array_equal(idx.cpu().numpy(), o_idx)
 
 
 def test_equal_keys_degenerate():
