@@ -55,9 +55,11 @@ def _load():
         lib.oracle_token_select.argtypes = [P, P, P, I, P, P, P, I, I, I, I, I, P, I, P, P, I]
         lib.oracle_dsa.argtypes = [P, P, P, P, P, I, I, I, I, P, I, P, P, I]
         lib.oracle_hisa.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P, I, P, P, P, P, I]
+        lib.oracle_sparse_attention.argtypes = [P, P, P, P, P, P, I, I, I, I, I,
+                                                ctypes.c_double, P, P, I]
         lib.oracle_set_mutation.argtypes = [I]
         lib.oracle_get_mutation.restype = I
-        for f in ("oracle_pool", "oracle_block_select", "oracle_block_scores",
+        for f in ("oracle_sparse_attention", "oracle_pool", "oracle_block_select", "oracle_block_scores",
                   "oracle_token_select", "oracle_dsa", "oracle_hisa"):
             getattr(lib, f).restype = I
         _lib = lib
@@ -198,3 +200,28 @@ def hisa_workload(w, rows=None, nthreads: int = 0):
 def dsa_workload(w, rows=None, nthreads: int = 0):
     """oracle.dsa on a synth.Workload."""
     return dsa(w.q, w.k, w.cu_q, w.cu_k, w.seqlens, w.topk, rows, nthreads)
+
+
+def sparse_attention(q, k, v, idx, cu_q, cu_k, H: int, scale: float, nthreads: int = 0):
+    """Attention over the selected tokens (see hisa_oracle.c, oracle_sparse_attention).
+
+    q: bf16 bits [total_q, H, dv]; k, v: bf16 bits [rows_k, dv]; idx: int32
+    [total_q, topk] sequence-local positions, -1 = none.  Returns (out f64
+    [total_q, H, dv], lse f64 [total_q, H]).
+    """
+    L = _load()
+    q = _c(q, np.uint16)
+    k = _c(k, np.uint16)
+    v = _c(v, np.uint16)
+    idx = _c(idx, np.int32)
+    cu_q = _c(cu_q, np.int32)
+    cu_k = _c(cu_k, np.int32)
+    total_q, topk = idx.shape
+    dv = k.shape[1]
+    assert q.shape == (total_q, H, dv) and v.shape == k.shape
+    out = np.zeros((total_q, H, dv), np.float64)
+    lse = np.zeros((total_q, H), np.float64)
+    _check(L.oracle_sparse_attention(_p(q), _p(k), _p(v), _p(idx), _p(cu_q), _p(cu_k),
+                                     len(cu_q) - 1, total_q, H, dv, topk, float(scale), _p(out),
+                                     _p(lse), nthreads), "oracle_sparse_attention")
+    return out, lse

@@ -79,3 +79,25 @@ def dsa_row(qrow_u16, keys_u16, pos: int, topk: int):
     qv = _vals(np.asarray(qrow_u16)[None])[0]
     cands = [(dot(qv, keys[j]), j) for j in range(pos + 1)]
     return ranked_top(cands, topk)
+
+
+def attention(q_heads, keys, values, idx, scale):
+    """Attention of one query row over its selected tokens, written independently of
+    the C oracle: each weight is 1 / sum_t exp(s_t - s_j) (no running maximum), every
+    sum is math.fsum.  q_heads: H lists of dv floats; keys / values: token -> dv
+    floats; idx: token positions, -1 = none.  Returns (H lists of dv floats, H lse)."""
+    import math
+    sel = [j for j in idx if j >= 0]
+    outs, lses = [], []
+    for qh in q_heads:
+        if not sel:
+            outs.append([0.0] * len(qh))
+            lses.append(-math.inf)
+            continue
+        s = [scale * math.fsum(a * b for a, b in zip(qh, keys[j])) for j in sel]
+        w = [1.0 / math.fsum(math.exp(st - sj) for st in s) for sj in s]
+        outs.append([math.fsum(w[t] * values[j][d] for t, j in enumerate(sel))
+                     for d in range(len(qh))])
+        top = max(s)
+        lses.append(top + math.log(math.fsum(math.exp(st - top) for st in s)))
+    return outs, lses

@@ -516,3 +516,115 @@ int oracle_hisa(const uint16_t *q, const uint16_t *k, const int32_t *cu_q, const
   if (!blocks_out) free(blk);
   return e;
 }
+
+/* ------------------------------------------------------------------------- */
+/* The sparse attention step that consumes the selected indices.
+ *
+ * [HISA/kv]: the top-k token indices keep the DSA output structure and go to the
+ * sparse attention operator; [DSA]: attention is then computed only over the
+ * selected tokens.  The pages name that operator but do not write out its
+ * arithmetic; the reading used here is the textbook scaled dot-product attention
+ * restricted to the selected tokens, with the heads of a query sharing its
+ * selection and one key row and one value row per token shared by every head:
+ *   s_j      = scale * q[i][h] . kv_key[j]          for the entries j >= 0 of idx[i]
+ *   w_j      = exp(s_j - max s) / sum exp(s - max s)
+ *   o[i][h]  = sum_j w_j * kv_val[j],   lse[i][h] = log sum_j exp(s_j)
+ * A row with no valid index gets o = 0 and lse = -inf.  Sums in double, in index
+ * order for the weights and dimension order for the dot products. */
+
+typedef struct {
+  const uint16_t *q, *k, *v;
+  const int32_t *idx, *cu_q, *cu_k;
+  int S, total_q, H, dv, topk;
+  double scale;
+  double *out, *lse;
+  int next, err;
+  pthread_mutex_t mu;
+} att_job;
+
+static void att_row(att_job *J, int row, double *s) {
+  int sq = 0;
+  while (sq + 1 < J->S && J->cu_q[sq + 1] <= row) sq++;
+  const int64_t kbase = J->cu_k[sq];
+  const int32_t *ir = J->idx + (int64_t)row * J->topk;
+  for (int h = 0; h < J->H; h++) {
+    const uint16_t *qh = J->q + ((int64_t)row * J->H + h) * J->dv;
+    double *o = J->out + ((int64_t)row * J->H + h) * J->dv;
+    for (int d = 0; d < J->dv; d++) o[d] = 0.0;
+    double mx = -INFINITY;
+    int n = 0;
+    for (int t = 0; t < J->topk; t++) {
+      int j = ir[t];
+      if (j < 0) {
+        if (g_mutation != 10) {
+          s[t] = -INFINITY;
+          continue;
+        }
+        j = 0;  /* planted mistake: padding read as token 0 */
+      }
+      const uint16_t *kr = J->k + (kbase + j) * J->dv;
+      double acc = 0.0;
+      for (int d = 0; d < J->dv; d++) acc += bf16_value(qh[d]) * bf16_value(kr[d]);
+      s[t] = (g_mutation == 11 ? 1.0 : J->scale) * acc;
+      if (s[t] > mx) mx = s[t];
+      n++;
+    }
+    if (n == 0) {
+      if (J->lse) J->lse[(int64_t)row * J->H + h] = -INFINITY;
+      continue;
+    }
+    double sum = 0.0;
+    for (int t = 0; t < J->topk; t++)
+      if (s[t] != -INFINITY) sum += exp(s[t] - mx);
+    for (int t = 0; t < J->topk; t++) {
+      if (s[t] == -INFINITY) continue;
+      const int j = ir[t] >= 0 ? ir[t] : 0;
+      const double w = g_mutation == 12 ? exp(s[t] - mx) : exp(s[t] - mx) / sum;
+      const uint16_t *vr = (g_mutation == 13 ? J->k : J->v) + (kbase + j) * J->dv;
+      for (int d = 0; d < J->dv; d++) o[d] += w * bf16_value(vr[d]);
+    }
+    if (J->lse) J->lse[(int64_t)row * J->H + h] = mx + log(sum);
+  }
+}
+
+static void *att_worker(void *arg) {
+  att_job *J = (att_job *)arg;
+  double *s = (double *)malloc(sizeof(double) * (size_t)(J->topk > 0 ? J->topk : 1));
+  if (!s) {
+    pthread_mutex_lock(&J->mu);
+    J->err = ORC_ERR_ALLOC;
+    pthread_mutex_unlock(&J->mu);
+    return NULL;
+  }
+  for (;;) {
+    pthread_mutex_lock(&J->mu);
+    const int row = J->next++;
+    pthread_mutex_unlock(&J->mu);
+    if (row >= J->total_q) break;
+    att_row(J, row, s);
+  }
+  free(s);
+  return NULL;
+}
+
+int oracle_sparse_attention(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                            const int32_t *idx, const int32_t *cu_q, const int32_t *cu_k, int S,
+                            int total_q, int H, int dv, int topk, double scale, double *out,
+                            double *lse, int nthreads) {
+  if (!q || !k || !v || !idx || !cu_q || !cu_k || !out || S < 1 || total_q < 0 || H < 1 ||
+      dv < 1 || topk < 1)
+    return ORC_ERR_ARG;
+  if (cu_q[0] != 0 || cu_q[S] != total_q) return ORC_ERR_ARG;
+  att_job J = {q, k, v, idx, cu_q, cu_k, S, total_q, H, dv, topk, scale, out, lse, 0, 0,
+               PTHREAD_MUTEX_INITIALIZER};
+  if (nthreads <= 0) nthreads = (int)sysconf(_SC_NPROCESSORS_ONLN);
+  if (nthreads < 1) nthreads = 1;
+  if (nthreads > 256) nthreads = 256;
+  pthread_t th[256];
+  int started = 0;
+  for (int t = 0; t < nthreads; t++)
+    if (pthread_create(&th[t], NULL, att_worker, &J) == 0) started++;
+  if (started == 0) att_worker(&J);
+  for (int t = 0; t < started; t++) pthread_join(th[t], NULL);
+  return J.err;
+}

@@ -299,7 +299,123 @@ def pin_scaling_and_ties():
         assert list(idx[pos]) == want, pos
 
 
+# ---------------------------------------------------------------------------
+# the sparse attention step over the selected tokens
+
+def _att_case(rng, S, H, dv, topk, lengths):
+    """Random tiny attention problem: small-integer bf16 q/k/v, index rows with
+    padding and arbitrary order."""
+    cu_k = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    rows_k = int(cu_k[-1])
+    k = _bf(rng.integers(-3, 4, size=(rows_k, dv)).astype(np.float32))
+    v = _bf(rng.integers(-5, 6, size=(rows_k, dv)).astype(np.float32))
+    nq = [int(rng.integers(1, 4)) for _ in range(S)]
+    cu_q = np.concatenate([[0], np.cumsum(nq)]).astype(np.int32)
+    total_q = int(cu_q[-1])
+    q = _bf(rng.integers(-2, 3, size=(total_q, H, dv)).astype(np.float32))
+    idx = np.full((total_q, topk), -1, np.int32)
+    for s_ in range(S):
+        for r in range(int(cu_q[s_]), int(cu_q[s_ + 1])):
+            n = int(rng.integers(0, min(topk, lengths[s_]) + 1))
+            sel = rng.choice(lengths[s_], size=n, replace=False)
+            slots = rng.choice(topk, size=n, replace=False)
+            idx[r, slots] = sel
+    return q, k, v, idx, cu_q, cu_k
+
+
+def _att_brute_row(q, k, v, idx, cu_q, cu_k, row, scale):
+    s_ = int(np.searchsorted(cu_q, row, side="right") - 1)
+    base = int(cu_k[s_])
+    kf, vf, qf = bf16_to_f32(k).astype(float), bf16_to_f32(v).astype(float), bf16_to_f32(q[row]).astype(float)
+    n = int(cu_k[s_ + 1]) - base
+    keys = {j: list(kf[base + j]) for j in range(n)}
+    vals = {j: list(vf[base + j]) for j in range(n)}
+    return brute.attention([list(x) for x in qf], keys, vals, list(idx[row]), scale)
+
+
+def pin_attention_brute():
+    rng = np.random.Generator(np.random.PCG64(77))
+    for case in range(8):
+        H, dv, topk = [(1, 2, 3), (3, 5, 4), (2, 4, 6), (1, 7, 5)][case % 4]
+        lengths = [int(x) for x in rng.integers(2, 9, size=int(rng.integers(1, 4)))]
+        q, k, v, idx, cu_q, cu_k = _att_case(rng, len(lengths), H, dv, topk, lengths)
+        scale = float(rng.uniform(0.1, 0.9))
+        out, lse = oracle.sparse_attention(q, k, v, idx, cu_q, cu_k, H, scale, nthreads=2)
+        for row in range(idx.shape[0]):
+            bo, bl = _att_brute_row(q, k, v, idx, cu_q, cu_k, row, scale)
+            assert np.allclose(out[row], np.array(bo), rtol=1e-12, atol=1e-12), (case, row)
+            for h in range(H):
+                if np.isinf(bl[h]):
+                    assert np.isinf(lse[row, h]) and lse[row, h] < 0
+                else:
+                    assert abs(lse[row, h] - bl[h]) <= 1e-12 * max(1.0, abs(bl[h])), (case, row)
+
+
+def pin_attention_golden():
+    g = json.load(open(os.path.join(GOLDEN, "attention_example.json")))
+    k = _bf(np.asarray(g["keys"], np.float32))
+    v = _bf(np.asarray(g["values"], np.float32))
+    q = _bf(np.asarray(g["q"], np.float32).reshape(1, 1, -1))
+    idx = np.asarray([g["idx"]], np.int32)
+    cu_q, cu_k = np.array([0, 1], np.int32), np.array([0, 2], np.int32)
+    out, lse = oracle.sparse_attention(q, k, v, idx, cu_q, cu_k, 1, np.log(3.0))
+    assert np.allclose(out[0, 0], g["out"], rtol=0, atol=1e-14), out
+    assert abs(lse[0, 0] - np.log(4.0)) < 1e-14, lse
+    out2, _ = oracle.sparse_attention(q, k, v, idx[:, ::-1].copy(), cu_q, cu_k, 1, np.log(3.0))
+    assert np.allclose(out2, out, rtol=0, atol=1e-14)
+
+
+def pin_attention_single_index():
+    """One selected token: its weight is 1, the output is its value row, lse its score."""
+    rng = np.random.Generator(np.random.PCG64(78))
+    q, k, v, idx, cu_q, cu_k = _att_case(rng, 2, 2, 6, 5, [7, 5])
+    idx[:] = -1
+    for row in range(idx.shape[0]):
+        s_ = int(np.searchsorted(cu_q, row, side="right") - 1)
+        idx[row, row % 5] = row % (int(cu_k[s_ + 1]) - int(cu_k[s_]))
+    out, lse = oracle.sparse_attention(q, k, v, idx, cu_q, cu_k, 2, 0.5)
+    vf, kf, qf = bf16_to_f32(v).astype(float), bf16_to_f32(k).astype(float), bf16_to_f32(q).astype(float)
+    for row in range(idx.shape[0]):
+        s_ = int(np.searchsorted(cu_q, row, side="right") - 1)
+        j = int(cu_k[s_]) + int(idx[row].max())
+        for h in range(2):
+            assert np.array_equal(out[row, h], vf[j]), (row, h)
+            assert lse[row, h] == 0.5 * float(np.dot(qf[row, h], kf[j]))
+
+
+def pin_attention_uniform():
+    """A zero query scores every token 0: the output is the mean of the selected values."""
+    rng = np.random.Generator(np.random.PCG64(79))
+    q, k, v, idx, cu_q, cu_k = _att_case(rng, 2, 3, 4, 6, [8, 6])
+    q[:] = 0
+    out, lse = oracle.sparse_attention(q, k, v, idx, cu_q, cu_k, 3, 0.7)
+    vf = bf16_to_f32(v).astype(float)
+    for row in range(idx.shape[0]):
+        s_ = int(np.searchsorted(cu_q, row, side="right") - 1)
+        sel = [int(cu_k[s_]) + int(j) for j in idx[row] if j >= 0]
+        for h in range(3):
+            if not sel:
+                assert np.all(out[row, h] == 0)
+                continue
+            exact = [float(sum(Fraction(vf[j][d]) for j in sel) / len(sel)) for d in range(4)]
+            assert np.allclose(out[row, h], exact, rtol=1e-14, atol=1e-14), (row, h)
+            assert abs(lse[row, h] - np.log(len(sel))) < 1e-13
+
+
+def pin_attention_order_invariant():
+    """The output does not depend on where the selected tokens sit in the index row."""
+    rng = np.random.Generator(np.random.PCG64(80))
+    q, k, v, idx, cu_q, cu_k = _att_case(rng, 3, 2, 5, 6, [9, 4, 7])
+    out, lse = oracle.sparse_attention(q, k, v, idx, cu_q, cu_k, 2, 0.3)
+    perm = np.stack([rng.permutation(row) for row in idx])
+    out2, lse2 = oracle.sparse_attention(q, k, v, perm, cu_q, cu_k, 2, 0.3)
+    assert np.allclose(out, out2, rtol=1e-13, atol=1e-13)
+    assert np.allclose(lse, lse2, rtol=1e-13, atol=1e-13)
+
+
 ALL_PINS = [
+    pin_attention_brute, pin_attention_golden, pin_attention_single_index,
+    pin_attention_uniform, pin_attention_order_invariant,
     pin_golden_three_block,
     pin_golden_five_block,
     pin_brute_force,

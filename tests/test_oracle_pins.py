@@ -16,6 +16,10 @@ MUTATIONS = {
     7: "block scores negated (lowest blocks kept)",
     8: "first block not forced",
     9: "take-all threshold off by one (m+1 blocks kept)",
+    10: "attention reads a padding entry as token 0",
+    11: "attention scores not scaled",
+    12: "attention weights not normalised",
+    13: "attention values read from the key rows",
 }
 
 
