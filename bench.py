@@ -508,6 +508,7 @@ def extras(args, w4, q4, k4, cu_q4, cu_k4, sl4, out4, flush, stream, hbm_peak):
         del ov, wsv
     det["prefill_32k"]["variants"] = variants
     det["dsa_128k"]["hisa_speedup_over_dsa"] = None  # filled by the caller
+    det["attention"] = attention_bench(w3, o3, flush, stream, hbm_peak)
     del q3, k3, o3, d3, ws3, dws3
     torch.cuda.empty_cache()
     det["decode"] = decode_bench(flush, stream, hbm_peak)
@@ -592,6 +593,66 @@ def decode_bench(flush, stream, hbm_peak, n_states=4, steps=256):
             "algorithmic_MB_per_step": round(per_seq * S / 1e6, 2),
             "GBs": round(gbs, 1), "frac_of_hbm_peak": round(gbs / hbm_peak, 4),
             "states": n_states, "kernel_us_per_step_eager": breakdown}
+
+
+def attention_bench(w3, o3, flush, stream, hbm_peak, heads=16):
+    """The sparse attention step over the selected tokens (synthetic q/k/v of width
+    128, N(0,1) bf16, 16 heads sharing one key and one value row per token): decode
+    (16 queries, the indices HISA selects on the decode workload) and the 32K needle
+    prefill (the indices of its HISA run)."""
+    import torch
+    import sparse_attention_top_hisa_b200 as H
+    from synth import config_workload
+    res = {}
+    rng = np.random.Generator(np.random.PCG64(31))
+    D = 128
+    scale = 1.0 / np.sqrt(D)
+
+    def rnd(shape):
+        return to_dev_bf16(bf16_rows(rng, shape))
+
+    # decode: 16 sequences x 32768 keys, k = 2048
+    dw = config_workload(2, steps=1)
+    S, cap, m, K = dw.num_seqs, dw.capacity, dw.m, dw.topk
+    cu_k, cu_q = to_dev_i32(dw.cu_k), to_dev_i32(np.arange(S + 1))
+    kc, lens = to_dev_bf16(dw.k_cache), to_dev_i32(dw.seqlens0)
+    reps = H.hisa_pool_blocks(kc, cu_k, lens, cap)
+    idx = H.hisa_select(to_dev_bf16(dw.queries[0]), kc, reps, cu_q, cu_k, lens, cap, m, K)
+    ka, va = rnd((S * cap, D)), rnd((S * cap, D))
+    qa = rnd((S * heads, D)).view(S, heads, D)
+    out = torch.empty(S, heads, D, dtype=torch.float32, device="cuda")
+    fn = lambda: H.hisa_sparse_attention(qa, ka, va, idx, cu_q, cu_k, scale, out=out)
+    fn()
+    us = statistics.median(time_events(fn, 5, flush, stream)) * 1e3
+    nbytes = S * (K * 2 * D * 2 + heads * D * 2 + heads * D * 4)
+    res["decode_16q"] = {"heads": heads, "k": K, "us": round(us, 2),
+                         "algorithmic_MB": round(nbytes / 1e6, 2),
+                         "GBs": round(nbytes / (us * 1e-6) / 1e9, 1),
+                         "frac_of_hbm_peak": round(nbytes / (us * 1e-6) / 1e9 / hbm_peak, 4)}
+    del kc, reps, ka, va, qa, out
+    # prefill: the 32K needle prefill's HISA indices
+    nq = w3.total_q
+    ka, va = rnd((w3.k.shape[0], D)), rnd((w3.k.shape[0], D))
+    qa = rnd((nq * heads, D)).view(nq, heads, D)
+    out = torch.empty(nq, heads, D, dtype=torch.float32, device="cuda")
+    cq, ck = to_dev_i32(w3.cu_q), to_dev_i32(w3.cu_k)
+    fn = lambda: H.hisa_sparse_attention(qa, ka, va, o3, cq, ck, scale, out=out)
+    fn()
+    ms = statistics.median(time_events(fn, 3, flush, stream))
+    valid = int((o3 >= 0).sum().item())
+    flop = 2.0 * 2.0 * heads * D * valid
+    res["prefill_32k"] = {"heads": heads, "k": w3.topk, "ms": round(ms, 3),
+                          "queries_per_s": round(nq / (ms / 1e3), 1),
+                          "TFLOPs": round(flop / (ms / 1e3) / 1e12, 2),
+                          "frac_of_fp32_alu_peak": round(flop / (ms / 1e3) / 1e12 / ALU_PEAK_TFLOPS, 4)}
+    del ka, va, qa, out
+    torch.cuda.empty_cache()
+    return res
+
+
+def bf16_rows(rng, shape):
+    from synth import bf16_from_f32
+    return bf16_from_f32(rng.standard_normal(shape, dtype=np.float32))
 
 
 def cpu_baseline(w, budget_s: float = 15.0):

@@ -195,6 +195,39 @@ hisa_status dsa_flat_select(const hisa_bf16 *q_idx, const hisa_bf16 *k_idx,
 size_t dsa_flat_workspace_size(int total_q, int num_seqs, int max_seqlen_k, int k);
 
 /*
+ * hisa_sparse_attention — the sparse attention step that consumes the selected
+ * indices (HISA summary page, paragraph on keeping the DSA output structure: the
+ * top-k token indices go unchanged to the sparse attention operator, which attends
+ * only to the selected tokens).  The pages name the operator without writing out its
+ * arithmetic; this library computes the textbook scaled dot-product attention
+ * restricted to the selection, with the heads of a query sharing its selection and
+ * one key row and one value row per token shared by every head (one latent KV head,
+ * as in multi-head latent attention):
+ *   s_j       = scale * q_att[i][h] . k_att[j]        for the entries j >= 0 of topk_idx[i]
+ *   out[i][h] = sum_j softmax(s)_j * v_att[j]          (fp32 accumulation)
+ *   lse[i][h] = log sum_j exp(s_j)                     (-inf for a row with no index)
+ *
+ *   q_att        bf16 [total_q, num_heads, HISA_ATT_DIM]
+ *   k_att, v_att bf16 [rows_k, HISA_ATT_DIM]: sequence s owns rows
+ *                [cu_seqlens_k[s], cu_seqlens_k[s+1]) (the indexer's key regions).
+ *   topk_idx     int32 [total_q, k]: sequence-local token positions, -1 = none (the
+ *                out_idx of hisa_select or dsa_flat_select).  A position outside the
+ *                sequence's region is ignored and HISA_ERR_INVALID_ARG is raised in
+ *                the device status word.
+ *   out (out)    fp32 [total_q, num_heads, HISA_ATT_DIM]; rows with no index are 0.
+ *   lse (out)    fp32 [total_q, num_heads] or NULL.
+ * 1 <= num_heads <= HISA_ATT_MAX_HEADS.  No workspace; q_att, k_att and v_att must be
+ * 16-byte aligned.
+ */
+#define HISA_ATT_DIM 128
+#define HISA_ATT_MAX_HEADS 32
+hisa_status hisa_sparse_attention(const hisa_bf16 *q_att, const hisa_bf16 *k_att,
+                                  const hisa_bf16 *v_att, const int32_t *topk_idx,
+                                  const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
+                                  int num_seqs, int total_q, int num_heads, int k, float scale,
+                                  float *out, float *lse, hisa_stream_t stream);
+
+/*
  * hisa_device_status — wait for `stream`, then copy the sticky device status word
  * of the current device into *status (0 = no device-side error; otherwise the
  * OR of (1 << hisa_status) bits).  clear != 0 resets the word afterwards.

@@ -7,6 +7,7 @@ provides device memory and streams.
 
 from .binding import (  # noqa: F401
     EXPORTED,
+    HISA_ATT_DIM,
     HISA_BLOCK,
     HISA_INDEX_DIM,
     HISA_MAX_M,
@@ -20,6 +21,7 @@ from .binding import (  # noqa: F401
     hisa_pool_blocks,
     hisa_select,
     hisa_select_workspace_size,
+    hisa_sparse_attention,
     hisa_timing_collect,
     hisa_timing_enable,
     lib,

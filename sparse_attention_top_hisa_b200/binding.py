@@ -46,6 +46,7 @@ EXPORTED = (
     "dsa_flat_select",
     "dsa_flat_workspace_size",
     "hisa_device_status",
+    "hisa_sparse_attention",
     "hisa_timing_enable",
     "hisa_kernel_kinds",
     "hisa_kernel_name",
@@ -91,8 +92,10 @@ def lib() -> ctypes.CDLL:
         L.hisa_kernel_name.restype = ctypes.c_char_p
         L.hisa_timing_collect.argtypes = [P, P, P, I, I]
         L.hisa_timing_collect.restype = I
+        L.hisa_sparse_attention.argtypes = [P, P, P, P, P, P, I, I, I, I, ctypes.c_float, P, P,
+                                            P]
         for f in ("hisa_pool_blocks", "hisa_append_keys", "hisa_select", "dsa_flat_select",
-                  "hisa_device_status"):
+                  "hisa_device_status", "hisa_sparse_attention"):
             getattr(L, f).restype = I
         _lib = L
     return _lib
@@ -257,3 +260,35 @@ def hisa_timing_collect(reset: bool = True) -> dict:
            "hisa_timing_collect")
     return {L.hisa_kernel_name(i).decode(): {"ms": ms[i], "launches": launches[i],
                                              "timed": timed[i]} for i in range(n)}
+
+
+HISA_ATT_DIM = 128
+
+
+def hisa_sparse_attention(q_att: torch.Tensor, k_att: torch.Tensor, v_att: torch.Tensor,
+                          topk_idx: torch.Tensor, cu_seqlens_q: torch.Tensor,
+                          cu_seqlens_k: torch.Tensor, scale: float,
+                          out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                          stream=None) -> torch.Tensor:
+    """Attention over each query's selected tokens; returns out fp32 [total_q, H, 128]."""
+    _need(q_att, "q_att", torch.bfloat16)
+    _need(k_att, "k_att", torch.bfloat16, HISA_ATT_DIM)
+    _need(v_att, "v_att", torch.bfloat16, HISA_ATT_DIM)
+    _need(topk_idx, "topk_idx", torch.int32)
+    _need(cu_seqlens_q, "cu_seqlens_q", torch.int32)
+    _need(cu_seqlens_k, "cu_seqlens_k", torch.int32)
+    if q_att.dim() != 3 or q_att.shape[2] != HISA_ATT_DIM:
+        raise ValueError(f"q_att must be [total_q, H, {HISA_ATT_DIM}], got {tuple(q_att.shape)}")
+    total_q, H = q_att.shape[0], q_att.shape[1]
+    if topk_idx.dim() != 2 or topk_idx.shape[0] != total_q:
+        raise ValueError("topk_idx must be [total_q, k]")
+    if out is None:
+        out = torch.empty(total_q, H, HISA_ATT_DIM, dtype=torch.float32, device=q_att.device)
+    _need(out, "out", torch.float32)
+    _need(lse, "lse", torch.float32, optional=True)
+    _check(lib().hisa_sparse_attention(_ptr(q_att), _ptr(k_att), _ptr(v_att), _ptr(topk_idx),
+                                       _ptr(cu_seqlens_q), _ptr(cu_seqlens_k),
+                                       cu_seqlens_q.numel() - 1, total_q, H, topk_idx.shape[1],
+                                       float(scale), _ptr(out), _ptr(lse), _stream(stream)),
+           "hisa_sparse_attention")
+    return out

@@ -34,6 +34,10 @@ cudaError_t launch_dsa(const uint16_t *q, const uint16_t *k, const int32_t *cu_q
 size_t dsa_workspace_bytes(int total_q, int num_seqs, int max_seqlen_k, int topk);
 bool use_tc_path(int total_q, int num_sms);
 bool decode_path_fits(int max_seqlen_k);
+cudaError_t launch_sparse_attention(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                                    const int32_t *idx, const int32_t *cu_q, const int32_t *cu_k,
+                                    int S, int total_q, int H, int topk, float scale, float *out,
+                                    float *lse, int num_sms, int *status, cudaStream_t st);
 cudaError_t launch_decode_select(const uint16_t *q, const uint16_t *k, const float *reps,
                                  const int32_t *cu_q, const int32_t *cu_k,
                                  const int32_t *seqlens, int S, int total_q, int max_seqlen_k,
@@ -51,7 +55,7 @@ const char *kKindNames[K_NUM_KINDS] = {
     "pool_blocks",        "append_keys",         "block_select",   "token_fused",
     "token_score_split",  "token_select_scratch", "key_norm",      "dsa_filter",
     "dsa_select",         "dsa_fallback",         "inv_lists",      "inv_scan",
-    "token_score_tc",     "reps_split",          "block_score_tc",  "decode_select"};
+    "token_score_tc",     "reps_split",          "block_score_tc",  "decode_select",  "sparse_attention"};
 long long g_launches[K_NUM_KINDS];
 double g_ms[K_NUM_KINDS];
 long long g_timed[K_NUM_KINDS];
@@ -277,6 +281,30 @@ hisa_status dsa_flat_select(const hisa_bf16 *q_idx, const hisa_bf16 *k_idx,
   return from_cuda(launch_dsa(q_idx, k_idx, cu_seqlens_q, cu_seqlens_k, seqlens_k, num_seqs,
                               total_q, max_seqlen_k, k, out_idx, out_scores,
                               static_cast<uint8_t *>(ws), st, static_cast<cudaStream_t>(stream)));
+}
+
+hisa_status hisa_sparse_attention(const hisa_bf16 *q_att, const hisa_bf16 *k_att,
+                                  const hisa_bf16 *v_att, const int32_t *topk_idx,
+                                  const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
+                                  int num_seqs, int total_q, int num_heads, int k, float scale,
+                                  float *out, float *lse, hisa_stream_t stream) {
+  if (num_heads < 1 || num_heads > HISA_ATT_MAX_HEADS || k < 1 || num_seqs < 0 || total_q < 0 ||
+      !(scale == scale))
+    return HISA_ERR_INVALID_ARG;
+  if (total_q == 0) return HISA_OK;
+  if (num_seqs == 0 || total_q >= (1 << 25)) return HISA_ERR_INVALID_ARG;
+  if (!q_att || !k_att || !v_att || !topk_idx || !cu_seqlens_q || !cu_seqlens_k || !out)
+    return HISA_ERR_INVALID_ARG;
+  if (!aligned(q_att, 16) || !aligned(k_att, 16) || !aligned(v_att, 16) ||
+      !aligned(topk_idx, 4) || !aligned(cu_seqlens_q, 4) || !aligned(cu_seqlens_k, 4) ||
+      !aligned(out, 4) || !aligned(lse, 4))
+    return HISA_ERR_UNALIGNED;
+  int *st = status_word();
+  if (!st) return HISA_ERR_CUDA;
+  return from_cuda(launch_sparse_attention(q_att, k_att, v_att, topk_idx, cu_seqlens_q,
+                                           cu_seqlens_k, num_seqs, total_q, num_heads, k, scale,
+                                           out, lse, num_sms(), st,
+                                           static_cast<cudaStream_t>(stream)));
 }
 
 hisa_status hisa_timing_enable(int on) {

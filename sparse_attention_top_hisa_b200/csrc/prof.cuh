@@ -24,6 +24,7 @@ enum KernelKind {
   K_REPS_SPLIT,
   K_BLOCK_SCORE_TC,
   K_DECODE_SELECT,
+  K_SPARSE_ATTENTION,
   K_NUM_KINDS
 };
 

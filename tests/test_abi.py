@@ -29,7 +29,8 @@ def lib():
 
 def test_header_declares_the_entry_points():
     names = declared_functions()
-    for n in ("hisa_pool_blocks", "hisa_append_keys", "hisa_select", "dsa_flat_select"):
+    for n in ("hisa_pool_blocks", "hisa_append_keys", "hisa_select", "dsa_flat_select",
+              "hisa_sparse_attention"):
         assert n in names
 
 
@@ -69,6 +70,18 @@ def test_host_validation_needs_no_gpu(lib):
     # empty problems are a no-op
     assert lib.hisa_select(None, None, None, None, None, None, 0, 0, 0, 128, 8, 16, None, None,
                            None, None, 0, None) == 0
+    # sparse attention: heads and k out of range, unaligned, empty
+    F = ctypes.c_float
+    assert lib.hisa_sparse_attention(dummy, dummy, dummy, dummy, dummy, dummy, 1, 4, 0, 16, F(0.1),
+                                     dummy, None, None) == 1
+    assert lib.hisa_sparse_attention(dummy, dummy, dummy, dummy, dummy, dummy, 1, 4, 33, 16,
+                                     F(0.1), dummy, None, None) == 1
+    assert lib.hisa_sparse_attention(dummy, dummy, dummy, dummy, dummy, dummy, 1, 4, 8, 0, F(0.1),
+                                     dummy, None, None) == 1
+    assert lib.hisa_sparse_attention(P(4096 + 2), dummy, dummy, dummy, dummy, dummy, 1, 4, 8, 16,
+                                     F(0.1), dummy, None, None) == 2
+    assert lib.hisa_sparse_attention(None, None, None, None, None, None, 0, 0, 8, 16, F(0.1), None,
+                                     None, None) == 0
     # unaligned pointers
     odd = P(4096 + 2)
     assert lib.hisa_select(odd, dummy, dummy, dummy, dummy, None, 1, 4, 128, 128, 8, 16, dummy,
