@@ -102,7 +102,8 @@ dsa_select_kernel(int row0, int topk, int cap, const float *__restrict__ buf_key
   LinShared &sh = *reinterpret_cast<LinShared *>(smem + (size_t)16 * topk);
   int32_t *oi = out_idx + (size_t)row * topk;
   float *os = out_scores ? out_scores + (size_t)row * topk : nullptr;
-  select_topk_reg<DSA_SEL_THREADS, DSA_SEL_KPT>(buf_key + (size_t)local * cap, n, topk, sh, work,
+  select_topk_reg<DSA_SEL_THREADS, DSA_SEL_KPT>(RowScores{buf_key + (size_t)local * cap}, n, topk,
+                                                sh, work,
                                                 DsaOut{oi, os, buf_j + (size_t)local * cap},
                                                 DsaPad{oi, os});
 }

@@ -280,11 +280,28 @@ __device__ __forceinline__ uint64_t rank_key(float s, int c) {
   return ((uint64_t)score_key(s) << 32) | (uint32_t)(~(uint32_t)c);
 }
 
-// sc: the n raw scores (global or shared memory, 16-byte aligned).
-// work: 4*k words (2*k uint64) of shared scratch.
-template <int NT, int KPT, class Out, class Pad>
-__device__ void select_topk_reg(const float *sc, int n, int k, LinShared &sh, uint32_t *work,
-                                Out out, Pad pad) {
+// Sources of a row of raw scores in candidate order.
+// A contiguous row (global or shared memory, 16-byte aligned):
+struct RowScores {
+  const float *p;
+  __device__ float4 ld4(int c) const { return *reinterpret_cast<const float4 *>(p + c); }
+  __device__ float ld1(int c) const { return p[c]; }
+};
+// A row assembled from segments of 128 scores: candidate c is score c % 128 of
+// segment seg[c / 128], which starts at base + seg[c / 128] * 128.
+struct SegScores {
+  const float *base;
+  const int32_t *seg;
+  __device__ const float *at(int c) const { return base + (size_t)seg[c >> 7] * 128 + (c & 127); }
+  __device__ float4 ld4(int c) const { return *reinterpret_cast<const float4 *>(at(c)); }
+  __device__ float ld1(int c) const { return *at(c); }
+};
+
+// sc: the n raw scores (RowScores or SegScores; four consecutive candidates never
+// straddle a segment).  work: 4*k words (2*k uint64) of shared scratch.
+template <int NT, int KPT, class Src, class Out, class Pad>
+__device__ void select_topk_reg(Src sc, int n, int k, LinShared &sh, uint32_t *work, Out out,
+                                Pad pad) {
   static_assert(KPT % 4 == 0, "scores are loaded four at a time");
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   constexpr int NW = NT / 32;
@@ -300,11 +317,11 @@ __device__ void select_topk_reg(const float *sc, int n, int k, LinShared &sh, ui
     const int c0 = (j * NT + tid) * 4;
     float4 v = make_float4(NEG, NEG, NEG, NEG);
     if (c0 + 3 < n) {
-      v = *reinterpret_cast<const float4 *>(sc + c0);
+      v = sc.ld4(c0);
     } else if (c0 < n) {
-      v.x = sc[c0];
-      if (c0 + 1 < n) v.y = sc[c0 + 1];
-      if (c0 + 2 < n) v.z = sc[c0 + 2];
+      v.x = sc.ld1(c0);
+      if (c0 + 1 < n) v.y = sc.ld1(c0 + 1);
+      if (c0 + 2 < n) v.z = sc.ld1(c0 + 2);
     }
     f[4 * j] = v.x;
     f[4 * j + 1] = v.y;
@@ -409,7 +426,7 @@ __device__ void select_topk_reg(const float *sc, int n, int k, LinShared &sh, ui
   if (nbnd > k) {  // heavy ties at the boundary: exact radix route
     __syncthreads();
     auto key = [&](int c) -> uint32_t {
-      const float x = sc[c];
+      const float x = sc.ld1(c);
       return x != NEG ? score_key(x) : 0u;
     };
     select_topk<NT>(key, n, k, sh.radix, work, reinterpret_cast<int *>(work + k), work + 2 * k,

@@ -86,9 +86,10 @@ struct RowPad {
   }
 };
 
-// shared memory of the selecting kernel: work (4k words) | LinShared | the block list
+// shared memory of the selecting kernel: work (4k words) | LinShared | the block list |
+// the score segments of the blocks
 __host__ __device__ inline size_t token_smem_bytes(int m, int topk) {
-  return (size_t)16 * topk + sizeof(LinShared) + (size_t)m * 4;
+  return (size_t)16 * topk + sizeof(LinShared) + (size_t)m * 8;
 }
 
 __global__ void __launch_bounds__(TS_THREADS)
@@ -119,11 +120,13 @@ __global__ void __launch_bounds__(NT, 1024 / NT)
 token_select_scratch_kernel(const int32_t *__restrict__ cu_q, const int32_t *__restrict__ cu_k,
                             const int32_t *__restrict__ seqlens, int S, int m, int topk,
                             const int32_t *__restrict__ blk, const float *__restrict__ scratch,
-                            int32_t *__restrict__ out_idx, float *__restrict__ out_scores) {
+                            const int32_t *__restrict__ pmap, int32_t *__restrict__ out_idx,
+                            float *__restrict__ out_scores) {
   extern __shared__ __align__(16) uint8_t smem[];
   uint32_t *work = reinterpret_cast<uint32_t *>(smem);
   LinShared &sh = *reinterpret_cast<LinShared *>(smem + (size_t)16 * topk);
   int32_t *sblk = reinterpret_cast<int32_t *>(smem + (size_t)16 * topk + sizeof(LinShared));
+  int32_t *sseg = sblk + m;
   const int row = blockIdx.x;
   RowPad pad{out_idx + (size_t)row * topk, out_scores ? out_scores + (size_t)row * topk : nullptr};
   const QueryInfo qi = locate(cu_q, cu_k, seqlens, S, row, nullptr);
@@ -133,10 +136,17 @@ token_select_scratch_kernel(const int32_t *__restrict__ cu_q, const int32_t *__r
   }
   // the block stage keeps exactly min(m, own block + 1) blocks of a valid query
   const int nsel = min(m, qi.pos / BLK + 1);
-  for (int i = threadIdx.x; i < nsel; i += NT) sblk[i] = blk[(size_t)row * m + i];
+  for (int i = threadIdx.x; i < nsel; i += NT) {
+    sblk[i] = blk[(size_t)row * m + i];
+    if (pmap) sseg[i] = pmap[(size_t)row * m + i];
+  }
   __syncthreads();
   TokenOut out{pad.idx, pad.scores, sblk};
-  select_topk_reg<NT, KPT>(scratch + (size_t)row * m * BLK, nsel * BLK, topk, sh, work, out, pad);
+  if (pmap)  // scores of slot i in segment sseg[i] of the buffer
+    select_topk_reg<NT, KPT>(SegScores{scratch, sseg}, nsel * BLK, topk, sh, work, out, pad);
+  else       // one contiguous score row per query
+    select_topk_reg<NT, KPT>(RowScores{scratch + (size_t)row * m * BLK}, nsel * BLK, topk, sh,
+                             work, out, pad);
 }
 
 // Tensor-core schedule when there are enough queries to fill the GPU with tiles;
@@ -149,8 +159,8 @@ size_t block_tc_workspace_bytes(int total_q, int num_seqs, int max_seqlen_k);
 cudaError_t launch_token_score_tc(const uint16_t *q, const uint16_t *k, const int32_t *cu_q,
                                   const int32_t *cu_k, const int32_t *seqlens, int S,
                                   int total_q, int max_seqlen_k, int m, const int32_t *blk,
-                                  uint8_t *ws, float **scores_out, int num_sms, int *status,
-                                  cudaStream_t st);
+                                  uint8_t *ws, float **scores_out, const int32_t **pmap_out,
+                                  int num_sms, int *status, cudaStream_t st);
 
 size_t token_scratch_bytes(int total_q, int num_seqs, int max_seqlen_k, int m, int num_sms) {
   if (token_use_split(total_q, num_sms)) return (size_t)total_q * m * BLK * 4;
@@ -168,6 +178,7 @@ cudaError_t launch_token_select(const uint16_t *q, const uint16_t *k, const int3
   if (total_q == 0) return cudaSuccess;
   cudaError_t e;
   float *scores = reinterpret_cast<float *>(ws);
+  const int32_t *pmap = nullptr;  // contiguous score rows unless the tensor-core path maps them
   if (token_use_split(total_q, num_sms)) {
     // spread each query's blocks over enough CTAs to cover the SMs about twice
     int splits = (2 * num_sms + total_q - 1) / total_q;
@@ -183,7 +194,7 @@ cudaError_t launch_token_select(const uint16_t *q, const uint16_t *k, const int3
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   } else {
     e = launch_token_score_tc(q, k, cu_q, cu_k, seqlens, S, total_q, max_seqlen_k, m, blk, ws,
-                              &scores, num_sms, status, st);
+                              &scores, &pmap, num_sms, status, st);
     if (e != cudaSuccess) return e;
   }
   const size_t smem = token_smem_bytes(m, topk);
@@ -194,29 +205,29 @@ cudaError_t launch_token_select(const uint16_t *q, const uint16_t *k, const int3
       auto kern = token_select_scratch_kernel<1024, 8>;
       if ((e = set_smem_once((const void *)kern, smem, attr_c)) != cudaSuccess) return e;
       ProfScope ps(K_TOKEN_SELECT_SCRATCH, st);
-      kern<<<total_q, 1024, smem, st>>>(cu_q, cu_k, seqlens, S, m, topk, blk, scores, out_idx,
-                                        out_scores);
+      kern<<<total_q, 1024, smem, st>>>(cu_q, cu_k, seqlens, S, m, topk, blk, scores, pmap,
+                                        out_idx, out_scores);
     } else {
       auto kern = token_select_scratch_kernel<1024, 16>;
       if ((e = set_smem_once((const void *)kern, smem, attr_d)) != cudaSuccess) return e;
       ProfScope ps(K_TOKEN_SELECT_SCRATCH, st);
-      kern<<<total_q, 1024, smem, st>>>(cu_q, cu_k, seqlens, S, m, topk, blk, scores, out_idx,
-                                        out_scores);
+      kern<<<total_q, 1024, smem, st>>>(cu_q, cu_k, seqlens, S, m, topk, blk, scores, pmap,
+                                        out_idx, out_scores);
     }
   } else if (m * BLK <= 256 * 32) {
     static int attr_a[64];
     auto kern = token_select_scratch_kernel<256, 32>;
     if ((e = set_smem_once((const void *)kern, smem, attr_a)) != cudaSuccess) return e;
     ProfScope ps(K_TOKEN_SELECT_SCRATCH, st);
-    kern<<<total_q, 256, smem, st>>>(cu_q, cu_k, seqlens, S, m, topk, blk, scores, out_idx,
-                                     out_scores);
+    kern<<<total_q, 256, smem, st>>>(cu_q, cu_k, seqlens, S, m, topk, blk, scores, pmap,
+                                     out_idx, out_scores);
   } else {
     static int attr_b[64];
     auto kern = token_select_scratch_kernel<512, 32>;
     if ((e = set_smem_once((const void *)kern, smem, attr_b)) != cudaSuccess) return e;
     ProfScope ps(K_TOKEN_SELECT_SCRATCH, st);
-    kern<<<total_q, 512, smem, st>>>(cu_q, cu_k, seqlens, S, m, topk, blk, scores, out_idx,
-                                     out_scores);
+    kern<<<total_q, 512, smem, st>>>(cu_q, cu_k, seqlens, S, m, topk, blk, scores, pmap,
+                                     out_idx, out_scores);
   }
   return cudaGetLastError();
 }

@@ -20,8 +20,9 @@
 //      TMEM accumulators, so that the loads, the MMAs and the epilogue of
 //      consecutive tiles overlap.  The accumulator lane is the key row: each of the
 //      eight epilogue warps owns 32 key rows (TMEM lane quarter w % 4) of half of the
-//      queries (w / 4), and every store instruction writes the 32 consecutive scores
-//      of one query (one 128-byte line of its score row);
+//      queries (w / 4).  The scores of list entry p (a (query, slot) pair) go to
+//      segment p of the score buffer (128 fp32), so a tile writes one contiguous run of
+//      segments and every store instruction one 128-byte line of it;
 //   4. the exact select of token_select.cu reads the score rows.
 // Key j of block b is admitted for a query at position i only when j <= i.
 #include <cudaTypedefs.h>
@@ -67,7 +68,8 @@ constexpr size_t TC_SMEM_BYTES = sizeof(TcSmem) + 1024;
 // more compact blocks than fit in shared memory uses global atomics directly.
 //   mode 0: add the pair counts of every key block to cnt;
 //   mode 1: reserve each key block's share of its list (cursor holds the list
-//           starts) and write the entries row << 7 | slot.
+//           starts), write the entries row << 7 | slot, and record each pair's list
+//           position in pmap[row * m + slot] (where its scores will be).
 constexpr int INV_THREADS = 256;
 constexpr int INV_ROWS = 256;
 constexpr int INV_LOCAL_BINS = 8192;
@@ -75,7 +77,8 @@ constexpr int INV_LOCAL_BINS = 8192;
 __global__ void __launch_bounds__(INV_THREADS)
 inv_lists_kernel(const int32_t *__restrict__ blk, int total_q, int m,
                  const int32_t *__restrict__ cu_q, int S, int emax, int mode,
-                 int *__restrict__ cnt, int *__restrict__ cursor, uint32_t *__restrict__ list) {
+                 int *__restrict__ cnt, int *__restrict__ cursor, uint32_t *__restrict__ list,
+                 int32_t *__restrict__ pmap) {
   __shared__ int loc[INV_LOCAL_BINS];
   __shared__ int seq_range[2];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -106,7 +109,9 @@ inv_lists_kernel(const int32_t *__restrict__ blk, int total_q, int m,
       walk([&](int, int, int cb) { atomicAdd(cnt + cb, 1); });
     else
       walk([&](int row, int slot, int cb) {
-        list[atomicAdd(cursor + cb, 1)] = ((uint32_t)row << 7) | (uint32_t)slot;
+        const int p = atomicAdd(cursor + cb, 1);
+        list[p] = ((uint32_t)row << 7) | (uint32_t)slot;
+        pmap[(size_t)row * m + slot] = p;
       });
     return;
   }
@@ -123,7 +128,9 @@ inv_lists_kernel(const int32_t *__restrict__ blk, int total_q, int m,
     if (loc[i]) loc[i] = atomicAdd(cursor + base + i, loc[i]);
   __syncthreads();
   walk([&](int row, int slot, int cb) {
-    list[atomicAdd(&loc[cb - base], 1)] = ((uint32_t)row << 7) | (uint32_t)slot;
+    const int p = atomicAdd(&loc[cb - base], 1);
+    list[p] = ((uint32_t)row << 7) | (uint32_t)slot;
+    pmap[(size_t)row * m + slot] = p;
   });
 }
 
@@ -303,7 +310,6 @@ token_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const uint16_t *
     // ---------------- epilogue: thread = key row of the block ----------------
     const int h = warp >> 2, quarter = warp & 3;
     const int r = quarter * 32 + lane;  // key row of the block
-    const size_t row_stride = (size_t)m * BLK;
     const float NEG = -__int_as_float(0x7f800000);
     int i = 0;
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x, i++) {
@@ -339,8 +345,8 @@ token_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const uint16_t *
             for (int u = 0; u < 32; u++) {
               const uint32_t e = __shfl_sync(0xffffffffu, ej[j], u);
               if (c0 + u < c_end) {
-                const int row = (int)(e >> 7), slot = (int)(e & 127u);
-                scratch[(size_t)row * row_stride + (size_t)slot * BLK + r] =
+                const int row = (int)(e >> 7);
+                scratch[(size_t)(td.list_off + c0 + u) * BLK + r] =
                     row >= rlim ? __uint_as_float(v[u]) : NEG;
               }
             }
@@ -394,7 +400,7 @@ bool make_key_tensor_map(CUtensorMap *map, const uint16_t *k) {
 }
 
 struct TcPlan {
-  size_t off_cnt, off_cursor, off_ntiles, off_tiles, off_list, off_scores, total;
+  size_t off_cnt, off_cursor, off_ntiles, off_tiles, off_list, off_pmap, off_scores, total;
   int nb, max_tiles;
 };
 
@@ -417,6 +423,8 @@ TcPlan tc_plan(int total_q, int num_seqs, int max_seqlen_k, int m) {
   off = a256(off + (size_t)p.max_tiles * sizeof(TileDesc));
   p.off_list = off;
   off = a256(off + (size_t)pairs * 4);
+  p.off_pmap = off;
+  off = a256(off + (size_t)pairs * 4);
   p.off_scores = off;
   off = a256(off + (size_t)pairs * BLK * 4);
   p.total = off;
@@ -427,13 +435,14 @@ size_t tc_workspace_bytes(int total_q, int num_seqs, int max_seqlen_k, int m) {
   return tc_plan(total_q, num_seqs, max_seqlen_k, m).total;
 }
 
-// Scores every selected (query, block) pair into ws's score rows
-// ([total_q][m * 128] order-preserving keys), ready for the select kernel.
+// Scores every selected (query, block) pair into ws's score buffer (one 128-score
+// segment per list entry; *pmap_out[row * m + slot] names the segment of each pair),
+// ready for the select kernel.
 cudaError_t launch_token_score_tc(const uint16_t *q, const uint16_t *k, const int32_t *cu_q,
                                   const int32_t *cu_k, const int32_t *seqlens, int S,
                                   int total_q, int max_seqlen_k, int m, const int32_t *blk,
-                                  uint8_t *ws, float **scores_out, int num_sms, int *status,
-                                  cudaStream_t st) {
+                                  uint8_t *ws, float **scores_out, const int32_t **pmap_out,
+                                  int num_sms, int *status, cudaStream_t st) {
   const TcPlan p = tc_plan(total_q, S, max_seqlen_k, m);
   const int emax = (max_seqlen_k + BLK - 1) / BLK;
   int *cnt = reinterpret_cast<int *>(ws + p.off_cnt);
@@ -442,7 +451,9 @@ cudaError_t launch_token_score_tc(const uint16_t *q, const uint16_t *k, const in
   TileDesc *tiles = reinterpret_cast<TileDesc *>(ws + p.off_tiles);
   uint32_t *list = reinterpret_cast<uint32_t *>(ws + p.off_list);
   float *scores = reinterpret_cast<float *>(ws + p.off_scores);
+  int32_t *pmap = reinterpret_cast<int32_t *>(ws + p.off_pmap);
   *scores_out = scores;
+  *pmap_out = pmap;
   CUtensorMap kmap;
   if (!make_key_tensor_map(&kmap, k)) return cudaErrorInvalidValue;
   cudaError_t e = cudaMemsetAsync(cnt, 0, (size_t)p.nb * 4, st);
@@ -450,7 +461,8 @@ cudaError_t launch_token_score_tc(const uint16_t *q, const uint16_t *k, const in
   const int grid = (total_q + INV_ROWS - 1) / INV_ROWS;
   {
     ProfScope ps(K_INV_LISTS, st);
-    inv_lists_kernel<<<grid, INV_THREADS, 0, st>>>(blk, total_q, m, cu_q, S, emax, 0, cnt, cursor, list);
+    inv_lists_kernel<<<grid, INV_THREADS, 0, st>>>(blk, total_q, m, cu_q, S, emax, 0, cnt, cursor, list,
+                                                   pmap);
   }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   {
@@ -460,7 +472,8 @@ cudaError_t launch_token_score_tc(const uint16_t *q, const uint16_t *k, const in
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   {
     ProfScope ps(K_INV_LISTS, st);
-    inv_lists_kernel<<<grid, INV_THREADS, 0, st>>>(blk, total_q, m, cu_q, S, emax, 1, cnt, cursor, list);
+    inv_lists_kernel<<<grid, INV_THREADS, 0, st>>>(blk, total_q, m, cu_q, S, emax, 1, cnt, cursor, list,
+                                                   pmap);
   }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   static int attr[64];
