@@ -95,6 +95,10 @@ __device__ __forceinline__ void cp_async_16(uint32_t dst, const void *src) {
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+// wait until at most one committed group of this thread is still in flight
+__device__ __forceinline__ void cp_async_wait_group1() {
+  asm volatile("cp.async.wait_group 1;" ::: "memory");
+}
 
 // make generic-proxy writes to shared memory (cp.async, st.shared) visible to the
 // async proxy (tcgen05.mma operand reads)

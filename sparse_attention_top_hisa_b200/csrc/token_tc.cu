@@ -15,7 +15,7 @@
 //      tile the key block arrives by TMA (or by cp.async when it is the partial last
 //      block of a sequence) and the selecting queries are gathered with cp.async into
 //      the 128-byte-swizzled K-major layout, through a three-stage shared-memory ring
-//      filled by three loader warps.  One thread issues the tcgen05.mma chain
+//      filled by three loader warps (each with two tiles' copies in flight).  One thread issues the tcgen05.mma chain
 //      S = K_b [128 x 64] . Q_sel^T [64 x N] (K = 4 x 16, N <= 256) into one of two
 //      TMEM accumulators, so that the loads, the MMAs and the epilogue of
 //      consecutive tiles overlap.  The accumulator lane is the key row: each of the
@@ -277,9 +277,19 @@ token_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const uint16_t *
           }
         }
       }
+      // two tiles in flight: tile i's copies were just issued; tile i - 1's are
+      // waited for here and its stage released to the MMA thread
+      cp_async_commit();
+      if (i > 0) {
+        cp_async_wait_group1();
+        fence_proxy_async_smem();
+        mbar_arrive(&sm.full[(i - 1) % TC_STAGES]);
+      }
+    }
+    if (i > 0) {  // the last tile issued (nothing is pending after an abort's break)
       cp_async_wait_all();
       fence_proxy_async_smem();
-      mbar_arrive(&sm.full[s]);
+      if (!*abort_flag) mbar_arrive(&sm.full[(i - 1) % TC_STAGES]);
     }
   } else if (warp == TC_MMA_WARP) {
     // ---------------- MMA issue (one thread) ----------------
