@@ -9,202 +9,282 @@
 // over the entries j >= 0 of the index row; the heads of a query share its selection
 // and one key row and one value row per token (the single latent KV head of MLA).
 //
-// The index row is split over the C CTAs of a cluster (C = 8 when there are too few
-// queries to fill the GPU, else 1).  Each CTA walks its share in tiles of 32 tokens:
-// the tiles' key and value rows are gathered into shared memory by a double-buffered
-// cp.async ring (rows padded to 272 bytes so that lanes reading different rows hit
-// different banks), warp w scores heads w, w + 8, ... for the 32 tokens (lane = token),
-// keeps a running maximum and sum per head (online softmax), and the 256 threads
-// accumulate the output rows (head, 8 dims each).  The C partial results are merged
-// through distributed shared memory: CTA c finishes the heads h with h % C == c.
+// The index row is split over the C CTAs of a cluster (up to 8 when there are too
+// few queries to fill the GPU, else 1); each CTA runs both products of its tiles of
+// 128 selected tokens on the tensor cores (below), keeps an online softmax per head,
+// and the C partial results are merged through distributed shared memory: CTA c
+// finishes the heads h with h % C == c.
 #include <cooperative_groups.h>
 
-#include "common.cuh"
 #include "prof.cuh"
+#include "tc.cuh"
 
 namespace cg = cooperative_groups;
 
 namespace hisa {
 
 constexpr int SA_DV = HISA_ATT_DIM;   // 128
-constexpr int SA_THREADS = 256;
-constexpr int SA_WARPS = SA_THREADS / 32;
-constexpr int SA_TILE = 32;            // tokens per tile
-constexpr int SA_MAXH = HISA_ATT_MAX_HEADS;
-constexpr int SA_ROWB = SA_DV * 2 + 16;  // padded shared-memory row (272 bytes)
 constexpr int SA_MAX_CLUSTER = 8;
 
-struct SaSmem {
-  float q[SA_MAXH][SA_DV];                 // the query's heads, fp32
-  uint8_t kt[2][SA_TILE * SA_ROWB];        // key rows of the tile (ring of two)
-  uint8_t vt[2][SA_TILE * SA_ROWB];        // value rows of the tile
-  float p[SA_MAXH][SA_TILE];               // scores, then probabilities
-  int tok[2][SA_TILE];                     // token positions of the tile (-1 = none)
-  float m[SA_MAXH], l[SA_MAXH], alpha[SA_MAXH];
-  float opart[SA_MAXH][SA_DV];             // this CTA's unnormalised output (cluster merge)
+// ---------------------------------------------------------------------------
+// Tensor-core version.  Per tile of 128 selected tokens:
+//   S^T [128 tokens x Hp] = K_tile [128 x 128] . Q^T [128 x Hp]     (tcgen05, TMEM cols 0..)
+//   O^T [128 dims x Hp]  += V^T [128 x 128 tokens] . P^T [128 x Hp]  (TMEM cols 32..)
+// with Hp = the head count rounded up to 16.  Every operand is K-major with the
+// 128-byte swizzle (tiles of 64 K-elements, 8-row groups 1024 bytes apart): the key
+// tile is gathered with cp.async, the value tile is transposed while it is gathered
+// (two tokens' 16-byte pieces become four-byte pairs of eight V^T rows), and the
+// probabilities are split into bf16 hi + lo (two MMAs) so that they keep about 16
+// bits.  Thread t of the four warps is token t for the scores (online softmax per
+// head across the CTA, running maximum and sum in shared memory) and dimension t for
+// the output tile, which it folds into fp32 registers rescaled by the tile's factor.
+
+constexpr int AT_THREADS = 128;
+constexpr int AT_TILE = 128;                 // tokens per tile
+constexpr int AT_NH = 32;                    // head rows of the Q and P operands
+constexpr uint32_t AT_TMEM_COLS = 64;        // S^T in cols [0, 32), the O tile in [32, 64)
+
+struct AtSmem {
+  uint8_t kt[2 * AT_TILE * 128];   // key tile, two 64-dim atoms of 128 token rows
+  uint8_t vt[2 * SA_DV * 128];     // V^T tile, two 64-token atoms of 128 dim rows
+  uint8_t qb[2 * AT_NH * 128];     // Q, two 64-dim atoms of 32 head rows
+  uint8_t ph[2 * AT_NH * 128];     // P hi, two 64-token atoms of 32 head rows
+  uint8_t pl[2 * AT_NH * 128];     // P lo
+  int tok[AT_TILE];
+  float tmax[4][AT_NH], tsum[4][AT_NH];
+  float m[AT_NH], l[AT_NH], alpha[AT_NH], mnew[AT_NH];
+  float opart[AT_NH][SA_DV];
+  uint64_t bar_mma;
+  uint32_t tmem_base;
   int bad;
 };
+constexpr size_t AT_SMEM = sizeof(AtSmem) + 1024;
 
-__device__ __forceinline__ void sa_cp16(void *smem, const void *gmem) {
-  const unsigned s = (unsigned)__cvta_generic_to_shared(smem);
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gmem) : "memory");
+// byte offset of element (row, kidx) of a K-major SW128 operand whose 64-element atoms
+// hold `rows` rows each
+__device__ __forceinline__ uint32_t kmaj_off(int row, int kidx, int rows) {
+  return (uint32_t)((kidx >> 6) * rows * 128) + sw128_offset(row, (kidx & 63) >> 3) +
+         (uint32_t)((kidx & 7) * 2);
 }
 
-__global__ void __launch_bounds__(SA_THREADS, 1)
-sparse_attn_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ kv_k,
-                   const uint16_t *__restrict__ kv_v, const int32_t *__restrict__ idx,
-                   const int32_t *__restrict__ cu_q, const int32_t *__restrict__ cu_k, int S,
-                   int H, int topk, int per_cta, float scale, float *__restrict__ out,
-                   float *__restrict__ lse, int *status) {
-  extern __shared__ __align__(16) uint8_t sa_raw[];
-  SaSmem &sm = *reinterpret_cast<SaSmem *>(sa_raw);
+__device__ __forceinline__ uint16_t bf16_rn_bits(float x) {
+  const uint32_t u = __float_as_uint(x);
+  return (uint16_t)((u + 0x7fffu + ((u >> 16) & 1u)) >> 16);  // finite x
+}
+
+__global__ void __launch_bounds__(AT_THREADS, 1)
+sparse_attn_tc_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ kv_k,
+                      const uint16_t *__restrict__ kv_v, const int32_t *__restrict__ idx,
+                      const int32_t *__restrict__ cu_q, const int32_t *__restrict__ cu_k, int S,
+                      int H, int topk, int per_cta, float scale, float *__restrict__ out,
+                      float *__restrict__ lse, int *status) {
+  extern __shared__ uint8_t at_raw[];
+  AtSmem &sm = *reinterpret_cast<AtSmem *>((reinterpret_cast<uintptr_t>(at_raw) + 1023) &
+                                           ~(uintptr_t)1023);
   cg::cluster_group cl = cg::this_cluster();
   const int C = (int)cl.num_blocks();
   const int me = (int)cl.block_rank();
   const int row = blockIdx.x / C;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const float NEG = -__int_as_float(0x7f800000);
+  const int Hp = (H + 15) & ~15;
 
-  // the query's sequence (every CTA of the cluster finds the same one)
   const int s = find_seq(cu_q, S, row);
   const int kbase = __ldg(cu_k + s), kcap = __ldg(cu_k + s + 1) - kbase;
-  // the query's heads, fp32
-  for (int i = tid; i < H * SA_DV; i += SA_THREADS)
-    sm.q[i / SA_DV][i % SA_DV] = __uint_as_float((uint32_t)__ldg(q + (size_t)row * H * SA_DV + i) << 16);
-  if (tid < H) {
+  if (tid == 0) {
+    mbar_init(&sm.bar_mma, 1);
+    fence_barrier_init();
+    sm.bad = 0;
+  }
+  if (warp == 0) {
+    tmem_alloc(&sm.tmem_base, AT_TMEM_COLS);
+    tmem_relinquish();
+  }
+  // Q (zero rows for padded heads) and zeroed P rows for padded heads
+  for (int x = tid; x < AT_NH * 16; x += AT_THREADS) {
+    const int h = x >> 4, c = x & 15;
+    uint4 w = make_uint4(0u, 0u, 0u, 0u);
+    if (h < H) w = __ldg(reinterpret_cast<const uint4 *>(q + ((size_t)row * H + h) * SA_DV) + c);
+    *reinterpret_cast<uint4 *>(sm.qb + (c >> 3) * AT_NH * 128 + sw128_offset(h, c & 7)) = w;
+    const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+    *reinterpret_cast<uint4 *>(sm.ph + (c >> 3) * AT_NH * 128 + sw128_offset(h, c & 7)) = z;
+    *reinterpret_cast<uint4 *>(sm.pl + (c >> 3) * AT_NH * 128 + sw128_offset(h, c & 7)) = z;
+  }
+  if (tid < AT_NH) {
     sm.m[tid] = NEG;
     sm.l[tid] = 0.f;
   }
-  if (tid == 0) sm.bad = 0;
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+  const uint32_t skt = smem_u32(sm.kt), svt = smem_u32(sm.vt), sqb = smem_u32(sm.qb);
+  const uint32_t sph = smem_u32(sm.ph), spl = smem_u32(sm.pl);
+  const uint32_t id = idesc_bf16_f32(AT_TILE, Hp);
+
+  float oacc[AT_NH];
+#pragma unroll
+  for (int h = 0; h < AT_NH; h++) oacc[h] = 0.f;
 
   const int e0 = me * per_cta, e1 = min(topk, e0 + per_cta);
-  const int ntiles = e1 > e0 ? (e1 - e0 + SA_TILE - 1) / SA_TILE : 0;
+  const int ntiles = e1 > e0 ? (e1 - e0 + AT_TILE - 1) / AT_TILE : 0;
   const int32_t *irow = idx + (size_t)row * topk;
-  auto gather = [&](int t, int buf) {  // tile t into ring slot buf
-    const int base = e0 + t * SA_TILE;
-    if (tid < SA_TILE) {
+  uint32_t phase = 0;
+  for (int t = 0; t < ntiles; t++) {
+    const int base = e0 + t * AT_TILE;
+    {  // the tile's tokens (-1 = none; outside the region = none, reported)
       int j = base + tid < e1 ? __ldg(irow + base + tid) : -1;
-      if (j >= kcap) {  // outside the sequence's key region: not attended, reported
+      if (j >= kcap) {
         sm.bad = 1;
         j = -1;
       }
-      sm.tok[buf][tid] = j;
+      sm.tok[tid] = j < 0 ? -1 : j;
     }
     __syncthreads();
-    // 32 rows x 16 pieces of 16 bytes, for keys and for values
-    for (int x = tid; x < SA_TILE * 16; x += SA_THREADS) {
+    // key tile: row r = token, 16 pieces of 8 dims
+    for (int x = tid; x < AT_TILE * 16; x += AT_THREADS) {
       const int r = x >> 4, c = x & 15;
-      const int j = sm.tok[buf][r];
-      if (j >= 0) {
-        sa_cp16(sm.kt[buf] + r * SA_ROWB + c * 16, kv_k + (size_t)(kbase + j) * SA_DV + c * 8);
-        sa_cp16(sm.vt[buf] + r * SA_ROWB + c * 16, kv_v + (size_t)(kbase + j) * SA_DV + c * 8);
+      const int j = sm.tok[r];
+      if (j >= 0)
+        cp_async_16(skt + (c >> 3) * AT_TILE * 128 + sw128_offset(r, c & 7),
+                    kv_k + (size_t)(kbase + j) * SA_DV + c * 8);
+    }
+    cp_async_commit();
+    // V^T tile: token pair (2p, 2p + 1) x 8 dims -> eight 4-byte pairs, zeros for none.
+    // Lanes take consecutive pairs of one 8-dim piece: a warp's stores to a V^T row
+    // then cover 32 distinct banks (8 swizzled 16-byte chunks x 4 pairs).
+#pragma unroll 2
+    for (int x = tid; x < (AT_TILE / 2) * 16; x += AT_THREADS) {
+      const int pr = x & 63, c = x >> 6;
+      const int t0 = 2 * pr;
+      const int j0 = sm.tok[t0], j1 = sm.tok[t0 + 1];
+      uint4 a = make_uint4(0u, 0u, 0u, 0u), b = a;
+      if (j0 >= 0) a = __ldg(reinterpret_cast<const uint4 *>(kv_v + (size_t)(kbase + j0) * SA_DV) + c);
+      if (j1 >= 0) b = __ldg(reinterpret_cast<const uint4 *>(kv_v + (size_t)(kbase + j1) * SA_DV) + c);
+      const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int i = 0; i < 8; i++) {
+        const uint32_t lo16 = (i & 1) ? (aw[i >> 1] >> 16) : (aw[i >> 1] & 0xffffu);
+        const uint32_t hi16 = (i & 1) ? (bw[i >> 1] >> 16) : (bw[i >> 1] & 0xffffu);
+        *reinterpret_cast<uint32_t *>(sm.vt + kmaj_off(c * 8 + i, t0, SA_DV)) = lo16 | (hi16 << 16);
       }
     }
-    asm volatile("cp.async.commit_group;\n" ::: "memory");
-  };
-
-  // output accumulators: thread handles (head, 8 dims) pairs hg = tid, tid + 256
-  float oacc[2][8];
-#pragma unroll
-  for (int a = 0; a < 2; a++)
-#pragma unroll
-    for (int d = 0; d < 8; d++) oacc[a][d] = 0.f;
-
-  __syncthreads();
-  if (ntiles > 0) gather(0, 0);
-  for (int t = 0; t < ntiles; t++) {
-    const int buf = t & 1;
-    if (t + 1 < ntiles) {
-      gather(t + 1, buf ^ 1);
-      asm volatile("cp.async.wait_group 1;\n" ::: "memory");
-    } else {
-      asm volatile("cp.async.wait_group 0;\n" ::: "memory");
-    }
+    cp_async_wait_all();
+    fence_proxy_async_smem();
     __syncthreads();
-    // scores: warp w, heads w, w + 8, ...; lane = token of the tile
+    // S^T = K_tile . Q^T
+    if (tid == 0) {
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < 8; kk++)
+        umma_bf16(tmem, sdesc_k_sw128(skt + (kk >> 2) * AT_TILE * 128 + (kk & 3) * 32),
+                  sdesc_k_sw128(sqb + (kk >> 2) * AT_NH * 128 + (kk & 3) * 32), id, kk > 0);
+      umma_commit(&sm.bar_mma);
+    }
+    __syncwarp();
+    mbar_wait(&sm.bar_mma, phase, status);
+    phase ^= 1u;
+    tc_fence_after();
+    // scores of token tid, online softmax per head across the tile
+    float sc[AT_NH];
     {
-      const int j = sm.tok[buf][lane];
-      const uint8_t *kr = sm.kt[buf] + lane * SA_ROWB;
-      for (int h = warp; h < H; h += SA_WARPS) {
-        float acc = 0.f;
-        if (j >= 0) {
-#pragma unroll 4
-          for (int c = 0; c < 16; c++) {
-            const uint4 w = *reinterpret_cast<const uint4 *>(kr + c * 16);
-            const float4 qa = *reinterpret_cast<const float4 *>(&sm.q[h][c * 8]);
-            const float4 qb = *reinterpret_cast<const float4 *>(&sm.q[h][c * 8 + 4]);
-            acc = fmaf(qa.x, bf_lo(w.x), acc);
-            acc = fmaf(qa.y, bf_hi(w.x), acc);
-            acc = fmaf(qa.z, bf_lo(w.y), acc);
-            acc = fmaf(qa.w, bf_hi(w.y), acc);
-            acc = fmaf(qb.x, bf_lo(w.z), acc);
-            acc = fmaf(qb.y, bf_hi(w.z), acc);
-            acc = fmaf(qb.z, bf_lo(w.w), acc);
-            acc = fmaf(qb.w, bf_hi(w.w), acc);
-          }
-        }
-        const float sc = j >= 0 ? acc * scale : NEG;
-        // online softmax for head h over this tile
-        float tmax = sc;
+      uint32_t v[16];
+      tmem_ld16(tmem + lane_base, v);
+      tmem_wait_ld();
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, o));
-        const float m_old = sm.m[h];
-        const float m_new = fmaxf(m_old, tmax);
-        const float pj = (j >= 0) ? expf(sc - m_new) : 0.f;
-        float psum = pj;
+      for (int u = 0; u < 16; u++) sc[u] = __uint_as_float(v[u]);
+      if (Hp > 16) {
+        tmem_ld16(tmem + lane_base + 16, v);
+        tmem_wait_ld();
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) psum += __shfl_xor_sync(0xffffffffu, psum, o);
-        sm.p[h][lane] = pj;
-        __syncwarp();
-        if (lane == 0) {
-          const float a = (m_new == NEG) ? 1.f : expf(m_old - m_new);  // m_old = -inf gives 0
-          sm.alpha[h] = a;
-          sm.l[h] = sm.l[h] * a + psum;
-          sm.m[h] = m_new;
-        }
+        for (int u = 0; u < 16; u++) sc[16 + u] = __uint_as_float(v[u]);
+      }
+    }
+    const bool live = sm.tok[tid] >= 0;
+#pragma unroll
+    for (int h = 0; h < AT_NH; h++) {
+      if (h < H) {
+        sc[h] = live ? sc[h] * scale : NEG;
+        float mx = sc[h];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        if (lane == 0) sm.tmax[warp][h] = mx;
       }
     }
     __syncthreads();
-    // output rows: rescale, then add the tile's weighted values
+    if (tid < H) {
+      const float tm = fmaxf(fmaxf(sm.tmax[0][tid], sm.tmax[1][tid]),
+                             fmaxf(sm.tmax[2][tid], sm.tmax[3][tid]));
+      const float mo = sm.m[tid], mn = fmaxf(mo, tm);
+      sm.mnew[tid] = mn;
+      sm.alpha[tid] = (mn == NEG) ? 1.f : expf(mo - mn);  // mo = -inf gives 0
+    }
+    __syncthreads();
 #pragma unroll
-    for (int a = 0; a < 2; a++) {
-      const int hg = tid + a * SA_THREADS;
-      if (hg < H * 16) {
-        const int h = hg >> 4, dg = hg & 15;
-        const float al = sm.alpha[h];
+    for (int h = 0; h < AT_NH; h++) {
+      if (h < H) {
+        const float p = live ? expf(sc[h] - sm.mnew[h]) : 0.f;
+        const uint16_t hb = bf16_rn_bits(p);
+        const uint16_t lb = bf16_rn_bits(p - __uint_as_float((uint32_t)hb << 16));
+        *reinterpret_cast<uint16_t *>(sm.ph + kmaj_off(h, tid, AT_NH)) = hb;
+        *reinterpret_cast<uint16_t *>(sm.pl + kmaj_off(h, tid, AT_NH)) = lb;
+        float ps = p;
 #pragma unroll
-        for (int d = 0; d < 8; d++) oacc[a][d] *= al;
-        for (int r = 0; r < SA_TILE; r++) {
-          const float pr = sm.p[h][r];
-          if (pr != 0.f) {
-            const uint4 w = *reinterpret_cast<const uint4 *>(sm.vt[buf] + r * SA_ROWB + dg * 16);
-            oacc[a][0] = fmaf(pr, bf_lo(w.x), oacc[a][0]);
-            oacc[a][1] = fmaf(pr, bf_hi(w.x), oacc[a][1]);
-            oacc[a][2] = fmaf(pr, bf_lo(w.y), oacc[a][2]);
-            oacc[a][3] = fmaf(pr, bf_hi(w.y), oacc[a][3]);
-            oacc[a][4] = fmaf(pr, bf_lo(w.z), oacc[a][4]);
-            oacc[a][5] = fmaf(pr, bf_hi(w.z), oacc[a][5]);
-            oacc[a][6] = fmaf(pr, bf_lo(w.w), oacc[a][6]);
-            oacc[a][7] = fmaf(pr, bf_hi(w.w), oacc[a][7]);
-          }
-        }
+        for (int o = 16; o > 0; o >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
+        if (lane == 0) sm.tsum[warp][h] = ps;
       }
     }
-    __syncthreads();  // the ring slot is refilled by the next iteration's gather
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (tid < H) {
+      sm.l[tid] = sm.l[tid] * sm.alpha[tid] + (sm.tsum[0][tid] + sm.tsum[1][tid]) +
+                  (sm.tsum[2][tid] + sm.tsum[3][tid]);
+      sm.m[tid] = sm.mnew[tid];
+    }
+    // O^T tile = V^T . (P_hi + P_lo)^T
+    if (tid == 0) {
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < 8; kk++)
+        umma_bf16(tmem + 32, sdesc_k_sw128(svt + (kk >> 2) * SA_DV * 128 + (kk & 3) * 32),
+                  sdesc_k_sw128(sph + (kk >> 2) * AT_NH * 128 + (kk & 3) * 32), id, kk > 0);
+#pragma unroll
+      for (int kk = 0; kk < 8; kk++)
+        umma_bf16(tmem + 32, sdesc_k_sw128(svt + (kk >> 2) * SA_DV * 128 + (kk & 3) * 32),
+                  sdesc_k_sw128(spl + (kk >> 2) * AT_NH * 128 + (kk & 3) * 32), id, 1u);
+      umma_commit(&sm.bar_mma);
+    }
+    __syncwarp();
+    mbar_wait(&sm.bar_mma, phase, status);
+    phase ^= 1u;
+    tc_fence_after();
+    // fold the tile into dimension tid's accumulators
+    {
+      uint32_t v[16];
+      tmem_ld16(tmem + lane_base + 32, v);
+      tmem_wait_ld();
+#pragma unroll
+      for (int u = 0; u < 16; u++)
+        if (u < H) oacc[u] = fmaf(oacc[u], sm.alpha[u], __uint_as_float(v[u]));
+      if (Hp > 16) {
+        tmem_ld16(tmem + lane_base + 48, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int u = 0; u < 16; u++)
+          if (16 + u < H) oacc[16 + u] = fmaf(oacc[16 + u], sm.alpha[16 + u], __uint_as_float(v[u]));
+      }
+    }
+    tc_fence_before();
+    __syncthreads();  // the next tile overwrites the operands and the accumulators
   }
   if (tid == 0 && sm.bad) raise_status(status, HISA_ERR_INVALID_ARG);
 
-  // merge: this CTA's partial output into shared memory, then CTA c finishes heads
-  // h % C == c from every CTA's (max, sum, partial output)
+  // merge across the cluster: CTA c finishes heads h % C == c
 #pragma unroll
-  for (int a = 0; a < 2; a++) {
-    const int hg = tid + a * SA_THREADS;
-    if (hg < H * 16) {
-      const int h = hg >> 4, dg = hg & 15;
-#pragma unroll
-      for (int d = 0; d < 8; d++) sm.opart[h][dg * 8 + d] = oacc[a][d];
-    }
-  }
+  for (int h = 0; h < AT_NH; h++)
+    if (h < H) sm.opart[h][tid] = oacc[h];
   cl.sync();
   for (int h = me; h < H; h += C) {
     float M = NEG;
@@ -215,7 +295,7 @@ sparse_attn_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ 
       if (mc != NEG) L += expf(mc - M) * cl.map_shared_rank(&sm.l[0], c)[h];
     }
     float *orow = out + ((size_t)row * H + h) * SA_DV;
-    for (int d = tid; d < SA_DV; d += SA_THREADS) {
+    for (int d = tid; d < SA_DV; d += AT_THREADS) {
       float acc = 0.f;
       for (int c = 0; c < C; c++) {
         const float mc = cl.map_shared_rank(&sm.m[0], c)[h];
@@ -225,7 +305,8 @@ sparse_attn_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ 
     }
     if (lse && tid == 0) lse[(size_t)row * H + h] = L > 0.f ? M + logf(L) : NEG;
   }
-  cl.sync();  // every CTA's shared memory stays readable until the merge is done
+  cl.sync();
+  if (warp == 0) tmem_dealloc(tmem, AT_TMEM_COLS);
 }
 
 cudaError_t launch_sparse_attention(const uint16_t *q, const uint16_t *k, const uint16_t *v,
@@ -234,16 +315,16 @@ cudaError_t launch_sparse_attention(const uint16_t *q, const uint16_t *k, const 
                                     float *lse, int num_sms, int *status, cudaStream_t st) {
   if (total_q == 0) return cudaSuccess;
   static int attr[64];
-  cudaError_t e = set_smem_once((const void *)sparse_attn_kernel, sizeof(SaSmem), attr);
+  cudaError_t e = set_smem_once((const void *)sparse_attn_tc_kernel, AT_SMEM, attr);
   if (e != cudaSuccess) return e;
   int C = 1;
   while (C < SA_MAX_CLUSTER && total_q * C < 2 * num_sms) C *= 2;
   int per = (topk + C - 1) / C;
-  per = (per + SA_TILE - 1) / SA_TILE * SA_TILE;
+  per = (per + AT_TILE - 1) / AT_TILE * AT_TILE;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(total_q * C);
-  cfg.blockDim = dim3(SA_THREADS);
-  cfg.dynamicSmemBytes = sizeof(SaSmem);
+  cfg.blockDim = dim3(AT_THREADS);
+  cfg.dynamicSmemBytes = AT_SMEM;
   cfg.stream = st;
   cudaLaunchAttribute attrs[1];
   attrs[0].id = cudaLaunchAttributeClusterDimension;
@@ -253,8 +334,8 @@ cudaError_t launch_sparse_attention(const uint16_t *q, const uint16_t *k, const 
   cfg.attrs = attrs;
   cfg.numAttrs = 1;
   ProfScope ps(K_SPARSE_ATTENTION, st);
-  return cudaLaunchKernelEx(&cfg, sparse_attn_kernel, q, k, v, idx, cu_q, cu_k, S, H, topk, per,
-                            scale, out, lse, status);
+  return cudaLaunchKernelEx(&cfg, sparse_attn_tc_kernel, q, k, v, idx, cu_q, cu_k, S, H, topk,
+                            per, scale, out, lse, status);
 }
 
 }  // namespace hisa
