@@ -65,7 +65,8 @@ def parse_args():
                     help="profiling runs: flat-scan calls on the same workload after the timed steps")
     ap.add_argument("--decode-profile", type=int, default=0, metavar="N",
                     help="profiling runs: only N eager decode steps (16 x 32768 keys, append + "
-                         "selection on the default stream), then exit")
+                         "selection on the default stream) and two attention calls over the "
+                         "last selection, then exit")
     return ap.parse_args()
 
 
@@ -725,6 +726,13 @@ def decode_profile(steps):
     for i in range(steps):
         H.hisa_append_keys(kc, reps, cu_k, lens, newk[i])
         H.hisa_select(qs[i], kc, reps, cu_q, cu_k, lens, cap, m, K, out_idx=out, workspace=ws)
+    # then the attention step over the last selection (16 heads, width 128)
+    rng = np.random.Generator(np.random.PCG64(31))
+    ka = to_dev_bf16(bf16_rows(rng, (S * cap, 128)))
+    va = to_dev_bf16(bf16_rows(rng, (S * cap, 128)))
+    qa = to_dev_bf16(bf16_rows(rng, (S * 16, 128))).view(S, 16, 128)
+    for _ in range(2):
+        H.hisa_sparse_attention(qa, ka, va, out, cu_q, cu_k, 1.0 / np.sqrt(128))
     torch.cuda.synchronize()
     assert H.hisa_device_status() == 0
 
