@@ -45,10 +45,10 @@ L2_FLUSH_BYTES = 256 << 20
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from an ncu
 # capture, keyed by kernel kind, with the sha256 of the kernel's sources at capture time
 # (a changed source voids the figure).  token_select_scratch: captured on the 32768-token
-# prefill (1.203 GB for 1.84 M selected pairs, 0.987 of its algorithmic bytes) and scaled
+# prefill (1.212 GB for 1.84 M selected pairs, 0.995 of its algorithmic bytes) and scaled
 # to the 131072-token launch by selected pairs (8.13 M): see
 # profiles/token_select_scratch_prefill_L32768.md.
-TRAFFIC = {"token_select_scratch": (5203113956, "5ba765819dfc6bf0", ("token_select.cu", "select.cuh"))}
+TRAFFIC = {"token_select_scratch": (5241752391, "741119f642a38df2", ("token_select.cu", "select.cuh"))}
 
 
 def parse_args():
@@ -513,7 +513,30 @@ def extras(args, w4, q4, k4, cu_q4, cu_k4, sl4, out4, flush, stream, hbm_peak):
     del q3, k3, o3, d3, ws3, dws3
     torch.cuda.empty_cache()
     det["decode"] = decode_bench(flush, stream, hbm_peak)
+    det["hbm_stream_ceilings"] = stream_ceilings(stream)
     return det
+
+
+def stream_ceilings(stream, nbytes=4 << 30, reps=5):
+    """Plain torch fill (write only) and copy (read + write) of 4 GiB: the ceilings the
+    write-bound scoring kernel and the HBM peak are compared against."""
+    import torch
+    x = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    y = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    res = {}
+    for name, fn, moved in (("write_only_fill_GBs", lambda: x.fill_(3), nbytes),
+                            ("copy_read_plus_write_GBs", lambda: y.copy_(x), 2 * nbytes)):
+        fn()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            fn()
+        b.record(stream)
+        b.synchronize()
+        res[name] = round(moved / (a.elapsed_time(b) / reps / 1e3) / 1e9, 1)
+    del x, y
+    torch.cuda.empty_cache()
+    return res
 
 
 def decode_bench(flush, stream, hbm_peak, n_states=4, steps=256):
