@@ -25,36 +25,42 @@ namespace hisa {
 
 constexpr int SA_DV = HISA_ATT_DIM;   // 128
 constexpr int SA_MAX_CLUSTER = 8;
+static_assert(SA_DV == 128, "the merge and the tile layouts take 128-dim rows");
 
 // ---------------------------------------------------------------------------
 // Tensor-core version.  Per tile of 128 selected tokens:
 //   S^T [128 tokens x Hp] = K_tile [128 x 128] . Q^T [128 x Hp]     (tcgen05, TMEM cols 0..)
-//   O^T [128 dims x Hp]  += V^T [128 x 128 tokens] . P^T [128 x Hp]  (TMEM cols 32..)
-// with Hp = the head count rounded up to 16.  Every operand is K-major with the
-// 128-byte swizzle (tiles of 64 K-elements, 8-row groups 1024 bytes apart): the key
-// tile is gathered with cp.async, the value tile is transposed while it is gathered
-// (two tokens' 16-byte pieces become four-byte pairs of eight V^T rows), and the
-// probabilities are split into bf16 hi + lo (two MMAs) so that they keep about 16
-// bits.  Thread t of the four warps is token t for the scores (online softmax per
-// head across the CTA, running maximum and sum in shared memory) and dimension t for
-// the output tile, which it folds into fp32 registers rescaled by the tile's factor.
+//   O^T [128 dims x Hp]   = V^T [128 x 128 tokens] . P^T [128 x Hp] (TMEM cols 32..)
+// with Hp = the head count rounded up to 16.  The key and value tiles are gathered
+// with cp.async in the cache's own row layout (token rows, 128-byte swizzle): K is
+// the K-major A operand of the first product and V the MN-major A operand of the
+// second.  Q and the probabilities P are K-major B operands; P is split into bf16
+// hi + lo (two MMAs) so that it keeps about 16 bits.  Four loader warps fill a
+// two-stage ring; thread t of the four compute warps is token t for the scores
+// (online softmax per head, running maximum and sum in shared memory) and dimension
+// t for the output tile, which it folds into fp32 registers rescaled by the tile's
+// factor.  The next tile's score product is issued as soon as the current scores
+// have been read, so it runs under the softmax.
 
-constexpr int AT_THREADS = 128;
+constexpr int AT_COMPUTE = 128;              // warps 0-3: MMAs, softmax, output fold
+constexpr int AT_LOADERS = 128;              // warps 4-7: token ids, key and V^T tiles
+constexpr int AT_THREADS = AT_COMPUTE + AT_LOADERS;
 constexpr int AT_TILE = 128;                 // tokens per tile
 constexpr int AT_NH = 32;                    // head rows of the Q and P operands
 constexpr uint32_t AT_TMEM_COLS = 64;        // S^T in cols [0, 32), the O tile in [32, 64)
 
 struct AtSmem {
-  uint8_t kt[2 * AT_TILE * 128];   // key tile, two 64-dim atoms of 128 token rows
-  uint8_t vt[2 * SA_DV * 128];     // V^T tile, two 64-token atoms of 128 dim rows
-  uint8_t qb[2 * AT_NH * 128];     // Q, two 64-dim atoms of 32 head rows
-  uint8_t ph[2 * AT_NH * 128];     // P hi, two 64-token atoms of 32 head rows
-  uint8_t pl[2 * AT_NH * 128];     // P lo
-  int tok[AT_TILE];
-  float tmax[4][AT_NH], tsum[4][AT_NH];
-  float m[AT_NH], l[AT_NH], alpha[AT_NH], mnew[AT_NH];
+  uint8_t kt[2][2 * AT_TILE * 128];  // key tiles (two stages), two 64-dim atoms of 128 rows
+  uint8_t vt[2][2 * AT_TILE * 128];  // value tiles, same layout as the key tiles
+  uint8_t qb[2 * AT_NH * 128];       // Q, two 64-dim atoms of 32 head rows
+  uint8_t ph[2 * AT_NH * 128];       // P hi, two 64-token atoms of 32 head rows
+  uint8_t pl[2 * AT_NH * 128];       // P lo
+  int tok[2][AT_TILE];
+  float tmax[2][4][AT_NH], tsum[2][4][AT_NH];  // per warp and head, by tile parity
+  float m[AT_NH], l[AT_NH];
   float opart[AT_NH][SA_DV];
-  uint64_t bar_mma;
+  float wm[AT_NH][SA_MAX_CLUSTER], wl[AT_NH][SA_MAX_CLUSTER];  // merge weights per (head, rank)
+  uint64_t bar_s, bar_o, full[2], empty[2];
   uint32_t tmem_base;
   int bad;
 };
@@ -67,9 +73,186 @@ __device__ __forceinline__ uint32_t kmaj_off(int row, int kidx, int rows) {
          (uint32_t)((kidx & 7) * 2);
 }
 
+// barrier among the four compute warps only (the loaders never take id 1)
+__device__ __forceinline__ void compute_sync() {
+  asm volatile("bar.sync 1, %0;" ::"n"(AT_COMPUTE) : "memory");
+}
+
+// barrier among the four loader warps only
+__device__ __forceinline__ void loader_sync() {
+  asm volatile("bar.sync 2, %0;" ::"n"(AT_LOADERS) : "memory");
+}
+
+// Transposed warp reduction of NH values per lane (NH = 16 or 32): each step trades
+// half of the live values with the partner lane and combines the other half, so the
+// whole reduction takes NH - 1 independent shuffles.  Afterwards lane l holds the
+// result for head l (NH = 32) or head l >> 1 (NH = 16, lanes 2h and 2h + 1).
+template <int NH, bool MAX>
+__device__ __forceinline__ float xreduce(float (&v)[NH], int lane) {
+  constexpr int STEPS = NH == 32 ? 5 : 4;
+#pragma unroll
+  for (int st = 0; st < STEPS; st++) {
+    const int o = 16 >> st, half = (NH >> st) >> 1;
+    const bool up = (lane & o) != 0;
+#pragma unroll
+    for (int i = 0; i < half; i++) {
+      const float send = up ? v[i] : v[i + half];
+      const float keep = up ? v[i + half] : v[i];
+      const float r = __shfl_xor_sync(0xffffffffu, send, o);
+      v[i] = MAX ? fmaxf(keep, r) : keep + r;
+    }
+  }
+  if (NH == 16) {
+    const float r = __shfl_xor_sync(0xffffffffu, v[0], 1);
+    v[0] = MAX ? fmaxf(v[0], r) : v[0] + r;
+  }
+  return v[0];
+}
+
 __device__ __forceinline__ uint16_t bf16_rn_bits(float x) {
   const uint32_t u = __float_as_uint(x);
   return (uint16_t)((u + 0x7fffu + ((u >> 16) & 1u)) >> 16);  // finite x
+}
+
+// The compute warps' side of one CTA: tiles 0 .. ntiles - 1 of stages t & 1; NH = the
+// padded head count (16 or 32), heads h >= H are masked.  Leaves the CTA's
+// unnormalised output for dimension tid in oacc and the running maximum and sum per
+// head in sm.m and sm.l.
+template <int NH>
+__device__ __forceinline__ void attn_compute(AtSmem &sm, uint32_t tmem, uint32_t sqb, int ntiles,
+                                             int H, float scale, int *status,
+                                             float (&oacc)[AT_NH]) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const float NEG = -__int_as_float(0x7f800000);
+  const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+  const uint32_t sph = smem_u32(sm.ph), spl = smem_u32(sm.pl);
+  const uint32_t id = idesc_bf16_f32(AT_TILE, NH), idv = idesc_bf16_f32_amn(SA_DV, NH);
+  const int hl = NH == 32 ? lane : lane >> 1;  // head whose warp reduction this lane holds
+  const bool hl_writer = NH == 32 || (lane & 1) == 0;
+
+  // S^T = K_tile . Q^T for tile t (thread 0)
+  auto issue_scores = [&](int t) {
+    const int st = t & 1;
+    mbar_wait(&sm.full[st], (uint32_t)(t >> 1) & 1u, status);
+    tc_fence_after();
+    const uint32_t skt = smem_u32(sm.kt[st]);
+#pragma unroll
+    for (int kk = 0; kk < 8; kk++)
+      umma_bf16(tmem, sdesc_k_sw128(skt + (kk >> 2) * AT_TILE * 128 + (kk & 3) * 32),
+                sdesc_k_sw128(sqb + (kk >> 2) * AT_NH * 128 + (kk & 3) * 32), id, kk > 0);
+    umma_commit(&sm.bar_s);
+  };
+  if (tid == 0 && ntiles > 0) issue_scores(0);
+  __syncwarp();
+
+  for (int t = 0; t < ntiles; t++) {
+    const int st = t & 1, par = t & 1;
+    // all compute threads see the stage filled (the tokens' liveness) and the scores
+    mbar_wait(&sm.full[st], (uint32_t)(t >> 1) & 1u, status);
+    const bool live = sm.tok[st][tid] >= 0;
+    mbar_wait(&sm.bar_s, (uint32_t)par, status);
+    tc_fence_after();
+    float sc[NH];
+    {
+      uint32_t v[16];
+      tmem_ld16(tmem + lane_base, v);
+      tmem_wait_ld();
+#pragma unroll
+      for (int u = 0; u < 16; u++) sc[u] = __uint_as_float(v[u]);
+      if (NH == 32) {
+        tmem_ld16(tmem + lane_base + 16, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int u = 0; u < 16; u++) sc[(16 + u) % NH] = __uint_as_float(v[u]);
+      }
+    }
+#pragma unroll
+    for (int h = 0; h < NH; h++) sc[h] = (live && h < H) ? sc[h] * scale : NEG;
+    {
+      float w[NH];
+#pragma unroll
+      for (int h = 0; h < NH; h++) w[h] = sc[h];
+      const float mx = xreduce<NH, true>(w, lane);
+      if (hl_writer) sm.tmax[par][warp][hl] = mx;
+    }
+    tc_fence_before();
+    compute_sync();  // (1) the tile's maxima are in; the scores in TMEM are consumed
+    if (tid == 0 && t + 1 < ntiles) issue_scores(t + 1);
+    __syncwarp();
+    // new running maximum and the rescale factor per head, probabilities of token tid
+    float mnew[NH], alpha[NH];
+#pragma unroll
+    for (int h = 0; h < NH; h++) {
+      const float mo = sm.m[h];
+      const float tm = fmaxf(fmaxf(sm.tmax[par][0][h], sm.tmax[par][1][h]),
+                             fmaxf(sm.tmax[par][2][h], sm.tmax[par][3][h]));
+      mnew[h] = fmaxf(mo, tm);
+      alpha[h] = (mnew[h] == NEG) ? 1.f : expf(mo - mnew[h]);  // mo = -inf gives 0
+    }
+    {
+      float w[NH];
+#pragma unroll
+      for (int h = 0; h < NH; h++) {
+        const float p = (live && h < H) ? expf(sc[h] - mnew[h]) : 0.f;
+        const uint16_t hb = bf16_rn_bits(p);
+        const uint16_t lb = bf16_rn_bits(p - __uint_as_float((uint32_t)hb << 16));
+        *reinterpret_cast<uint16_t *>(sm.ph + kmaj_off(h, tid, AT_NH)) = hb;
+        *reinterpret_cast<uint16_t *>(sm.pl + kmaj_off(h, tid, AT_NH)) = lb;
+        w[h] = p;
+      }
+      const float ps = xreduce<NH, false>(w, lane);
+      if (hl_writer) sm.tsum[par][warp][hl] = ps;
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    compute_sync();  // (2) P and the tile's sums are in; the previous fold is done
+    if (tid < H) {
+      const float mo = sm.m[tid];
+      const float tm = fmaxf(fmaxf(sm.tmax[par][0][tid], sm.tmax[par][1][tid]),
+                             fmaxf(sm.tmax[par][2][tid], sm.tmax[par][3][tid]));
+      const float mn = fmaxf(mo, tm);
+      const float al = (mn == NEG) ? 1.f : expf(mo - mn);
+      sm.l[tid] = sm.l[tid] * al + (sm.tsum[par][0][tid] + sm.tsum[par][1][tid]) +
+                  (sm.tsum[par][2][tid] + sm.tsum[par][3][tid]);
+      sm.m[tid] = mn;
+    }
+    // O^T tile = V^T . (P_hi + P_lo)^T, V^T read MN-major from the value rows: dims
+    // 0-63 and 64-127 are 16 KB apart, 8-token groups 1 KB apart, 16 tokens per MMA.
+    // The stage is free once these have run.
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t svt = smem_u32(sm.vt[st]);
+#pragma unroll
+      for (int kk = 0; kk < 8; kk++)
+        umma_bf16(tmem + 32, sdesc_mn_sw128(svt + kk * 2048, AT_TILE * 128, 1024),
+                  sdesc_k_sw128(sph + (kk >> 2) * AT_NH * 128 + (kk & 3) * 32), idv, kk > 0);
+#pragma unroll
+      for (int kk = 0; kk < 8; kk++)
+        umma_bf16(tmem + 32, sdesc_mn_sw128(svt + kk * 2048, AT_TILE * 128, 1024),
+                  sdesc_k_sw128(spl + (kk >> 2) * AT_NH * 128 + (kk & 3) * 32), idv, 1u);
+      umma_commit(&sm.bar_o);
+      if (t + 2 < ntiles) umma_commit(&sm.empty[st]);
+    }
+    __syncwarp();
+    mbar_wait(&sm.bar_o, (uint32_t)par, status);
+    tc_fence_after();
+    // fold the tile into dimension tid's accumulators
+    {
+      uint32_t v[16];
+      tmem_ld16(tmem + lane_base + 32, v);
+      tmem_wait_ld();
+#pragma unroll
+      for (int u = 0; u < 16; u++) oacc[u] = fmaf(oacc[u], alpha[u], __uint_as_float(v[u]));
+      if (NH == 32) {
+        tmem_ld16(tmem + lane_base + 48, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int u = 0; u < 16; u++)
+          oacc[16 + u] = fmaf(oacc[16 + u], alpha[(16 + u) % NH], __uint_as_float(v[u]));
+      }
+    }
+    tc_fence_before();
+  }
 }
 
 __global__ void __launch_bounds__(AT_THREADS, 1)
@@ -85,14 +268,19 @@ sparse_attn_tc_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict
   const int C = (int)cl.num_blocks();
   const int me = (int)cl.block_rank();
   const int row = blockIdx.x / C;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tid = threadIdx.x, warp = tid >> 5;
   const float NEG = -__int_as_float(0x7f800000);
   const int Hp = (H + 15) & ~15;
 
   const int s = find_seq(cu_q, S, row);
   const int kbase = __ldg(cu_k + s), kcap = __ldg(cu_k + s + 1) - kbase;
   if (tid == 0) {
-    mbar_init(&sm.bar_mma, 1);
+    mbar_init(&sm.bar_s, 1);
+    mbar_init(&sm.bar_o, 1);
+    for (int i = 0; i < 2; i++) {
+      mbar_init(&sm.full[i], AT_LOADERS);
+      mbar_init(&sm.empty[i], 1);
+    }
     fence_barrier_init();
     sm.bad = 0;
   }
@@ -117,193 +305,97 @@ sparse_attn_tc_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = sm.tmem_base;
-  const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-  const uint32_t skt = smem_u32(sm.kt), svt = smem_u32(sm.vt), sqb = smem_u32(sm.qb);
-  const uint32_t sph = smem_u32(sm.ph), spl = smem_u32(sm.pl);
-  const uint32_t id = idesc_bf16_f32(AT_TILE, Hp);
-
+  const uint32_t tmem = sm.tmem_base, sqb = smem_u32(sm.qb);
+  const int e0 = me * per_cta, e1 = min(topk, e0 + per_cta);
+  const int ntiles = e1 > e0 ? (e1 - e0 + AT_TILE - 1) / AT_TILE : 0;
+  const int32_t *irow = idx + (size_t)row * topk;
   float oacc[AT_NH];
 #pragma unroll
   for (int h = 0; h < AT_NH; h++) oacc[h] = 0.f;
 
-  const int e0 = me * per_cta, e1 = min(topk, e0 + per_cta);
-  const int ntiles = e1 > e0 ? (e1 - e0 + AT_TILE - 1) / AT_TILE : 0;
-  const int32_t *irow = idx + (size_t)row * topk;
-  uint32_t phase = 0;
-  for (int t = 0; t < ntiles; t++) {
-    const int base = e0 + t * AT_TILE;
-    {  // the tile's tokens (-1 = none; outside the region = none, reported)
-      int j = base + tid < e1 ? __ldg(irow + base + tid) : -1;
-      if (j >= kcap) {
-        sm.bad = 1;
-        j = -1;
+  if (tid >= AT_COMPUTE) {
+    // ---- loaders: fill stage t & 1 with the tile's token ids and its key and value
+    // rows; both tiles keep the row layout of the cache (token rows, dims contiguous),
+    // swizzled in 128-byte rows. Rows of no token are zeros.
+    const int lt = tid - AT_COMPUTE;
+    for (int t = 0; t < ntiles; t++) {
+      const int st = t & 1, base = e0 + t * AT_TILE;
+      if (t >= 2) mbar_wait(&sm.empty[st], (uint32_t)((t >> 1) - 1) & 1u, status);
+      {  // token of tile position lt (-1 = none; outside the region = none, reported)
+        const int j = base + lt < e1 ? __ldg(irow + base + lt) : -1;
+        if (j >= kcap) sm.bad = 1;
+        sm.tok[st][lt] = j < kcap ? j : -1;
       }
-      sm.tok[tid] = j < 0 ? -1 : j;
-    }
-    __syncthreads();
-    // key tile: row r = token, 16 pieces of 8 dims
-    for (int x = tid; x < AT_TILE * 16; x += AT_THREADS) {
-      const int r = x >> 4, c = x & 15;
-      const int j = sm.tok[r];
-      if (j >= 0)
-        cp_async_16(skt + (c >> 3) * AT_TILE * 128 + sw128_offset(r, c & 7),
-                    kv_k + (size_t)(kbase + j) * SA_DV + c * 8);
-    }
-    cp_async_commit();
-    // V^T tile: token pair (2p, 2p + 1) x 8 dims -> eight 4-byte pairs, zeros for none.
-    // Lanes take consecutive pairs of one 8-dim piece: a warp's stores to a V^T row
-    // then cover 32 distinct banks (8 swizzled 16-byte chunks x 4 pairs).
-#pragma unroll 2
-    for (int x = tid; x < (AT_TILE / 2) * 16; x += AT_THREADS) {
-      const int pr = x & 63, c = x >> 6;
-      const int t0 = 2 * pr;
-      const int j0 = sm.tok[t0], j1 = sm.tok[t0 + 1];
-      uint4 a = make_uint4(0u, 0u, 0u, 0u), b = a;
-      if (j0 >= 0) a = __ldg(reinterpret_cast<const uint4 *>(kv_v + (size_t)(kbase + j0) * SA_DV) + c);
-      if (j1 >= 0) b = __ldg(reinterpret_cast<const uint4 *>(kv_v + (size_t)(kbase + j1) * SA_DV) + c);
-      const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-      for (int i = 0; i < 8; i++) {
-        const uint32_t lo16 = (i & 1) ? (aw[i >> 1] >> 16) : (aw[i >> 1] & 0xffffu);
-        const uint32_t hi16 = (i & 1) ? (bw[i >> 1] >> 16) : (bw[i >> 1] & 0xffffu);
-        *reinterpret_cast<uint32_t *>(sm.vt + kmaj_off(c * 8 + i, t0, SA_DV)) = lo16 | (hi16 << 16);
+      loader_sync();
+      const uint32_t skt = smem_u32(sm.kt[st]), svt = smem_u32(sm.vt[st]);
+#pragma unroll 4
+      for (int x = lt; x < AT_TILE * 16; x += AT_LOADERS) {
+        const int r = x >> 4, c = x & 15;
+        const int j = sm.tok[st][r];
+        const uint32_t off = (c >> 3) * AT_TILE * 128 + sw128_offset(r, c & 7);
+        if (j >= 0) {
+          const size_t src = (size_t)(kbase + j) * SA_DV + c * 8;
+          cp_async_16(skt + off, kv_k + src);
+          cp_async_16(svt + off, kv_v + src);
+        } else {
+          const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+          *reinterpret_cast<uint4 *>(sm.kt[st] + off) = z;
+          *reinterpret_cast<uint4 *>(sm.vt[st] + off) = z;
+        }
       }
+      cp_async_commit();
+      cp_async_wait_all();
+      fence_proxy_async_smem();
+      mbar_arrive(&sm.full[st]);
     }
-    cp_async_wait_all();
-    fence_proxy_async_smem();
-    __syncthreads();
-    // S^T = K_tile . Q^T
-    if (tid == 0) {
-      tc_fence_after();
-#pragma unroll
-      for (int kk = 0; kk < 8; kk++)
-        umma_bf16(tmem, sdesc_k_sw128(skt + (kk >> 2) * AT_TILE * 128 + (kk & 3) * 32),
-                  sdesc_k_sw128(sqb + (kk >> 2) * AT_NH * 128 + (kk & 3) * 32), id, kk > 0);
-      umma_commit(&sm.bar_mma);
-    }
-    __syncwarp();
-    mbar_wait(&sm.bar_mma, phase, status);
-    phase ^= 1u;
-    tc_fence_after();
-    // scores of token tid, online softmax per head across the tile
-    float sc[AT_NH];
-    {
-      uint32_t v[16];
-      tmem_ld16(tmem + lane_base, v);
-      tmem_wait_ld();
-#pragma unroll
-      for (int u = 0; u < 16; u++) sc[u] = __uint_as_float(v[u]);
-      if (Hp > 16) {
-        tmem_ld16(tmem + lane_base + 16, v);
-        tmem_wait_ld();
-#pragma unroll
-        for (int u = 0; u < 16; u++) sc[16 + u] = __uint_as_float(v[u]);
-      }
-    }
-    const bool live = sm.tok[tid] >= 0;
-#pragma unroll
-    for (int h = 0; h < AT_NH; h++) {
-      if (h < H) {
-        sc[h] = live ? sc[h] * scale : NEG;
-        float mx = sc[h];
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        if (lane == 0) sm.tmax[warp][h] = mx;
-      }
-    }
-    __syncthreads();
-    if (tid < H) {
-      const float tm = fmaxf(fmaxf(sm.tmax[0][tid], sm.tmax[1][tid]),
-                             fmaxf(sm.tmax[2][tid], sm.tmax[3][tid]));
-      const float mo = sm.m[tid], mn = fmaxf(mo, tm);
-      sm.mnew[tid] = mn;
-      sm.alpha[tid] = (mn == NEG) ? 1.f : expf(mo - mn);  // mo = -inf gives 0
-    }
-    __syncthreads();
-#pragma unroll
-    for (int h = 0; h < AT_NH; h++) {
-      if (h < H) {
-        const float p = live ? expf(sc[h] - sm.mnew[h]) : 0.f;
-        const uint16_t hb = bf16_rn_bits(p);
-        const uint16_t lb = bf16_rn_bits(p - __uint_as_float((uint32_t)hb << 16));
-        *reinterpret_cast<uint16_t *>(sm.ph + kmaj_off(h, tid, AT_NH)) = hb;
-        *reinterpret_cast<uint16_t *>(sm.pl + kmaj_off(h, tid, AT_NH)) = lb;
-        float ps = p;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
-        if (lane == 0) sm.tsum[warp][h] = ps;
-      }
-    }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    if (tid < H) {
-      sm.l[tid] = sm.l[tid] * sm.alpha[tid] + (sm.tsum[0][tid] + sm.tsum[1][tid]) +
-                  (sm.tsum[2][tid] + sm.tsum[3][tid]);
-      sm.m[tid] = sm.mnew[tid];
-    }
-    // O^T tile = V^T . (P_hi + P_lo)^T
-    if (tid == 0) {
-      tc_fence_after();
-#pragma unroll
-      for (int kk = 0; kk < 8; kk++)
-        umma_bf16(tmem + 32, sdesc_k_sw128(svt + (kk >> 2) * SA_DV * 128 + (kk & 3) * 32),
-                  sdesc_k_sw128(sph + (kk >> 2) * AT_NH * 128 + (kk & 3) * 32), id, kk > 0);
-#pragma unroll
-      for (int kk = 0; kk < 8; kk++)
-        umma_bf16(tmem + 32, sdesc_k_sw128(svt + (kk >> 2) * SA_DV * 128 + (kk & 3) * 32),
-                  sdesc_k_sw128(spl + (kk >> 2) * AT_NH * 128 + (kk & 3) * 32), id, 1u);
-      umma_commit(&sm.bar_mma);
-    }
-    __syncwarp();
-    mbar_wait(&sm.bar_mma, phase, status);
-    phase ^= 1u;
-    tc_fence_after();
-    // fold the tile into dimension tid's accumulators
-    {
-      uint32_t v[16];
-      tmem_ld16(tmem + lane_base + 32, v);
-      tmem_wait_ld();
-#pragma unroll
-      for (int u = 0; u < 16; u++)
-        if (u < H) oacc[u] = fmaf(oacc[u], sm.alpha[u], __uint_as_float(v[u]));
-      if (Hp > 16) {
-        tmem_ld16(tmem + lane_base + 48, v);
-        tmem_wait_ld();
-#pragma unroll
-        for (int u = 0; u < 16; u++)
-          if (16 + u < H) oacc[16 + u] = fmaf(oacc[16 + u], sm.alpha[16 + u], __uint_as_float(v[u]));
-      }
-    }
-    tc_fence_before();
-    __syncthreads();  // the next tile overwrites the operands and the accumulators
+  } else if (Hp == 16) {
+    attn_compute<16>(sm, tmem, sqb, ntiles, H, scale, status, oacc);
+  } else {
+    attn_compute<32>(sm, tmem, sqb, ntiles, H, scale, status, oacc);
   }
+  __syncthreads();
   if (tid == 0 && sm.bad) raise_status(status, HISA_ERR_INVALID_ARG);
 
-  // merge across the cluster: CTA c finishes heads h % C == c
+  // merge across the cluster: CTA me finishes heads me, me + C, ... Every remote read
+  // of a step is issued at once: (head, rank) pairs, then (head, dim) outputs.
+  if (tid < AT_COMPUTE) {
 #pragma unroll
-  for (int h = 0; h < AT_NH; h++)
-    if (h < H) sm.opart[h][tid] = oacc[h];
+    for (int h = 0; h < AT_NH; h++)
+      if (h < H) sm.opart[h][tid] = oacc[h];
+  }
   cl.sync();
-  for (int h = me; h < H; h += C) {
+  const int nloc = me < H ? (H - me + C - 1) / C : 0;
+  if (tid < nloc * C) {
+    const int i = tid / C, c = tid - i * C, h = me + C * i;
+    sm.wm[i][c] = cl.map_shared_rank(&sm.m[0], c)[h];
+    sm.wl[i][c] = cl.map_shared_rank(&sm.l[0], c)[h];
+  }
+  __syncthreads();
+  if (tid < nloc) {
     float M = NEG;
-    for (int c = 0; c < C; c++) M = fmaxf(M, cl.map_shared_rank(&sm.m[0], c)[h]);
+    for (int c = 0; c < C; c++) M = fmaxf(M, sm.wm[tid][c]);
     float L = 0.f;
     for (int c = 0; c < C; c++) {
-      const float mc = cl.map_shared_rank(&sm.m[0], c)[h];
-      if (mc != NEG) L += expf(mc - M) * cl.map_shared_rank(&sm.l[0], c)[h];
+      const float mc = sm.wm[tid][c];
+      sm.wm[tid][c] = mc != NEG ? expf(mc - M) : 0.f;
+      L += sm.wm[tid][c] * sm.wl[tid][c];
     }
-    float *orow = out + ((size_t)row * H + h) * SA_DV;
-    for (int d = tid; d < SA_DV; d += AT_THREADS) {
-      float acc = 0.f;
-      for (int c = 0; c < C; c++) {
-        const float mc = cl.map_shared_rank(&sm.m[0], c)[h];
-        if (mc != NEG) acc += expf(mc - M) * cl.map_shared_rank(&sm.opart[0][0], c)[h * SA_DV + d];
-      }
-      orow[d] = L > 0.f ? acc / L : 0.f;
-    }
-    if (lse && tid == 0) lse[(size_t)row * H + h] = L > 0.f ? M + logf(L) : NEG;
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+    for (int c = 0; c < C; c++) sm.wm[tid][c] *= inv;
+    if (lse) lse[(size_t)row * H + me + C * tid] = L > 0.f ? M + logf(L) : NEG;
+  }
+  __syncthreads();
+  for (int x = tid; x < nloc * SA_DV; x += AT_THREADS) {
+    const int i = x >> 7, d = x & (SA_DV - 1), h = me + C * i;
+    float part[SA_MAX_CLUSTER];
+#pragma unroll
+    for (int c = 0; c < SA_MAX_CLUSTER; c++)
+      part[c] = c < C ? cl.map_shared_rank(&sm.opart[0][0], c)[h * SA_DV + d] : 0.f;
+    float acc = 0.f;
+#pragma unroll
+    for (int c = 0; c < SA_MAX_CLUSTER; c++)
+      if (c < C) acc = fmaf(sm.wm[i][c], part[c], acc);
+    out[((size_t)row * H + h) * SA_DV + d] = acc;
   }
   cl.sync();
   if (warp == 0) tmem_dealloc(tmem, AT_TMEM_COLS);
@@ -317,22 +409,43 @@ cudaError_t launch_sparse_attention(const uint16_t *q, const uint16_t *k, const 
   static int attr[64];
   cudaError_t e = set_smem_once((const void *)sparse_attn_tc_kernel, AT_SMEM, attr);
   if (e != cudaSuccess) return e;
-  int C = 1;
-  while (C < SA_MAX_CLUSTER && total_q * C < 2 * num_sms) C *= 2;
-  int per = (topk + C - 1) / C;
-  per = (per + AT_TILE - 1) / AT_TILE * AT_TILE;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(total_q * C);
   cfg.blockDim = dim3(AT_THREADS);
   cfg.dynamicSmemBytes = AT_SMEM;
   cfg.stream = st;
   cudaLaunchAttribute attrs[1];
   attrs[0].id = cudaLaunchAttributeClusterDimension;
-  attrs[0].val.clusterDim.x = C;
   attrs[0].val.clusterDim.y = 1;
   attrs[0].val.clusterDim.z = 1;
   cfg.attrs = attrs;
   cfg.numAttrs = 1;
+  // Split the rows over clusters of C CTAs while the grid is small, but only as far
+  // as every cluster of the launch can be resident at once (a second wave of
+  // clusters would cost more than the split saves).
+  static int fits[64][SA_MAX_CLUSTER + 1];  // clusters resident at once, per device
+  int dev = 0;
+  cudaGetDevice(&dev);
+  int C = 1;
+  while (C < SA_MAX_CLUSTER && total_q * C < 2 * num_sms) {
+    const int c2 = 2 * C;
+    int &n = fits[dev & 63][c2];
+    if (n == 0) {
+      cfg.gridDim = dim3(c2);
+      attrs[0].val.clusterDim.x = c2;
+      if (cudaOccupancyMaxActiveClusters(&n, sparse_attn_tc_kernel, &cfg) != cudaSuccess) {
+        (void)cudaGetLastError();  // the query's own error; the launch below decides
+        n = -1;
+      } else if (n <= 0) {
+        n = -1;
+      }
+    }
+    if (n < total_q) break;
+    C = c2;
+  }
+  int per = (topk + C - 1) / C;
+  per = (per + AT_TILE - 1) / AT_TILE * AT_TILE;
+  cfg.gridDim = dim3(total_q * C);
+  attrs[0].val.clusterDim.x = C;
   ProfScope ps(K_SPARSE_ATTENTION, st);
   return cudaLaunchKernelEx(&cfg, sparse_attn_tc_kernel, q, k, v, idx, cu_q, cu_k, S, H, topk,
                             per, scale, out, lse, status);

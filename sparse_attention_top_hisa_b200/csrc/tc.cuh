@@ -122,6 +122,20 @@ __device__ __forceinline__ uint64_t sdesc_k_sw128(uint32_t addr) {
   return d;
 }
 
+// Shared-memory descriptor of an MN-major SW128 bf16 operand: each 128-byte row holds
+// 64 consecutive M (or N) elements of one K index, rows k .. k + 7 form a 1024-byte
+// swizzle atom; `lbo` is the byte distance between 64-element groups along M (N) and
+// `sbo` the byte distance between 8-row groups along K (both multiples of 16).
+__device__ __forceinline__ uint64_t sdesc_mn_sw128(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((addr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1u << 46;
+  d |= (uint64_t)2u << 61;
+  return d;
+}
+
 // Instruction descriptor: bf16 x bf16 -> fp32, A and B K-major, shape M x N.
 __host__ __device__ __forceinline__ uint32_t idesc_bf16_f32(int M, int N) {
   return (1u << 4)                    // D format fp32
@@ -129,6 +143,10 @@ __host__ __device__ __forceinline__ uint32_t idesc_bf16_f32(int M, int N) {
          | (1u << 10)                 // B format bf16
          | ((uint32_t)(N >> 3) << 17) // N / 8
          | ((uint32_t)(M >> 4) << 24);// M / 16
+}
+// The same with A read MN-major (the transpose-A bit).
+__host__ __device__ __forceinline__ uint32_t idesc_bf16_f32_amn(int M, int N) {
+  return idesc_bf16_f32(M, N) | (1u << 15);
 }
 
 // ---------------------------------------------------------------------------
