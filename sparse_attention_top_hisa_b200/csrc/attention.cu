@@ -43,28 +43,30 @@ static_assert(SA_DV == 128, "the merge and the tile layouts take 128-dim rows");
 // have been read, so it runs under the softmax.
 
 constexpr int AT_COMPUTE = 128;              // warps 0-3: MMAs, softmax, output fold
-constexpr int AT_LOADERS = 128;              // warps 4-7: token ids, key and V^T tiles
+constexpr int AT_LOADERS = 128;              // warps 4-7: token ids, key and value tiles
 constexpr int AT_THREADS = AT_COMPUTE + AT_LOADERS;
 constexpr int AT_TILE = 128;                 // tokens per tile
-constexpr int AT_NH = 32;                    // head rows of the Q and P operands
-constexpr uint32_t AT_TMEM_COLS = 64;        // S^T in cols [0, 32), the O tile in [32, 64)
+constexpr int AT_STAGES = 3;                 // tiles in the loaders' ring
+constexpr int AT_NH = 32;                    // head rows of the Q operand
+constexpr uint32_t AT_TMEM_COLS = 128;       // S^T in cols [0, NH), O hi | lo in [32, 32 + 2 NH)
+constexpr float AT_TAU = 8.f;                // tolerated growth of a head's maximum (nats)
 
 struct AtSmem {
-  uint8_t kt[2][2 * AT_TILE * 128];  // key tiles (two stages), two 64-dim atoms of 128 rows
-  uint8_t vt[2][2 * AT_TILE * 128];  // value tiles, same layout as the key tiles
-  uint8_t qb[2 * AT_NH * 128];       // Q, two 64-dim atoms of 32 head rows
-  uint8_t ph[2 * AT_NH * 128];       // P hi, two 64-token atoms of 32 head rows
-  uint8_t pl[2 * AT_NH * 128];       // P lo
-  int tok[2][AT_TILE];
+  uint8_t kt[AT_STAGES][2 * AT_TILE * 128];  // key tiles: two 64-dim atoms of 128 token rows
+  uint8_t vt[AT_STAGES][2 * AT_TILE * 128];  // value tiles, same layout
+  uint8_t qb[2 * AT_NH * 128];               // Q, two 64-dim atoms of 32 head rows
+  uint8_t pb[2 * 2 * AT_NH * 128];           // P: two 64-token atoms of 2 NH rows (hi, lo)
+  int tok[AT_STAGES][AT_TILE];
   float tmax[2][4][AT_NH], tsum[2][4][AT_NH];  // per warp and head, by tile parity
-  float m[AT_NH], l[AT_NH];
-  float opart[AT_NH][SA_DV];
-  float wm[AT_NH][SA_MAX_CLUSTER], wl[AT_NH][SA_MAX_CLUSTER];  // merge weights per (head, rank)
-  uint64_t bar_s, bar_o, full[2], empty[2];
+  float m[AT_NH], l[AT_NH];                    // the CTA's reference maximum and sum
+  float wm[AT_NH][SA_MAX_CLUSTER], wl[AT_NH][SA_MAX_CLUSTER];  // merge weights
+  uint64_t bar_s, bar_o, full[AT_STAGES], empty[AT_STAGES];
   uint32_t tmem_base;
   int bad;
 };
 constexpr size_t AT_SMEM = sizeof(AtSmem) + 1024;
+static_assert(AT_SMEM <= 232448, "one CTA per SM");
+static_assert(AT_NH * SA_DV * 4 <= 2 * AT_TILE * 128, "the merge's partial outputs fit a key stage");
 
 // byte offset of element (row, kidx) of a K-major SW128 operand whose 64-element atoms
 // hold `rows` rows each
@@ -77,7 +79,19 @@ __device__ __forceinline__ uint32_t kmaj_off(int row, int kidx, int rows) {
 __device__ __forceinline__ void compute_sync() {
   asm volatile("bar.sync 1, %0;" ::"n"(AT_COMPUTE) : "memory");
 }
-
+// the same barrier, returning whether any compute thread passed v = true
+__device__ __forceinline__ bool compute_vote(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.or.pred p, 1, %2, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v), "n"(AT_COMPUTE)
+      : "memory");
+  return r != 0;
+}
 // barrier among the four loader warps only
 __device__ __forceinline__ void loader_sync() {
   asm volatile("bar.sync 2, %0;" ::"n"(AT_LOADERS) : "memory");
@@ -114,10 +128,14 @@ __device__ __forceinline__ uint16_t bf16_rn_bits(float x) {
   return (uint16_t)((u + 0x7fffu + ((u >> 16) & 1u)) >> 16);  // finite x
 }
 
-// The compute warps' side of one CTA: tiles 0 .. ntiles - 1 of stages t & 1; NH = the
-// padded head count (16 or 32), heads h >= H are masked.  Leaves the CTA's
-// unnormalised output for dimension tid in oacc and the running maximum and sum per
-// head in sm.m and sm.l.
+// The compute warps' side of one CTA over tiles 0 .. ntiles - 1 (stage t % AT_STAGES);
+// NH = the padded head count (16 or 32), heads h >= H are masked.  The probabilities
+// of a tile are taken against a reference maximum per head that every compute thread
+// holds in registers; it is raised (and the output and sum rescaled) only on a tile
+// where some score exceeds it by more than AT_TAU, which one barrier vote detects, so
+// most tiles need neither the maximum reduction nor a rescale.  Leaves the CTA's
+// unnormalised output for dimension tid in oacc and the reference maximum and the
+// sum per head in sm.m and sm.l.
 template <int NH>
 __device__ __forceinline__ void attn_compute(AtSmem &sm, uint32_t tmem, uint32_t sqb, int ntiles,
                                              int H, float scale, int *status,
@@ -125,15 +143,16 @@ __device__ __forceinline__ void attn_compute(AtSmem &sm, uint32_t tmem, uint32_t
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const float NEG = -__int_as_float(0x7f800000);
   const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-  const uint32_t sph = smem_u32(sm.ph), spl = smem_u32(sm.pl);
-  const uint32_t id = idesc_bf16_f32(AT_TILE, NH), idv = idesc_bf16_f32_amn(SA_DV, NH);
+  const uint32_t spb = smem_u32(sm.pb);
+  const uint32_t id = idesc_bf16_f32(AT_TILE, NH), idv = idesc_bf16_f32_amn(SA_DV, 2 * NH);
   const int hl = NH == 32 ? lane : lane >> 1;  // head whose warp reduction this lane holds
   const bool hl_writer = NH == 32 || (lane & 1) == 0;
 
   // S^T = K_tile . Q^T for tile t (thread 0)
   auto issue_scores = [&](int t) {
-    const int st = t & 1;
-    mbar_wait(&sm.full[st], (uint32_t)(t >> 1) & 1u, status);
+    const int st = t % AT_STAGES;
+    mbar_wait(&sm.full[st], (uint32_t)(t / AT_STAGES) & 1u, status);
+    fence_proxy_async_smem();
     tc_fence_after();
     const uint32_t skt = smem_u32(sm.kt[st]);
 #pragma unroll
@@ -145,10 +164,13 @@ __device__ __forceinline__ void attn_compute(AtSmem &sm, uint32_t tmem, uint32_t
   if (tid == 0 && ntiles > 0) issue_scores(0);
   __syncwarp();
 
+  float mref[NH];
+#pragma unroll
+  for (int h = 0; h < NH; h++) mref[h] = NEG;
+  float lsum = 0.f;  // thread h < H: the running sum of head h
   for (int t = 0; t < ntiles; t++) {
-    const int st = t & 1, par = t & 1;
-    // all compute threads see the stage filled (the tokens' liveness) and the scores
-    mbar_wait(&sm.full[st], (uint32_t)(t >> 1) & 1u, status);
+    const int st = t % AT_STAGES, par = t & 1;
+    mbar_wait(&sm.full[st], (uint32_t)(t / AT_STAGES) & 1u, status);
     const bool live = sm.tok[st][tid] >= 0;
     mbar_wait(&sm.bar_s, (uint32_t)par, status);
     tc_fence_after();
@@ -166,38 +188,46 @@ __device__ __forceinline__ void attn_compute(AtSmem &sm, uint32_t tmem, uint32_t
         for (int u = 0; u < 16; u++) sc[(16 + u) % NH] = __uint_as_float(v[u]);
       }
     }
-#pragma unroll
-    for (int h = 0; h < NH; h++) sc[h] = (live && h < H) ? sc[h] * scale : NEG;
-    {
-      float w[NH];
-#pragma unroll
-      for (int h = 0; h < NH; h++) w[h] = sc[h];
-      const float mx = xreduce<NH, true>(w, lane);
-      if (hl_writer) sm.tmax[par][warp][hl] = mx;
-    }
-    tc_fence_before();
-    compute_sync();  // (1) the tile's maxima are in; the scores in TMEM are consumed
-    if (tid == 0 && t + 1 < ntiles) issue_scores(t + 1);
-    __syncwarp();
-    // new running maximum and the rescale factor per head, probabilities of token tid
-    float mnew[NH], alpha[NH];
+    bool over = false;
 #pragma unroll
     for (int h = 0; h < NH; h++) {
-      const float mo = sm.m[h];
-      const float tm = fmaxf(fmaxf(sm.tmax[par][0][h], sm.tmax[par][1][h]),
-                             fmaxf(sm.tmax[par][2][h], sm.tmax[par][3][h]));
-      mnew[h] = fmaxf(mo, tm);
-      alpha[h] = (mnew[h] == NEG) ? 1.f : expf(mo - mnew[h]);  // mo = -inf gives 0
+      sc[h] = (live && h < H) ? sc[h] * scale : NEG;
+      over |= sc[h] > mref[h] + AT_TAU;  // a live score over a reference of -inf counts
+    }
+    tc_fence_before();
+    const bool rescale = compute_vote(over);  // (1) the scores in TMEM are consumed
+    if (tid == 0 && t + 1 < ntiles) issue_scores(t + 1);
+    __syncwarp();
+    float alpha_own = 1.f;  // thread h < H: the factor of head h's sum
+    if (rescale) {
+      {
+        float w[NH];
+#pragma unroll
+        for (int h = 0; h < NH; h++) w[h] = sc[h];
+        const float mx = xreduce<NH, true>(w, lane);
+        if (hl_writer) sm.tmax[par][warp][hl] = mx;
+      }
+      compute_sync();
+#pragma unroll
+      for (int h = 0; h < NH; h++) {
+        const float tm = fmaxf(fmaxf(sm.tmax[par][0][h], sm.tmax[par][1][h]),
+                               fmaxf(sm.tmax[par][2][h], sm.tmax[par][3][h]));
+        const float mn = fmaxf(mref[h], tm);
+        const float a = (mn == NEG) ? 1.f : __expf(mref[h] - mn);  // reference -inf gives 0
+        oacc[h] *= a;
+        if (h == tid) alpha_own = a;
+        mref[h] = mn;
+      }
     }
     {
       float w[NH];
 #pragma unroll
       for (int h = 0; h < NH; h++) {
-        const float p = (live && h < H) ? expf(sc[h] - mnew[h]) : 0.f;
+        const float p = (live && h < H) ? __expf(sc[h] - mref[h]) : 0.f;
         const uint16_t hb = bf16_rn_bits(p);
         const uint16_t lb = bf16_rn_bits(p - __uint_as_float((uint32_t)hb << 16));
-        *reinterpret_cast<uint16_t *>(sm.ph + kmaj_off(h, tid, AT_NH)) = hb;
-        *reinterpret_cast<uint16_t *>(sm.pl + kmaj_off(h, tid, AT_NH)) = lb;
+        *reinterpret_cast<uint16_t *>(sm.pb + kmaj_off(h, tid, 2 * NH)) = hb;
+        *reinterpret_cast<uint16_t *>(sm.pb + kmaj_off(NH + h, tid, 2 * NH)) = lb;
         w[h] = p;
       }
       const float ps = xreduce<NH, false>(w, lane);
@@ -206,52 +236,45 @@ __device__ __forceinline__ void attn_compute(AtSmem &sm, uint32_t tmem, uint32_t
     fence_proxy_async_smem();
     tc_fence_before();
     compute_sync();  // (2) P and the tile's sums are in; the previous fold is done
-    if (tid < H) {
-      const float mo = sm.m[tid];
-      const float tm = fmaxf(fmaxf(sm.tmax[par][0][tid], sm.tmax[par][1][tid]),
-                             fmaxf(sm.tmax[par][2][tid], sm.tmax[par][3][tid]));
-      const float mn = fmaxf(mo, tm);
-      const float al = (mn == NEG) ? 1.f : expf(mo - mn);
-      sm.l[tid] = sm.l[tid] * al + (sm.tsum[par][0][tid] + sm.tsum[par][1][tid]) +
-                  (sm.tsum[par][2][tid] + sm.tsum[par][3][tid]);
-      sm.m[tid] = mn;
-    }
-    // O^T tile = V^T . (P_hi + P_lo)^T, V^T read MN-major from the value rows: dims
-    // 0-63 and 64-127 are 16 KB apart, 8-token groups 1 KB apart, 16 tokens per MMA.
-    // The stage is free once these have run.
+    // [O_hi | O_lo]^T = V^T . [P_hi ; P_lo]^T, V^T read MN-major from the value rows:
+    // dims 0-63 and 64-127 are 16 KB apart, 8-token groups 1 KB apart, 16 tokens per
+    // MMA.  The stage is free once these have run.
     if (tid == 0) {
       tc_fence_after();
       const uint32_t svt = smem_u32(sm.vt[st]);
 #pragma unroll
       for (int kk = 0; kk < 8; kk++)
         umma_bf16(tmem + 32, sdesc_mn_sw128(svt + kk * 2048, AT_TILE * 128, 1024),
-                  sdesc_k_sw128(sph + (kk >> 2) * AT_NH * 128 + (kk & 3) * 32), idv, kk > 0);
-#pragma unroll
-      for (int kk = 0; kk < 8; kk++)
-        umma_bf16(tmem + 32, sdesc_mn_sw128(svt + kk * 2048, AT_TILE * 128, 1024),
-                  sdesc_k_sw128(spl + (kk >> 2) * AT_NH * 128 + (kk & 3) * 32), idv, 1u);
+                  sdesc_k_sw128(spb + (kk >> 2) * 2 * NH * 128 + (kk & 3) * 32), idv, kk > 0);
       umma_commit(&sm.bar_o);
-      if (t + 2 < ntiles) umma_commit(&sm.empty[st]);
+      if (t + AT_STAGES < ntiles) umma_commit(&sm.empty[st]);
     }
     __syncwarp();
+    if (tid < H)
+      lsum = lsum * alpha_own + (sm.tsum[par][0][tid] + sm.tsum[par][1][tid]) +
+             (sm.tsum[par][2][tid] + sm.tsum[par][3][tid]);
     mbar_wait(&sm.bar_o, (uint32_t)par, status);
     tc_fence_after();
     // fold the tile into dimension tid's accumulators
-    {
-      uint32_t v[16];
-      tmem_ld16(tmem + lane_base + 32, v);
+#pragma unroll
+    for (int g = 0; g < NH / 16; g++) {
+      uint32_t hi[16], lo[16];
+      tmem_ld16(tmem + lane_base + 32 + 16 * g, hi);
+      tmem_ld16(tmem + lane_base + 32 + NH + 16 * g, lo);
       tmem_wait_ld();
 #pragma unroll
-      for (int u = 0; u < 16; u++) oacc[u] = fmaf(oacc[u], alpha[u], __uint_as_float(v[u]));
-      if (NH == 32) {
-        tmem_ld16(tmem + lane_base + 48, v);
-        tmem_wait_ld();
-#pragma unroll
-        for (int u = 0; u < 16; u++)
-          oacc[16 + u] = fmaf(oacc[16 + u], alpha[(16 + u) % NH], __uint_as_float(v[u]));
-      }
+      for (int u = 0; u < 16; u++)
+        oacc[16 * g + u] += __uint_as_float(hi[u]) + __uint_as_float(lo[u]);
     }
     tc_fence_before();
+  }
+  if (tid < H) {
+    float mo = NEG;
+#pragma unroll
+    for (int h = 0; h < NH; h++)
+      if (h == tid) mo = mref[h];
+    sm.m[tid] = mo;
+    sm.l[tid] = lsum;
   }
 }
 
@@ -277,7 +300,7 @@ sparse_attn_tc_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict
   if (tid == 0) {
     mbar_init(&sm.bar_s, 1);
     mbar_init(&sm.bar_o, 1);
-    for (int i = 0; i < 2; i++) {
+    for (int i = 0; i < AT_STAGES; i++) {
       mbar_init(&sm.full[i], AT_LOADERS);
       mbar_init(&sm.empty[i], 1);
     }
@@ -288,20 +311,18 @@ sparse_attn_tc_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict
     tmem_alloc(&sm.tmem_base, AT_TMEM_COLS);
     tmem_relinquish();
   }
-  // Q (zero rows for padded heads) and zeroed P rows for padded heads
+  // Q, zero rows for padded heads
   for (int x = tid; x < AT_NH * 16; x += AT_THREADS) {
     const int h = x >> 4, c = x & 15;
     uint4 w = make_uint4(0u, 0u, 0u, 0u);
     if (h < H) w = __ldg(reinterpret_cast<const uint4 *>(q + ((size_t)row * H + h) * SA_DV) + c);
     *reinterpret_cast<uint4 *>(sm.qb + (c >> 3) * AT_NH * 128 + sw128_offset(h, c & 7)) = w;
-    const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-    *reinterpret_cast<uint4 *>(sm.ph + (c >> 3) * AT_NH * 128 + sw128_offset(h, c & 7)) = z;
-    *reinterpret_cast<uint4 *>(sm.pl + (c >> 3) * AT_NH * 128 + sw128_offset(h, c & 7)) = z;
   }
   if (tid < AT_NH) {
     sm.m[tid] = NEG;
     sm.l[tid] = 0.f;
   }
+  fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -314,13 +335,15 @@ sparse_attn_tc_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict
   for (int h = 0; h < AT_NH; h++) oacc[h] = 0.f;
 
   if (tid >= AT_COMPUTE) {
-    // ---- loaders: fill stage t & 1 with the tile's token ids and its key and value
-    // rows; both tiles keep the row layout of the cache (token rows, dims contiguous),
-    // swizzled in 128-byte rows. Rows of no token are zeros.
+    // ---- loaders: fill stage t % AT_STAGES with the tile's token ids and its key and
+    // value rows; both tiles keep the row layout of the cache (token rows, dims
+    // contiguous), swizzled in 128-byte rows; rows of no token are zeros.  A thread
+    // keeps two tiles' copies in flight and signals a tile once its copies are done.
     const int lt = tid - AT_COMPUTE;
     for (int t = 0; t < ntiles; t++) {
-      const int st = t & 1, base = e0 + t * AT_TILE;
-      if (t >= 2) mbar_wait(&sm.empty[st], (uint32_t)((t >> 1) - 1) & 1u, status);
+      const int st = t % AT_STAGES, base = e0 + t * AT_TILE;
+      if (t >= AT_STAGES)
+        mbar_wait(&sm.empty[st], (uint32_t)(t / AT_STAGES - 1) & 1u, status);
       {  // token of tile position lt (-1 = none; outside the region = none, reported)
         const int j = base + lt < e1 ? __ldg(irow + base + lt) : -1;
         if (j >= kcap) sm.bad = 1;
@@ -344,9 +367,16 @@ sparse_attn_tc_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict
         }
       }
       cp_async_commit();
+      if (t > 0) {
+        cp_async_wait_group1();
+        fence_proxy_async_smem();
+        mbar_arrive(&sm.full[(t - 1) % AT_STAGES]);
+      }
+    }
+    if (ntiles > 0) {
       cp_async_wait_all();
       fence_proxy_async_smem();
-      mbar_arrive(&sm.full[st]);
+      mbar_arrive(&sm.full[(ntiles - 1) % AT_STAGES]);
     }
   } else if (Hp == 16) {
     attn_compute<16>(sm, tmem, sqb, ntiles, H, scale, status, oacc);
@@ -357,11 +387,13 @@ sparse_attn_tc_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict
   if (tid == 0 && sm.bad) raise_status(status, HISA_ERR_INVALID_ARG);
 
   // merge across the cluster: CTA me finishes heads me, me + C, ... Every remote read
-  // of a step is issued at once: (head, rank) pairs, then (head, dim) outputs.
+  // of a step is issued at once: (head, rank) pairs, then (head, dim) outputs.  The
+  // partial outputs go to the first key stage, free now.
+  float *opart = reinterpret_cast<float *>(sm.kt[0]);
   if (tid < AT_COMPUTE) {
 #pragma unroll
     for (int h = 0; h < AT_NH; h++)
-      if (h < H) sm.opart[h][tid] = oacc[h];
+      if (h < H) opart[h * SA_DV + tid] = oacc[h];
   }
   cl.sync();
   const int nloc = me < H ? (H - me + C - 1) / C : 0;
@@ -390,7 +422,7 @@ sparse_attn_tc_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict
     float part[SA_MAX_CLUSTER];
 #pragma unroll
     for (int c = 0; c < SA_MAX_CLUSTER; c++)
-      part[c] = c < C ? cl.map_shared_rank(&sm.opart[0][0], c)[h * SA_DV + d] : 0.f;
+      part[c] = c < C ? cl.map_shared_rank(opart, c)[h * SA_DV + d] : 0.f;
     float acc = 0.f;
 #pragma unroll
     for (int c = 0; c < SA_MAX_CLUSTER; c++)
