@@ -1,8 +1,8 @@
 """The sparse attention step (hisa_sparse_attention) against the CPU oracle, through
 the C ABI.
 
-Inputs are bf16 (exact in both); the GPU accumulates in fp32 and uses the CUDA expf,
-the oracle works in fp64.  Tolerance, from the arithmetic: a score is an fp32 dot
+Inputs are bf16 (exact in both); the GPU accumulates in fp32 and uses the fast CUDA
+exponential (__expf, a few ulp), the oracle works in fp64.  Tolerance, from the arithmetic: a score is an fp32 dot
 product of 128 terms (relative error ~1e-5 of |q||k|, with scale 1/sqrt(128) at most
 ~1e-4 absolute), which moves a softmax weight by that much relative; the output is a
 convex combination of value rows of magnitude <= ~5, accumulated over <= 2048 terms in
@@ -128,4 +128,41 @@ def test_attention_out_of_region_index_is_reported():
     fixed = idx.copy()
     fixed[0, 2] = -1  # the reported entry is ignored
     ref_out, ref_lse = oracle.sparse_attention(q, k, v, fixed, cu_q, cu_k, 2, 0.1)
+    _check(out, lse, ref_out, ref_lse)
+
+
+@pytest.mark.parametrize("order", ["rising", "falling", "shuffled"])
+@pytest.mark.parametrize("heads", [8, 20])
+@pytest.mark.parametrize("nq", [1, 150])
+def test_attention_score_ramp(order, heads, nq):
+    """Scores that climb by about 12 nats per tile of 128 tokens (about 200 over the
+    row): visited in rising order every tile raises the running maximum (the rescale
+    of the output and the sum on each tile), falling order keeps the first maximum
+    and lets later probabilities underflow, shuffled order mixes both.  One query
+    per sequence runs on clusters, 150 per sequence on one CTA per query."""
+    rng = np.random.Generator(np.random.PCG64(heads * 7 + nq + len(order)))
+    S, L, topk = 2, 2048, 2048
+    u = rng.standard_normal(ATT_D)
+    u /= np.linalg.norm(u)
+    slope = 200.0 / (L * 15.0 / math.sqrt(ATT_D))  # score ~ 200 * j / L at a head factor of 15
+    k = np.concatenate([np.outer(np.arange(L) * slope, u) for _ in range(S)])
+    k = bf16_from_f32((k + 0.05 * rng.standard_normal(k.shape)).astype(np.float32))
+    v = bf16_from_f32(rng.standard_normal((S * L, ATT_D), dtype=np.float32))
+    total_q = S * nq
+    a = rng.uniform(10.0, 20.0, (total_q, heads))
+    q = bf16_from_f32((a[..., None] * u).astype(np.float32))
+    base = np.arange(L, dtype=np.int32)
+    if order == "falling":
+        base = base[::-1].copy()
+    idx = np.empty((total_q, topk), np.int32)
+    for r in range(total_q):
+        idx[r] = rng.permutation(base) if order == "shuffled" else base
+    cu_k = np.array([0, L, 2 * L], np.int32)
+    cu_q = np.array([0, nq, 2 * nq], np.int32)
+    scale = 1.0 / math.sqrt(ATT_D)
+    H().hisa_device_status(clear=True)
+    out, lse = _run(q, k, v, idx, cu_q, cu_k, heads, scale)
+    assert H().hisa_device_status() == 0
+    ref_out, ref_lse = oracle.sparse_attention(q, k, v, idx, cu_q, cu_k, heads, scale)
+    assert float(ref_lse.max()) > 150.0  # the ramp is as steep as intended
     _check(out, lse, ref_out, ref_lse)
