@@ -15,6 +15,7 @@
 // and the C partial results are merged through distributed shared memory: CTA c
 // finishes the heads h with h % C == c.
 #include <cooperative_groups.h>
+#include <cuda_bf16.h>
 
 #include "prof.cuh"
 #include "tc.cuh"
@@ -48,21 +49,23 @@ constexpr int AT_THREADS = AT_COMPUTE + AT_LOADERS;
 constexpr int AT_TILE = 128;                 // tokens per tile
 constexpr int AT_STAGES = 3;                 // tiles in the loaders' ring
 constexpr int AT_NH = 32;                    // head rows of the Q operand
-constexpr uint32_t AT_TMEM_COLS = 128;       // S^T in cols [0, NH), O hi | lo in [32, 32 + 2 NH)
+constexpr uint32_t AT_TMEM_COLS = 128;       // S^T of even / odd tiles at cols 0 / 32, O at 64
+constexpr int AT_PLO = 32;                   // P row: hi of head h at element h, lo at 32 + h
 constexpr float AT_TAU = 8.f;                // tolerated growth of a head's maximum (nats)
 
 struct AtSmem {
   uint8_t kt[AT_STAGES][2 * AT_TILE * 128];  // key tiles: two 64-dim atoms of 128 token rows
   uint8_t vt[AT_STAGES][2 * AT_TILE * 128];  // value tiles, same layout
   uint8_t qb[2 * AT_NH * 128];               // Q, two 64-dim atoms of 32 head rows
-  uint8_t pb[2 * 2 * AT_NH * 128];           // P: two 64-token atoms of 2 NH rows (hi, lo)
+  uint8_t pb[AT_TILE * 128];                 // P, MN-major: one 128-byte row per token
   int tok[AT_STAGES][AT_TILE];
   float tmax[2][4][AT_NH], tsum[2][4][AT_NH];  // per warp and head, by tile parity
   float m[AT_NH], l[AT_NH];                    // the CTA's reference maximum and sum
   float wm[AT_NH][SA_MAX_CLUSTER], wl[AT_NH][SA_MAX_CLUSTER];  // merge weights
-  uint64_t bar_s, bar_o, full[AT_STAGES], empty[AT_STAGES];
+  uint64_t bar_s[2], bar_o, full[AT_STAGES], empty[AT_STAGES];  // bar_s per S buffer
   uint32_t tmem_base;
   int bad;
+  int abort;  // set by the first wait that times out; the CTA's later waits give up
 };
 constexpr size_t AT_SMEM = sizeof(AtSmem) + 1024;
 static_assert(AT_SMEM <= 232448, "one CTA per SM");
@@ -129,7 +132,12 @@ __device__ __forceinline__ uint16_t bf16_rn_bits(float x) {
 }
 
 // The compute warps' side of one CTA over tiles 0 .. ntiles - 1 (stage t % AT_STAGES);
-// NH = the padded head count (16 or 32), heads h >= H are masked.  The probabilities
+// NH = the padded head count (16 or 32), heads h >= H are masked.  The scores of tile
+// t land in TMEM columns 32 (t & 1), so thread 0 issues the next tile's score product
+// as soon as its stage is filled, and it runs under the current tile's softmax.  P is
+// the MN-major B operand of the second product: thread t writes token t's 128-byte
+// row (hi of head h at element h, lo at 32 + h, zeros elsewhere), and the product's
+// N = 64 output columns are O hi | O lo.  The probabilities
 // of a tile are taken against a reference maximum per head that every compute thread
 // holds in registers; it is raised (and the output and sum rescaled) only on a tile
 // where some score exceeds it by more than AT_TAU, which one barrier vote detects, so
@@ -144,24 +152,37 @@ __device__ __forceinline__ void attn_compute(AtSmem &sm, uint32_t tmem, uint32_t
   const float NEG = -__int_as_float(0x7f800000);
   const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
   const uint32_t spb = smem_u32(sm.pb);
-  const uint32_t id = idesc_bf16_f32(AT_TILE, NH), idv = idesc_bf16_f32_amn(SA_DV, 2 * NH);
+  const uint32_t id = idesc_bf16_f32(AT_TILE, NH);
+  const uint32_t idv = idesc_bf16_f32_amn(SA_DV, 2 * AT_PLO) | (1u << 16);  // A and B MN-major
   const int hl = NH == 32 ? lane : lane >> 1;  // head whose warp reduction this lane holds
   const bool hl_writer = NH == 32 || (lane & 1) == 0;
 
-  // S^T = K_tile . Q^T for tile t (thread 0)
-  auto issue_scores = [&](int t) {
+  // S^T = K_tile . Q^T for tile t (thread 0), once its stage is filled; with
+  // `block` false it only tries.  Returns whether it issued.
+  auto issue_scores = [&](int t, bool block) -> bool {
     const int st = t % AT_STAGES;
-    mbar_wait(&sm.full[st], (uint32_t)(t / AT_STAGES) & 1u, status);
+    const uint32_t par = (uint32_t)(t / AT_STAGES) & 1u;
+    if (block) {
+      mbar_wait(&sm.full[st], par, status, &sm.abort);
+    } else if (!mbar_try_wait(&sm.full[st], par)) {
+      return false;
+    }
     fence_proxy_async_smem();
     tc_fence_after();
     const uint32_t skt = smem_u32(sm.kt[st]);
 #pragma unroll
     for (int kk = 0; kk < 8; kk++)
-      umma_bf16(tmem, sdesc_k_sw128(skt + (kk >> 2) * AT_TILE * 128 + (kk & 3) * 32),
+      umma_bf16(tmem + 32u * (uint32_t)(t & 1),
+                sdesc_k_sw128(skt + (kk >> 2) * AT_TILE * 128 + (kk & 3) * 32),
                 sdesc_k_sw128(sqb + (kk >> 2) * AT_NH * 128 + (kk & 3) * 32), id, kk > 0);
-    umma_commit(&sm.bar_s);
+    umma_commit(&sm.bar_s[t & 1]);
+    return true;
   };
-  if (tid == 0 && ntiles > 0) issue_scores(0);
+  int issued = 0;  // thread 0: score products issued so far
+  if (tid == 0 && ntiles > 0) {
+    issue_scores(0, true);
+    issued = 1;
+  }
   __syncwarp();
 
   float mref[NH];
@@ -170,19 +191,22 @@ __device__ __forceinline__ void attn_compute(AtSmem &sm, uint32_t tmem, uint32_t
   float lsum = 0.f;  // thread h < H: the running sum of head h
   for (int t = 0; t < ntiles; t++) {
     const int st = t % AT_STAGES, par = t & 1;
-    mbar_wait(&sm.full[st], (uint32_t)(t / AT_STAGES) & 1u, status);
+    if (tid == 0 && issued == t + 1 && t + 1 < ntiles && issue_scores(t + 1, false)) issued++;
+    __syncwarp();
+    mbar_wait(&sm.full[st], (uint32_t)(t / AT_STAGES) & 1u, status, &sm.abort);
     const bool live = sm.tok[st][tid] >= 0;
-    mbar_wait(&sm.bar_s, (uint32_t)par, status);
+    mbar_wait(&sm.bar_s[par], (uint32_t)(t >> 1) & 1u, status, &sm.abort);
     tc_fence_after();
+    const uint32_t scol = tmem + lane_base + 32u * (uint32_t)par;
     float sc[NH];
     {
       uint32_t v[16];
-      tmem_ld16(tmem + lane_base, v);
+      tmem_ld16(scol, v);
       tmem_wait_ld();
 #pragma unroll
       for (int u = 0; u < 16; u++) sc[u] = __uint_as_float(v[u]);
       if (NH == 32) {
-        tmem_ld16(tmem + lane_base + 16, v);
+        tmem_ld16(scol + 16, v);
         tmem_wait_ld();
 #pragma unroll
         for (int u = 0; u < 16; u++) sc[(16 + u) % NH] = __uint_as_float(v[u]);
@@ -195,8 +219,8 @@ __device__ __forceinline__ void attn_compute(AtSmem &sm, uint32_t tmem, uint32_t
       over |= sc[h] > mref[h] + AT_TAU;  // a live score over a reference of -inf counts
     }
     tc_fence_before();
-    const bool rescale = compute_vote(over);  // (1) the scores in TMEM are consumed
-    if (tid == 0 && t + 1 < ntiles) issue_scores(t + 1);
+    const bool rescale = compute_vote(over);  // (1) the tile's scores are read
+    if (tid == 0 && issued == t + 1 && t + 1 < ntiles && issue_scores(t + 1, true)) issued++;
     __syncwarp();
     float alpha_own = 1.f;  // thread h < H: the factor of head h's sum
     if (rescale) {
@@ -221,14 +245,26 @@ __device__ __forceinline__ void attn_compute(AtSmem &sm, uint32_t tmem, uint32_t
     }
     {
       float w[NH];
+      uint32_t hi2[NH / 2], lo2[NH / 2];
 #pragma unroll
-      for (int h = 0; h < NH; h++) {
-        const float p = (live && h < H) ? __expf(sc[h] - mref[h]) : 0.f;
-        const uint16_t hb = bf16_rn_bits(p);
-        const uint16_t lb = bf16_rn_bits(p - __uint_as_float((uint32_t)hb << 16));
-        *reinterpret_cast<uint16_t *>(sm.pb + kmaj_off(h, tid, 2 * NH)) = hb;
-        *reinterpret_cast<uint16_t *>(sm.pb + kmaj_off(NH + h, tid, 2 * NH)) = lb;
-        w[h] = p;
+      for (int h = 0; h < NH; h += 2) {
+        const float p0 = (live && h < H) ? __expf(sc[h] - mref[h]) : 0.f;
+        const float p1 = (live && h + 1 < H) ? __expf(sc[h + 1] - mref[h + 1]) : 0.f;
+        const __nv_bfloat162 hb = __floats2bfloat162_rn(p0, p1);
+        const __nv_bfloat162 lb = __floats2bfloat162_rn(p0 - __low2float(hb), p1 - __high2float(hb));
+        hi2[h >> 1] = *reinterpret_cast<const uint32_t *>(&hb);
+        lo2[h >> 1] = *reinterpret_cast<const uint32_t *>(&lb);
+        w[h] = p0;
+        w[h + 1] = p1;
+      }
+      // token tid's row: 16-byte chunk c (8 heads) at its swizzled place
+      uint8_t *prow = sm.pb + (tid >> 3) * 1024 + (tid & 7) * 128;
+#pragma unroll
+      for (int c = 0; c < NH / 8; c++) {
+        *reinterpret_cast<uint4 *>(prow + ((c ^ (tid & 7)) << 4)) =
+            make_uint4(hi2[4 * c], hi2[4 * c + 1], hi2[4 * c + 2], hi2[4 * c + 3]);
+        *reinterpret_cast<uint4 *>(prow + (((AT_PLO / 8 + c) ^ (tid & 7)) << 4)) =
+            make_uint4(lo2[4 * c], lo2[4 * c + 1], lo2[4 * c + 2], lo2[4 * c + 3]);
       }
       const float ps = xreduce<NH, false>(w, lane);
       if (hl_writer) sm.tsum[par][warp][hl] = ps;
@@ -236,16 +272,16 @@ __device__ __forceinline__ void attn_compute(AtSmem &sm, uint32_t tmem, uint32_t
     fence_proxy_async_smem();
     tc_fence_before();
     compute_sync();  // (2) P and the tile's sums are in; the previous fold is done
-    // [O_hi | O_lo]^T = V^T . [P_hi ; P_lo]^T, V^T read MN-major from the value rows:
-    // dims 0-63 and 64-127 are 16 KB apart, 8-token groups 1 KB apart, 16 tokens per
-    // MMA.  The stage is free once these have run.
+    // [O_hi | O_lo]^T = V^T . [P_hi | P_lo]^T, both operands read MN-major from token
+    // rows: V's dims 0-63 and 64-127 are 16 KB apart, 8-token groups 1 KB apart in both,
+    // 16 tokens per MMA.  The stage is free once these have run.
     if (tid == 0) {
       tc_fence_after();
       const uint32_t svt = smem_u32(sm.vt[st]);
 #pragma unroll
       for (int kk = 0; kk < 8; kk++)
-        umma_bf16(tmem + 32, sdesc_mn_sw128(svt + kk * 2048, AT_TILE * 128, 1024),
-                  sdesc_k_sw128(spb + (kk >> 2) * 2 * NH * 128 + (kk & 3) * 32), idv, kk > 0);
+        umma_bf16(tmem + 64, sdesc_mn_sw128(svt + kk * 2048, AT_TILE * 128, 1024),
+                  sdesc_mn_sw128(spb + kk * 2048, 1024, 1024), idv, kk > 0);
       umma_commit(&sm.bar_o);
       if (t + AT_STAGES < ntiles) umma_commit(&sm.empty[st]);
     }
@@ -253,14 +289,14 @@ __device__ __forceinline__ void attn_compute(AtSmem &sm, uint32_t tmem, uint32_t
     if (tid < H)
       lsum = lsum * alpha_own + (sm.tsum[par][0][tid] + sm.tsum[par][1][tid]) +
              (sm.tsum[par][2][tid] + sm.tsum[par][3][tid]);
-    mbar_wait(&sm.bar_o, (uint32_t)par, status);
+    mbar_wait(&sm.bar_o, (uint32_t)par, status, &sm.abort);
     tc_fence_after();
     // fold the tile into dimension tid's accumulators
 #pragma unroll
     for (int g = 0; g < NH / 16; g++) {
       uint32_t hi[16], lo[16];
-      tmem_ld16(tmem + lane_base + 32 + 16 * g, hi);
-      tmem_ld16(tmem + lane_base + 32 + NH + 16 * g, lo);
+      tmem_ld16(tmem + lane_base + 64 + 16 * g, hi);
+      tmem_ld16(tmem + lane_base + 64 + AT_PLO + 16 * g, lo);
       tmem_wait_ld();
 #pragma unroll
       for (int u = 0; u < 16; u++)
@@ -298,7 +334,8 @@ sparse_attn_tc_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict
   const int s = find_seq(cu_q, S, row);
   const int kbase = __ldg(cu_k + s), kcap = __ldg(cu_k + s + 1) - kbase;
   if (tid == 0) {
-    mbar_init(&sm.bar_s, 1);
+    mbar_init(&sm.bar_s[0], 1);
+    mbar_init(&sm.bar_s[1], 1);
     mbar_init(&sm.bar_o, 1);
     for (int i = 0; i < AT_STAGES; i++) {
       mbar_init(&sm.full[i], AT_LOADERS);
@@ -306,6 +343,7 @@ sparse_attn_tc_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict
     }
     fence_barrier_init();
     sm.bad = 0;
+    sm.abort = 0;
   }
   if (warp == 0) {
     tmem_alloc(&sm.tmem_base, AT_TMEM_COLS);
@@ -318,6 +356,8 @@ sparse_attn_tc_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict
     if (h < H) w = __ldg(reinterpret_cast<const uint4 *>(q + ((size_t)row * H + h) * SA_DV) + c);
     *reinterpret_cast<uint4 *>(sm.qb + (c >> 3) * AT_NH * 128 + sw128_offset(h, c & 7)) = w;
   }
+  for (int x = tid; x < AT_TILE * 8; x += AT_THREADS)
+    reinterpret_cast<uint4 *>(sm.pb)[x] = make_uint4(0u, 0u, 0u, 0u);
   if (tid < AT_NH) {
     sm.m[tid] = NEG;
     sm.l[tid] = 0.f;
@@ -343,7 +383,7 @@ sparse_attn_tc_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict
     for (int t = 0; t < ntiles; t++) {
       const int st = t % AT_STAGES, base = e0 + t * AT_TILE;
       if (t >= AT_STAGES)
-        mbar_wait(&sm.empty[st], (uint32_t)(t / AT_STAGES - 1) & 1u, status);
+        mbar_wait(&sm.empty[st], (uint32_t)(t / AT_STAGES - 1) & 1u, status, &sm.abort);
       {  // token of tile position lt (-1 = none; outside the region = none, reported)
         const int j = base + lt < e1 ? __ldg(irow + base + lt) : -1;
         if (j >= kcap) sm.bad = 1;

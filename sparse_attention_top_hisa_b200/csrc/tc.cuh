@@ -16,9 +16,10 @@
 
 namespace hisa {
 
-// Spin limit of every bounded wait (about a second or more); a wait that runs out
-// raises HISA_ERR_TIMEOUT and lets the kernel run to its end.
+// Limits of every bounded wait (about a second, and a cap on the tries); a wait that
+// runs out raises HISA_ERR_TIMEOUT and lets the kernel run to its end.
 constexpr long long kWaitLimit = 1ll << 26;
+constexpr uint64_t kWaitNs = 1000000000ull;  // one second
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return (uint32_t)__cvta_generic_to_shared(p);
@@ -62,11 +63,30 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Wait for the phase with the given parity to complete; false (and the status bit)
-// if the spin limit ran out.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int *status) {
-  for (long long i = 0; i < kWaitLimit; i++)
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Wait for the phase with the given parity to complete.  Gives up (false, and the
+// timeout bit in the status word) after about kWaitNs nanoseconds or kWaitLimit
+// tries; with `abort` (a shared flag of the CTA) it also gives up at once when the
+// flag is set, and sets it on a timeout, so that one stuck wait ends the CTA's later
+// waits quickly instead of each running to its own limit.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int *status,
+                                          volatile int *abort = nullptr) {
+  uint64_t t0 = 0;
+  for (long long i = 0; i < kWaitLimit; i++) {
     if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 63) == 63) {
+      if (abort && *abort) return false;
+      const uint64_t now = global_ns();
+      if (t0 == 0) t0 = now;
+      else if (now - t0 > kWaitNs) break;
+    }
+  }
+  if (abort) *abort = 1;
   raise_status(status, HISA_ERR_TIMEOUT);
   return false;
 }
