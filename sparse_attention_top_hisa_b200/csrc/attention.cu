@@ -30,18 +30,20 @@ static_assert(SA_DV == 128, "the merge and the tile layouts take 128-dim rows");
 
 // ---------------------------------------------------------------------------
 // Tensor-core version.  Per tile of 128 selected tokens:
-//   S^T [128 tokens x Hp] = K_tile [128 x 128] . Q^T [128 x Hp]     (tcgen05, TMEM cols 0..)
-//   O^T [128 dims x Hp]   = V^T [128 x 128 tokens] . P^T [128 x Hp] (TMEM cols 32..)
+//   S^T [128 tokens x Hp]  = K_tile [128 x 128] . Q^T [128 x Hp]        (TMEM cols 0 / 32)
+//   O^T [128 dims x 64]    = V^T [128 x 128 tokens] . [P_hi | P_lo]^T  (TMEM cols 64..127)
 // with Hp = the head count rounded up to 16.  The key and value tiles are gathered
 // with cp.async in the cache's own row layout (token rows, 128-byte swizzle): K is
 // the K-major A operand of the first product and V the MN-major A operand of the
-// second.  Q and the probabilities P are K-major B operands; P is split into bf16
-// hi + lo (two MMAs) so that it keeps about 16 bits.  Four loader warps fill a
-// two-stage ring; thread t of the four compute warps is token t for the scores
-// (online softmax per head, running maximum and sum in shared memory) and dimension
-// t for the output tile, which it folds into fp32 registers rescaled by the tile's
-// factor.  The next tile's score product is issued as soon as the current scores
-// have been read, so it runs under the softmax.
+// second.  Q is a K-major B operand; the probabilities are split into bf16 hi + lo
+// (about 16 bits) and stored MN-major, one 128-byte row per token holding the hi
+// values at elements 0.. and the lo values at 32.., so one product of N = 64 gives
+// O_hi and O_lo side by side.  Four loader warps fill a three-stage ring; thread t
+// of the four compute warps is token t for the scores and dimension t for the output
+// tile, which it folds into fp32 registers.  Each tcgen05 MMA of these shapes retires
+// about 85 cycles after the previous one whatever its N, so the kernel keeps the MMA
+// count low (eight per product) and overlaps the chains with the softmax rather
+// than splitting them.
 
 constexpr int AT_COMPUTE = 128;              // warps 0-3: MMAs, softmax, output fold
 constexpr int AT_LOADERS = 128;              // warps 4-7: token ids, key and value tiles
