@@ -385,7 +385,7 @@ def run_ours(args, world, rank):
                                          for n, v in kt.items() if v["launches"]},
                              "roofline_per_kernel": per_kernel}}
     if rank == 0 and not args.no_extras:
-        details.update(extras(args, w, q, k, cu_q, cu_k, sl, out, flush, stream, hbm_peak))
+        details.update(extras(args, w, q, k, cu_q, cu_k, sl, out, flush, stream, hbm_peak, tc_peak))
 
     clocks = sampler.stop() if sampler else None
     line = {
@@ -425,7 +425,7 @@ def time_events(fn, reps, flush, stream):
     return out
 
 
-def extras(args, w4, q4, k4, cu_q4, cu_k4, sl4, out4, flush, stream, hbm_peak):
+def extras(args, w4, q4, k4, cu_q4, cu_k4, sl4, out4, flush, stream, hbm_peak, tc_peak):
     """Flat DSA at 128K, the 32K needle prefill, decode, IoU."""
     import torch
     import sparse_attention_top_hisa_b200 as H
@@ -509,7 +509,7 @@ def extras(args, w4, q4, k4, cu_q4, cu_k4, sl4, out4, flush, stream, hbm_peak):
         del ov, wsv
     det["prefill_32k"]["variants"] = variants
     det["dsa_128k"]["hisa_speedup_over_dsa"] = None  # filled by the caller
-    det["attention"] = attention_bench(w3, o3, flush, stream, hbm_peak)
+    det["attention"] = attention_bench(w3, o3, flush, stream, hbm_peak, tc_peak)
     del q3, k3, o3, d3, ws3, dws3
     torch.cuda.empty_cache()
     det["decode"] = decode_bench(flush, stream, hbm_peak)
@@ -619,7 +619,7 @@ def decode_bench(flush, stream, hbm_peak, n_states=4, steps=256):
             "states": n_states, "kernel_us_per_step_eager": breakdown}
 
 
-def attention_bench(w3, o3, flush, stream, hbm_peak, heads=16):
+def attention_bench(w3, o3, flush, stream, hbm_peak, tc_peak, heads=16):
     """The sparse attention step over the selected tokens (synthetic q/k/v of width
     128, N(0,1) bf16, 16 heads sharing one key and one value row per token): decode
     (16 queries, the indices HISA selects on the decode workload) and the 32K needle
@@ -668,7 +668,8 @@ def attention_bench(w3, o3, flush, stream, hbm_peak, heads=16):
     res["prefill_32k"] = {"heads": heads, "k": w3.topk, "ms": round(ms, 3),
                           "queries_per_s": round(nq / (ms / 1e3), 1),
                           "TFLOPs": round(flop / (ms / 1e3) / 1e12, 2),
-                          "frac_of_fp32_alu_peak": round(flop / (ms / 1e3) / 1e12 / ALU_PEAK_TFLOPS, 4)}
+                          "flop": "2*2*heads*128 per valid selected token (q.k and p.v)",
+                          "frac_of_bf16_tensor_peak": round(flop / (ms / 1e3) / 1e12 / tc_peak, 4)}
     del ka, va, qa, out
     torch.cuda.empty_cache()
     return res
