@@ -147,7 +147,12 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # helpers
 
+PG_TIMEOUT_S = 120  # ranks that wait for one another end with an error, not a hang
+
+
 def dist_setup(args):
+    """One process per GPU (torchrun's RANK / LOCAL_RANK / WORLD_SIZE): NCCL on the
+    GPUs; gloo on CPU, where only the host-side plumbing runs (tests)."""
     import torch
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -155,29 +160,45 @@ def dist_setup(args):
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=PG_TIMEOUT_S))
     elif torch.cuda.is_available():
         torch.cuda.set_device(0)
     return world, rank, local
 
 
+def _reduce_device():
+    import torch.distributed as dist
+    return "cuda" if dist.get_backend() == "nccl" else "cpu"
+
+
 def barrier(world):
+    """Every rank reaches this point, then the device is idle on this rank."""
     import torch
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
-    torch.cuda.synchronize()
+    if torch.cuda.is_available():
+        torch.cuda.synchronize()
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """The largest of the ranks' values (every multi-GPU time is the slowest rank's)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=_reduce_device())
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(world: int, units_per_rank: int, ms: float) -> float:
+    """Whole-job throughput under weak scaling: every rank processes units_per_rank in
+    the max-over-ranks time ms."""
+    return world * units_per_rank / (ms / 1e3)
 
 
 def to_dev_bf16(a):
@@ -313,7 +334,7 @@ def run_ours(args, world, rank):
     step_ms = [a.elapsed_time(b) for a, b in ev]
     ms = max_over_ranks(sum(step_ms) / len(step_ms), world)
     launches = int(sum(v["launches"] for v in kt.values()))
-    value = world * nq / (ms / 1e3)
+    value = job_throughput(world, nq, ms)
 
     # ---- end to end: host buffers through the public API --------------------------
     hq = torch.from_numpy(np.ascontiguousarray(w.q).view(np.int16)).view(torch.bfloat16).pin_memory()
@@ -397,7 +418,7 @@ def run_ours(args, world, rank):
                    "d": 64, "B": B, "m": m, "k": K, "inputs": "bf16 q/k, PCG64 seed 20264",
                    "l2": "256 MiB flush before every timed step (outside the step events)",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
-        "e2e": {"value": round(world * nq / (e2e / 1e3), 1), "unit": UNIT,
+        "e2e": {"value": round(job_throughput(world, nq, e2e), 1), "unit": UNIT,
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                 "ms_per_step": round(e2e, 3)},
         "gpu_launches": launches,
