@@ -493,19 +493,22 @@ cudaError_t launch_sparse_attention(const uint16_t *q, const uint16_t *k, const 
   attrs[0].val.clusterDim.z = 1;
   cfg.attrs = attrs;
   cfg.numAttrs = 1;
-  // Split the rows over clusters of C CTAs while the grid is small, but only as far
-  // as every cluster of the launch can be resident at once (a second wave of
-  // clusters would cost more than the split saves).
+  // Split the rows over clusters of C CTAs while the grid is small: among the C whose
+  // clusters are all resident at once (a second wave of clusters costs more than the
+  // split saves), take the one with the fewest tiles per CTA, the smaller on a tie.
   static int fits[64][SA_MAX_CLUSTER + 1];  // clusters resident at once, per device
   int dev = 0;
   cudaGetDevice(&dev);
-  int C = 1;
-  while (C < SA_MAX_CLUSTER && total_q * C < 2 * num_sms) {
-    const int c2 = 2 * C;
-    int &n = fits[dev & 63][c2];
+  const int tiles = (topk + AT_TILE - 1) / AT_TILE;
+  int C = 1, best = tiles;
+  for (int c = 2; c <= SA_MAX_CLUSTER; c++) {
+    if (total_q * c > 2 * num_sms) break;  // enough CTAs without splitting this far
+    const int cost = (tiles + c - 1) / c;
+    if (cost >= best) continue;
+    int &n = fits[dev & 63][c];
     if (n == 0) {
-      cfg.gridDim = dim3(c2);
-      attrs[0].val.clusterDim.x = c2;
+      cfg.gridDim = dim3(c);
+      attrs[0].val.clusterDim.x = c;
       if (cudaOccupancyMaxActiveClusters(&n, sparse_attn_tc_kernel, &cfg) != cudaSuccess) {
         (void)cudaGetLastError();  // the query's own error; the launch below decides
         n = -1;
@@ -513,11 +516,11 @@ cudaError_t launch_sparse_attention(const uint16_t *q, const uint16_t *k, const 
         n = -1;
       }
     }
-    if (n < total_q) break;
-    C = c2;
+    if (n < total_q) continue;
+    C = c;
+    best = cost;
   }
-  int per = (topk + C - 1) / C;
-  per = (per + AT_TILE - 1) / AT_TILE * AT_TILE;
+  const int per = best * AT_TILE;
   cfg.gridDim = dim3(total_q * C);
   attrs[0].val.clusterDim.x = C;
   ProfScope ps(K_SPARSE_ATTENTION, st);
