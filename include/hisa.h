@@ -218,6 +218,13 @@ size_t dsa_flat_workspace_size(int total_q, int num_seqs, int max_seqlen_k, int 
  *   lse (out)    fp32 [total_q, num_heads] or NULL.
  * 1 <= num_heads <= HISA_ATT_MAX_HEADS.  No workspace; q_att, k_att and v_att must be
  * 16-byte aligned.
+ * Precision: the dot products are exact bf16 products summed in fp32 (tensor cores);
+ * the softmax weights use the fast exponential and enter the value product as bf16
+ * hi + lo (about 16 significant bits); sums and the output accumulate in fp32.
+ * Errors: a null pointer, num_heads outside [1, HISA_ATT_MAX_HEADS] or k < 1 returns
+ * HISA_ERR_INVALID_ARG and a misaligned pointer HISA_ERR_UNALIGNED, before any
+ * launch; a launch failure returns HISA_ERR_CUDA; a device-side wait that times out (it should not) raises
+ * HISA_ERR_TIMEOUT in the device status word and the call still completes.
  */
 #define HISA_ATT_DIM 128
 #define HISA_ATT_MAX_HEADS 32
