@@ -16,8 +16,8 @@ import pytest
 import torch
 
 import oracle
-from parity import dev_bf16, dev_i32
-from synth import bf16_from_f32, decode_workload, gaussian_prefill
+from parity import OnDevice, dev_bf16, dev_i32, sample_rows
+from synth import bf16_from_f32, config_workload, decode_workload, gaussian_prefill
 
 pytestmark = pytest.mark.gpu
 
@@ -165,4 +165,50 @@ def test_attention_score_ramp(order, heads, nq):
     assert H().hisa_device_status() == 0
     ref_out, ref_lse = oracle.sparse_attention(q, k, v, idx, cu_q, cu_k, heads, scale)
     assert float(ref_lse.max()) > 150.0  # the ramp is as steep as intended
+    _check(out, lse, ref_out, ref_lse)
+
+
+def test_attention_prefill_32k_full_size_sampled():
+    """The 32K needle prefill at the size the bench times: 32768 queries x 2048 selected
+    tokens (the indices hisa_select chose), 16 heads, one CTA per query; sampled rows
+    (seeded, plus sequence and block edges) against the oracle."""
+    h = H()
+    w = config_workload(3)
+    dw = OnDevice(w)
+    reps = h.hisa_pool_blocks(dw.k, dw.cu_k, dw.seqlens, dw.max_seqlen_k)
+    idx = h.hisa_select(dw.q, dw.k, reps, dw.cu_q, dw.cu_k, dw.seqlens, dw.max_seqlen_k, w.m,
+                        w.topk).cpu().numpy()
+    del dw, reps
+    heads = 16
+    q, k, v = _att_inputs(w.k.shape[0], w.total_q, heads, 11)
+    scale = 1.0 / math.sqrt(ATT_D)
+    h.hisa_device_status(clear=True)
+    out, lse = _run(q, k, v, idx, w.cu_q, w.cu_k, heads, scale)
+    assert h.hisa_device_status() == 0
+    rows = sample_rows(w, 40, 12)
+    ref_out, ref_lse = oracle.sparse_attention(q[rows], k, v, idx[rows],
+                                               np.array([0, len(rows)], np.int32), w.cu_k,
+                                               heads, scale)
+    _check(out[rows], lse[rows], ref_out, ref_lse)
+    assert np.all(np.isfinite(out)) and np.all(np.isfinite(lse))
+
+
+def test_attention_decode_full_size():
+    """The decode batch at the size the bench times: 16 sequences x 32768 keys, k = 2048,
+    16 heads (the split over a cluster per query); every row against the oracle."""
+    h = H()
+    d = config_workload(2, steps=1)
+    S, cap = d.num_seqs, d.capacity
+    kc, cu_k, lens = dev_bf16(d.k_cache), dev_i32(d.cu_k), dev_i32(d.seqlens0)
+    reps = h.hisa_pool_blocks(kc, cu_k, lens, cap)
+    idx = h.hisa_select(dev_bf16(d.queries[0]), kc, reps, dev_i32(np.arange(S + 1)), cu_k, lens,
+                        cap, d.m, d.topk).cpu().numpy()
+    heads = 16
+    q, k, v = _att_inputs(d.k_cache.shape[0], S, heads, 13)
+    cu_q = np.arange(S + 1, dtype=np.int32)
+    scale = 1.0 / math.sqrt(ATT_D)
+    h.hisa_device_status(clear=True)
+    out, lse = _run(q, k, v, idx, cu_q, d.cu_k, heads, scale)
+    assert h.hisa_device_status() == 0
+    ref_out, ref_lse = oracle.sparse_attention(q, k, v, idx, cu_q, d.cu_k, heads, scale)
     _check(out, lse, ref_out, ref_lse)
