@@ -151,18 +151,32 @@ inv_scan_kernel(const int *__restrict__ cnt, int nb, int *__restrict__ cursor,
   int total_c, total_t;
   int oc = block_exclusive_scan<SCAN_THREADS>(sc, warp_tot, &total_c);
   int ot = block_exclusive_scan<SCAN_THREADS>(st, warp_tot, &total_t);
-  for (int i = b0; i < b1; i++) {
-    const int c = cnt[i];
-    cursor[i] = oc;
-    for (int t = 0; t * TC_N < c; t++) {
-      TileDesc d;
-      d.list_off = oc + t * TC_N;
-      d.cb = i;
-      d.n = min(TC_N, c - t * TC_N);
-      d.pad = 0;
-      tiles[ot++] = d;
+  // Tile descriptors: the warp writes its lanes' blocks one after another, 32
+  // descriptors per store instruction (one block can own hundreds of tiles: block 0
+  // is selected by every query).
+  const int lane = threadIdx.x & 31;
+  for (int j = 0; j < per; j++) {
+    const int i = b0 + j;
+    const int c = i < b1 ? cnt[i] : 0;
+    if (i < b1) cursor[i] = oc;
+    const int nt = (c + TC_N - 1) / TC_N;
+    for (int src = 0; src < 32; src++) {
+      const int si = __shfl_sync(0xffffffffu, i, src);
+      const int sc_ = __shfl_sync(0xffffffffu, c, src);
+      const int soc = __shfl_sync(0xffffffffu, oc, src);
+      const int sot = __shfl_sync(0xffffffffu, ot, src);
+      const int snt = __shfl_sync(0xffffffffu, nt, src);
+      for (int t = lane; t < snt; t += 32) {
+        TileDesc d;
+        d.list_off = soc + t * TC_N;
+        d.cb = si;
+        d.n = min(TC_N, sc_ - t * TC_N);
+        d.pad = 0;
+        tiles[sot + t] = d;
+      }
     }
     oc += c;
+    ot += nt;
   }
   if (threadIdx.x == 0) *ntiles = total_t;
 }
