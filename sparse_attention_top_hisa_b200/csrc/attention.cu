@@ -73,13 +73,6 @@ constexpr size_t AT_SMEM = sizeof(AtSmem) + 1024;
 static_assert(AT_SMEM <= 232448, "one CTA per SM");
 static_assert(AT_NH * SA_DV * 4 <= 2 * AT_TILE * 128, "the merge's partial outputs fit a key stage");
 
-// byte offset of element (row, kidx) of a K-major SW128 operand whose 64-element atoms
-// hold `rows` rows each
-__device__ __forceinline__ uint32_t kmaj_off(int row, int kidx, int rows) {
-  return (uint32_t)((kidx >> 6) * rows * 128) + sw128_offset(row, (kidx & 63) >> 3) +
-         (uint32_t)((kidx & 7) * 2);
-}
-
 // barrier among the four compute warps only (the loaders never take id 1)
 __device__ __forceinline__ void compute_sync() {
   asm volatile("bar.sync 1, %0;" ::"n"(AT_COMPUTE) : "memory");
@@ -128,14 +121,9 @@ __device__ __forceinline__ float xreduce(float (&v)[NH], int lane) {
   return v[0];
 }
 
-__device__ __forceinline__ uint16_t bf16_rn_bits(float x) {
-  const uint32_t u = __float_as_uint(x);
-  return (uint16_t)((u + 0x7fffu + ((u >> 16) & 1u)) >> 16);  // finite x
-}
-
 // The compute warps' side of one CTA over tiles 0 .. ntiles - 1 (stage t % AT_STAGES);
 // NH = the padded head count (16 or 32), heads h >= H are masked.  The scores of tile
-// t land in TMEM columns 32 (t & 1), so thread 0 issues the next tile's score product
+// t land in TMEM columns from 32 * (t & 1), so thread 0 issues the next tile's score product
 // as soon as its stage is filled, and it runs under the current tile's softmax.  P is
 // the MN-major B operand of the second product: thread t writes token t's 128-byte
 // row (hi of head h at element h, lo at 32 + h, zeros elsewhere), and the product's
