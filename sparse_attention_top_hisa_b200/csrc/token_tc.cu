@@ -73,6 +73,8 @@ constexpr size_t TC_SMEM_BYTES = sizeof(TcSmem) + 1024;
 constexpr int INV_THREADS = 256;
 constexpr int INV_ROWS = 256;
 constexpr int INV_LOCAL_BINS = 8192;
+constexpr int INV_RB = 8;                      // rows whose block ids a warp loads at once
+constexpr int INV_SLOTS = (HISA_MAX_M + 31) / 32;  // slots per lane (m <= HISA_MAX_M)
 
 __global__ void __launch_bounds__(INV_THREADS)
 inv_lists_kernel(const int32_t *__restrict__ blk, int total_q, int m,
@@ -93,14 +95,30 @@ inv_lists_kernel(const int32_t *__restrict__ blk, int total_q, int m,
   const int base = s0 * emax;
   const int nbl = (s1 - s0 + 1) * emax;
   const bool local = nbl <= INV_LOCAL_BINS;
-  // walk the pairs: warp w takes rows r0 + w, r0 + w + NW, ...; lane = slot
+  // walk the pairs: warp w takes rows r0 + w, r0 + w + NW, ...; lane = slot.  The
+  // block ids of INV_RB rows are loaded before any is used, so that a warp keeps that
+  // many loads in flight instead of one.
   auto walk = [&](auto &&fn) {
     int s = s0;
-    for (int row = r0 + warp; row < r1; row += NW) {
-      while (s < s1 && __ldg(cu_q + s + 1) <= row) s++;
-      for (int slot = lane; slot < m; slot += 32) {
-        const int b = __ldg(blk + (size_t)row * m + slot);
-        if (b >= 0) fn(row, slot, s * emax + b);
+    for (int rb = r0 + warp; rb < r1; rb += NW * INV_RB) {
+      int b[INV_RB][INV_SLOTS];
+#pragma unroll
+      for (int u = 0; u < INV_RB; u++) {
+        const int row = rb + u * NW;
+#pragma unroll
+        for (int c = 0; c < INV_SLOTS; c++) {
+          const int slot = lane + 32 * c;
+          b[u][c] = (row < r1 && slot < m) ? __ldg(blk + (size_t)row * m + slot) : -1;
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < INV_RB; u++) {
+        const int row = rb + u * NW;
+        if (row >= r1) break;
+        while (s < s1 && __ldg(cu_q + s + 1) <= row) s++;
+#pragma unroll
+        for (int c = 0; c < INV_SLOTS; c++)
+          if (b[u][c] >= 0) fn(row, lane + 32 * c, s * emax + b[u][c]);
       }
     }
   };
