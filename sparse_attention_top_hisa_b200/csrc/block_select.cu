@@ -98,10 +98,19 @@ block_select_kernel(const int32_t *__restrict__ cu_q, const int32_t *__restrict_
 #pragma unroll
   for (int i = 0; i < 8; i++) hist[lane * 8 + i] = 0u;
   __syncwarp();
-  for (int b = lane; b < E; b += 32) {
-    const uint32_t u = __ldg(src + b);
-    keys[b] = u;
-    if (u != 0u) atomicAdd(&hist[u >> 24], 1u);
+  // eight keys per lane are loaded before any is used (the key matrix streams from
+  // HBM at long contexts, so one load in flight per lane would leave the warp waiting)
+  for (int b0 = lane; b0 < E; b0 += 32 * 8) {
+    uint32_t u[8];
+#pragma unroll
+    for (int j = 0; j < 8; j++) u[j] = b0 + 32 * j < E ? __ldg(src + b0 + 32 * j) : 0u;
+#pragma unroll
+    for (int j = 0; j < 8; j++) {
+      if (b0 + 32 * j < E) {
+        keys[b0 + 32 * j] = u[j];
+        if (u[j] != 0u) atomicAdd(&hist[u[j] >> 24], 1u);
+      }
+    }
   }
   __syncwarp();
   warp_select_blocks(keys, E, own, m, dst, dst2, hist, true);
