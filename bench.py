@@ -12,7 +12,9 @@ The same run measures, and reports under "details": the flat DSA scan on the
 same input (the HISA/DSA speedup), the 32768-token needle prefill (speedup,
 IoU and needle recall), and decode (16 sequences x 32768 keys, one append and
 one selection per step, 256 steps in a CUDA graph over four independent
-decode states so that the key caches cannot stay in L2).
+decode states so that the key caches cannot stay in L2), and the sparse
+attention step (16 heads x 128, bf16 K/V rows) over the decode batch's and the
+32K prefill's selections.
 
 Under torchrun (N > 1) every rank runs the same workload on its own GPU (weak
 scaling, no collective on the data path); times are the maximum over ranks.
