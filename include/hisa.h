@@ -41,6 +41,10 @@
  *     from a caller workspace sized by the matching *_workspace_size function.
  *   - Calls are asynchronous on the caller's stream (a cudaStream_t passed as
  *     void*; NULL = the legacy default stream) and never synchronise the host.
+ *   - Entry points may be called from several host threads at once: a call keeps
+ *     its state in its arguments and the library's per-device lookups are atomic.
+ *     The exceptions are noted where they apply (hisa_select_noalloc shares one
+ *     scratch array; the timing functions are not thread-safe).
  *   - Every call returns a hisa_status; nothing throws across the ABI.
  *     Argument errors visible on the host are returned directly and nothing is
  *     launched.  Errors that only the device can see (a region start that is

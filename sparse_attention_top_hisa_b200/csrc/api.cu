@@ -103,8 +103,10 @@ static __device__ int g_hisa_status;
 namespace {
 
 constexpr int kMaxDevices = 64;
-int *g_status_ptr[kMaxDevices];
-int g_num_sms[kMaxDevices];
+// Per-device values looked up once; atomic so that host threads calling the library at
+// the same time do not race (both may look the value up, harmlessly).
+std::atomic<int *> g_status_ptr[kMaxDevices];
+std::atomic<int> g_num_sms[kMaxDevices];
 
 int current_device() {
   int dev = 0;
@@ -116,24 +118,26 @@ int current_device() {
 int *status_word() {
   const int dev = current_device();
   if (dev < 0) return nullptr;
-  if (!g_status_ptr[dev]) {
+  int *sp = g_status_ptr[dev].load(std::memory_order_relaxed);
+  if (!sp) {
     void *p = nullptr;
     if (cudaGetSymbolAddress(&p, g_hisa_status) != cudaSuccess) return nullptr;
-    g_status_ptr[dev] = static_cast<int *>(p);
+    sp = static_cast<int *>(p);
+    g_status_ptr[dev].store(sp, std::memory_order_relaxed);
   }
-  return g_status_ptr[dev];
+  return sp;
 }
 
 int num_sms() {
   const int dev = current_device();
   if (dev < 0) return 148;
-  if (!g_num_sms[dev]) {
-    int n = 0;
+  int n = g_num_sms[dev].load(std::memory_order_relaxed);
+  if (!n) {
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
       n = 148;
-    g_num_sms[dev] = n;
+    g_num_sms[dev].store(n, std::memory_order_relaxed);
   }
-  return g_num_sms[dev];
+  return n;
 }
 
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
@@ -374,7 +378,7 @@ hisa_status hisa_device_status(int32_t *status, int clear, hisa_stream_t stream)
 static __device__ __align__(256) unsigned char g_noalloc_scratch[HISA_NOALLOC_SCRATCH_BYTES];
 
 namespace {
-uint8_t *g_noalloc_ptr[kMaxDevices];
+std::atomic<uint8_t *> g_noalloc_ptr[kMaxDevices];
 
 // Device address of the scratch array on the current device.  Host code only has a
 // host-side stand-in for the symbol, so the address is looked up once per device
@@ -382,12 +386,14 @@ uint8_t *g_noalloc_ptr[kMaxDevices];
 uint8_t *noalloc_scratch() {
   const int dev = current_device();
   if (dev < 0) return nullptr;
-  if (!g_noalloc_ptr[dev]) {
+  uint8_t *w = g_noalloc_ptr[dev].load(std::memory_order_relaxed);
+  if (!w) {
     void *p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return nullptr;
-    g_noalloc_ptr[dev] = static_cast<uint8_t *>(p);
+    w = static_cast<uint8_t *>(p);
+    g_noalloc_ptr[dev].store(w, std::memory_order_relaxed);
   }
-  return g_noalloc_ptr[dev];
+  return w;
 }
 }  // namespace
 

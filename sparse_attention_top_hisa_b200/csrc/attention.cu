@@ -468,7 +468,7 @@ cudaError_t launch_sparse_attention(const uint16_t *q, const uint16_t *k, const 
                                     int S, int total_q, int H, int topk, float scale, float *out,
                                     float *lse, int num_sms, int *status, cudaStream_t st) {
   if (total_q == 0) return cudaSuccess;
-  static int attr[64];
+  static std::atomic<int> attr[64];
   cudaError_t e = set_smem_once((const void *)sparse_attn_tc_kernel, AT_SMEM, attr);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -484,7 +484,7 @@ cudaError_t launch_sparse_attention(const uint16_t *q, const uint16_t *k, const 
   // Split the rows over clusters of C CTAs while the grid is small: among the C whose
   // clusters are all resident at once (a second wave of clusters costs more than the
   // split saves), take the one with the fewest tiles per CTA, the smaller on a tie.
-  static int fits[64][SA_MAX_CLUSTER + 1];  // clusters resident at once, per device
+  static std::atomic<int> fits[64][SA_MAX_CLUSTER + 1];  // clusters resident at once, per device
   int dev = 0;
   cudaGetDevice(&dev);
   const int tiles = (topk + AT_TILE - 1) / AT_TILE;
@@ -493,7 +493,7 @@ cudaError_t launch_sparse_attention(const uint16_t *q, const uint16_t *k, const 
     if (total_q * c > 2 * num_sms) break;  // enough CTAs without splitting this far
     const int cost = (tiles + c - 1) / c;
     if (cost >= best) continue;
-    int &n = fits[dev & 63][c];
+    int n = fits[dev & 63][c].load(std::memory_order_relaxed);
     if (n == 0) {
       cfg.gridDim = dim3(c);
       attrs[0].val.clusterDim.x = c;
@@ -503,6 +503,7 @@ cudaError_t launch_sparse_attention(const uint16_t *q, const uint16_t *k, const 
       } else if (n <= 0) {
         n = -1;
       }
+      fits[dev & 63][c].store(n, std::memory_order_relaxed);
     }
     if (n < total_q) continue;
     C = c;

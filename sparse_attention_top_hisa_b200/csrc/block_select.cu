@@ -176,7 +176,7 @@ cudaError_t launch_block_select(const uint16_t *q, const float *reps, const int3
   const int emax = (max_seqlen_k + BLK - 1) / BLK;
   if (tc_keys) {
     const size_t smem = (size_t)BS_WARPS * (256 + (emax > 0 ? emax : 1)) * sizeof(uint32_t);
-    static int attr[64];
+    static std::atomic<int> attr[64];
     if (smem > 48 * 1024) {
       cudaError_t e = set_smem_once((const void *)block_select_kernel, smem, attr);
       if (e != cudaSuccess) return e;
@@ -188,7 +188,7 @@ cudaError_t launch_block_select(const uint16_t *q, const float *reps, const int3
                                                          blk, out_blocks, status);
   } else {
     const size_t smem = (size_t)(256 + (emax > 0 ? emax : 1)) * sizeof(uint32_t);
-    static int attr_cta[64];
+    static std::atomic<int> attr_cta[64];
     if (smem > 48 * 1024) {
       cudaError_t e = set_smem_once((const void *)block_select_cta_kernel, smem, attr_cta);
       if (e != cudaSuccess) return e;

@@ -235,7 +235,7 @@ cudaError_t launch_block_score_tc(const uint16_t *q, const float *reps, const in
     reps_split_kernel<<<(S * emax + 3) / 4, 128, 0, st>>>(reps, cu_k, seqlens, S, emax, hi, lo);
   }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  static int attr[64];
+  static std::atomic<int> attr[64];
   if ((e = set_smem_once((const void *)block_score_tc_kernel, BS_TC_SMEM, attr)) != cudaSuccess)
     return e;
   const int tiles = (total_q + BLK - 1) / BLK + S;  // per-sequence tiles, upper bound

@@ -1,6 +1,8 @@
 // Shared device helpers for the HISA indexer kernels (sm_100a).
 #pragma once
 
+#include <atomic>
+
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -191,12 +193,14 @@ inline cudaError_t launch_pdl(const void *func, dim3 grid, dim3 block, size_t sm
 
 // Raise a kernel's dynamic shared-memory limit once per device; later calls (for
 // example while a CUDA graph is being captured) find it already set.
-inline cudaError_t set_smem_once(const void *func, size_t bytes, int *cache /*[64]*/) {
+// cache: one word per device (64), static storage; atomic so that host threads calling
+// the library at the same time do not race on it (both may set the attribute, harmlessly).
+inline cudaError_t set_smem_once(const void *func, size_t bytes, std::atomic<int> *cache) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
-  if (cache[dev] >= (int)bytes) return cudaSuccess;
+  if (cache[dev].load(std::memory_order_relaxed) >= (int)bytes) return cudaSuccess;
   cudaError_t e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
-  if (e == cudaSuccess) cache[dev] = (int)bytes;
+  if (e == cudaSuccess) cache[dev].store((int)bytes, std::memory_order_relaxed);
   return e;
 }
 

@@ -539,7 +539,7 @@ cudaError_t launch_decode_select(const uint16_t *q, const uint16_t *k, const flo
                                  int m, int topk, int32_t *out_idx, float *out_scores,
                                  int32_t *out_blocks, int *status, cudaStream_t st) {
   if (total_q == 0) return cudaSuccess;
-  static int attr[64];
+  static std::atomic<int> attr[64];
   cudaError_t e = set_smem_once((const void *)decode_select_kernel, sizeof(DcSmem), attr);
   if (e != cudaSuccess) return e;
   const int emax = (max_seqlen_k + BLK - 1) / BLK;

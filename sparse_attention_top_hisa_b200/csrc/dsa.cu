@@ -209,7 +209,7 @@ cudaError_t launch_dsa(const uint16_t *q, const uint16_t *k, const int32_t *cu_q
   }
   const size_t ssm = dsa_select_smem(topk);
   const size_t bsm = (size_t)16 * topk + sizeof(SelectShared);
-  static int attr_s[64], attr_b[64];
+  static std::atomic<int> attr_s[64], attr_b[64];
   if ((e = set_smem_once((const void *)dsa_select_kernel, ssm, attr_s)) != cudaSuccess) return e;
   if ((e = set_smem_once((const void *)dsa_fallback_kernel, bsm, attr_b)) != cudaSuccess) return e;
   for (int row0 = 0; row0 < total_q; row0 += p.chunk) {

@@ -265,7 +265,7 @@ cudaError_t launch_dsa_filter_tc(const uint16_t *q, const uint16_t *k, const int
   CUtensorMap qmap, kmap;
   if (!make_rows_tensor_map(&qmap, q, (uint64_t)total_q, BLK) || !make_key_tensor_map(&kmap, k))
     return cudaErrorInvalidValue;
-  static int attr[64];
+  static std::atomic<int> attr[64];
   cudaError_t e = set_smem_once((const void *)dsa_filter_tc_kernel, DSA_TC_SMEM, attr);
   if (e != cudaSuccess) return e;
   const int tiles = (nrows + BLK - 1) / BLK + S;  // per-sequence tiles, upper bound

@@ -200,7 +200,7 @@ cudaError_t launch_token_select(const uint16_t *q, const uint16_t *k, const int3
   const size_t smem = token_smem_bytes(m, topk);
   if (token_use_split(total_q, num_sms)) {
     // few queries: a wider CTA per query shortens each selection
-    static int attr_c[64], attr_d[64];
+    static std::atomic<int> attr_c[64], attr_d[64];
     if (m * BLK <= 1024 * 8) {
       auto kern = token_select_scratch_kernel<1024, 8>;
       if ((e = set_smem_once((const void *)kern, smem, attr_c)) != cudaSuccess) return e;
@@ -215,14 +215,14 @@ cudaError_t launch_token_select(const uint16_t *q, const uint16_t *k, const int3
                                         out_idx, out_scores);
     }
   } else if (m * BLK <= 256 * 32) {
-    static int attr_a[64];
+    static std::atomic<int> attr_a[64];
     auto kern = token_select_scratch_kernel<256, 32>;
     if ((e = set_smem_once((const void *)kern, smem, attr_a)) != cudaSuccess) return e;
     ProfScope ps(K_TOKEN_SELECT_SCRATCH, st);
     kern<<<total_q, 256, smem, st>>>(cu_q, cu_k, seqlens, S, m, topk, blk, scores, pmap,
                                      out_idx, out_scores);
   } else {
-    static int attr_b[64];
+    static std::atomic<int> attr_b[64];
     auto kern = token_select_scratch_kernel<512, 32>;
     if ((e = set_smem_once((const void *)kern, smem, attr_b)) != cudaSuccess) return e;
     ProfScope ps(K_TOKEN_SELECT_SCRATCH, st);

@@ -518,7 +518,7 @@ cudaError_t launch_token_score_tc(const uint16_t *q, const uint16_t *k, const in
                                                    pmap);
   }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  static int attr[64];
+  static std::atomic<int> attr[64];
   if ((e = set_smem_once((const void *)token_score_tc_kernel, TC_SMEM_BYTES, attr)) != cudaSuccess)
     return e;
   {
