@@ -100,3 +100,32 @@ def test_workspace_sizes_grow(lib):
     b = lib.hisa_select_workspace_size(32768, 1, 32768, 128, 64, 2048)
     assert 0 < a < b
     assert lib.dsa_flat_workspace_size(4096, 1, 4096, 256) > 0
+
+
+def test_no_cpu_fallback():
+    """The product path has no CPU route: host tensors are refused, and a missing
+    library is an error at the first call, not a silent fallback."""
+    import sys
+
+    import torch
+
+    import sparse_attention_top_hisa_b200 as H
+    k = torch.zeros(256, 64, dtype=torch.bfloat16)
+    cu = torch.tensor([0, 256], dtype=torch.int32)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        H.hisa_pool_blocks(k, cu, None, 256)
+    script = (
+        "import sys; sys.path.insert(0, %r)\n"
+        "import sparse_attention_top_hisa_b200.binding as b\n"
+        "b.LIB_PATH = '/nonexistent/libhisa.so'\n"
+        "try:\n"
+        "    b.lib()\n"
+        "except ImportError as e:\n"
+        "    print('refused:', e)\n"
+        "else:\n"
+        "    raise SystemExit('loaded a library that does not exist')\n"
+    ) % ROOT
+    p = subprocess.run([sys.executable, "-c", script], capture_output=True, text=True,
+                       timeout=120)
+    assert p.returncode == 0, p.stderr[-1500:]
+    assert "refused:" in p.stdout and "is missing" in p.stdout
