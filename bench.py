@@ -10,16 +10,21 @@ library's C ABI.  Inputs live in HBM before the timed region; L2 is flushed
 (a 256 MiB write) before every timed step, outside the step's CUDA events.
 The same run measures, and reports under "details": the flat DSA scan on the
 same input (the HISA/DSA speedup), the 32768-token needle prefill (speedup,
-IoU and needle recall), and decode (16 sequences x 32768 keys, one append and
-one selection per step, 256 steps in a CUDA graph over four independent
-decode states so that the key caches cannot stay in L2), and the sparse
-attention step (16 heads x 128, bf16 K/V rows) over the decode batch's and the
-32K prefill's selections.
+IoU, needle recall, stage 1 alone and a per-sequence block budget of half the
+blocks), the 4096-token integer prefill and the packed varlen prefill (times,
+agreement with the oracle, IoU), decode (16 sequences x 32768 keys, one
+append and one selection per step, 256 steps in a CUDA graph over four
+independent decode states so that the key caches cannot stay in L2), the
+sparse attention step (16 heads x 128, bf16 K/V rows) over the decode batch's
+and the 32K prefill's selections, and the CPU oracle timed on every
+configuration.
 
-Under torchrun (N > 1) every rank runs the same workload on its own GPU (weak
-scaling, no collective on the data path); times are the maximum over ranks.
-``--impl reference`` times the CPU oracle instead (the only other place this
-script runs the oracle) on seeded samples of the same workload.
+Under torchrun (N > 1) the ranks share the one workload: each takes a
+contiguous run of query rows balanced by estimated work, with its sequence's
+keys, and writes its own output rows -- no collective on the data path
+(strong scaling; times are the maximum over ranks).  ``--impl reference``
+times the CPU oracle instead (the only other place this script runs the
+oracle) on seeded samples of the same workload.
 """
 
 from __future__ import annotations
@@ -51,12 +56,10 @@ CONFIG_WORKLOADS = {
 }
 L2_FLUSH_BYTES = 256 << 20
 
-# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from an ncu
-# capture, keyed by kernel kind, with the sha256 of the kernel's sources at capture time
-# (a changed source voids the figure).  token_select_scratch: captured on the 32768-token
-# prefill (1.212 GB for 1.84 M selected pairs, 0.995 of its algorithmic bytes) and scaled
-# to the 131072-token launch by selected pairs (8.13 M): see
-# profiles/token_select_scratch_prefill_L32768.md.
+# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) of a kernel on
+# the 131072-token prefill, from an ncu capture of that kernel alone on the 32768-token
+# prefill scaled by the selected (query, block) pairs of the two launches, with the
+# sha256 prefix of the kernel's sources at capture time (a changed source voids it).
 TRAFFIC = {"token_select_scratch": (5241752391, "741119f642a38df2", ("token_select.cu", "select.cuh"))}
 
 
@@ -210,6 +213,32 @@ def job_throughput(world: int, units_per_rank: int, ms: float) -> float:
     return world * units_per_rank / (ms / 1e3)
 
 
+def local_workload(w, world: int, rank: int):
+    """This rank's shard of a workload: a contiguous run of query rows, cut so that the
+    ranks' estimated work is balanced, with its sequences' key regions (no exchange
+    between ranks; every rank writes its own output rows).  Returns the shard as a
+    workload of its own and its global rows [row0, row1)."""
+    if world == 1:
+        return w, 0, w.total_q
+    from synth import Workload
+    from sparse_attention_top_hisa_b200.shard import query_cost, row_bounds, shard
+    bounds = row_bounds(w.total_q, world, query_cost(w.cu_q, w.cu_k, w.seqlens, w.B, w.m))
+    sh = shard(w.cu_q, w.cu_k, w.seqlens, world, rank, w.B, bounds)
+    lw = Workload(f"{w.name}_shard{rank}of{world}", w.q[sh.row0:sh.row1], w.k[sh.key0:sh.key1],
+                  sh.cu_seqlens_q, sh.cu_seqlens_k, sh.seqlens_k, w.B, w.m, w.topk, w.d, w.exact)
+    return lw, sh.row0, sh.row1
+
+
+def sum_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=_reduce_device())
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
 def to_dev_bf16(a):
     import torch
     return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
@@ -218,10 +247,6 @@ def to_dev_bf16(a):
 def to_dev_i32(a):
     import torch
     return torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).cuda()
-
-
-ALU_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
-ALU_PEAK_SOURCE = "148 SMs x 128 FP32 lanes x 2 flop x 1965 MHz (max SM clock)"
 
 
 def query_positions(w) -> np.ndarray:
@@ -234,32 +259,65 @@ def query_positions(w) -> np.ndarray:
     return out
 
 
+def candidate_counts(w) -> np.ndarray:
+    """c_i of every query: the tokens j <= i of its selected blocks.  Every selected
+    block other than the query's own lies wholly before it; the own block (always
+    selected) contributes i % B + 1."""
+    pos = query_positions(w)
+    own = pos // w.B
+    nsel = np.minimum(w.m, own + 1)
+    return (nsel - 1) * w.B + pos % w.B + 1
+
+
 def algorithmic(w) -> dict:
-    """Algorithmic work per step of every kernel on the prefill path (bytes that must
-    move, or flops that must be done, counting nothing the method avoids)."""
+    """The method's own work per step of every kernel on the prefill path, as the
+    per-unit figures of the measurement plan fix it: bytes that must move (bound
+    "hbm") or flops that must be done (bound "tensor").  Intermediates this design
+    chooses to write and read back (block-score keys, (query, slot) lists, score rows)
+    are not counted; the ncu traffic of a kernel against these figures shows them."""
     B, m, K, d = w.B, w.m, w.topk, 64
     pos = query_positions(w)
     own = pos // B
     nsel = np.minimum(m, own + 1)
     pairs = float(nsel.sum())
-    scored_blocks = float(np.where(own + 1 > m, own + 1, 0).sum())
+    eligible = float(np.where(own + 1 > m, own + 1, 0).sum())  # blocks scored in stage 1
+    cands = float(candidate_counts(w).sum())
     live_rows = float(w.seqlens.sum())
     nblocks = float(((w.seqlens + B - 1) // B).sum())
     nq = float(w.total_q)
     return {
         "pool_blocks": {"bound": "hbm", "per_step": live_rows * 2 * d + nblocks * 4 * d,
-                        "what": "keys read once + fp32 representatives written"},
-        "block_score_tc": {"bound": "tensor", "per_step": scored_blocks * d * 2 * 2,
-                           "what": "q.rep_hi + q.rep_lo products of every eligible block (bf16 MMA)"},
-        "block_select": {"bound": "hbm", "per_step": scored_blocks * 4 + nq * m * 4,
-                         "what": "block-score keys read + selected block lists written"},
-        "inv_lists": {"bound": "hbm", "per_step": pairs * 4 * 2 + pairs * 4,
-                      "what": "block lists read twice + (query, slot) lists written"},
-        "token_score_tc": {"bound": "hbm", "per_step": pairs * B * 4 + nq * 2 * d + live_rows * 2 * d,
-                           "what": "score rows written (m*128 fp32 per query) + q, k read once"},
-        "token_select_scratch": {"bound": "hbm", "per_step": pairs * B * 4 + nq * K * 4 + nq * m * 4,
-                                 "what": "score rows read + k int32 indices written + block lists"},
+                        "what": "128 B of key read per live token + 256 B of fp32 representative "
+                                "written per block"},
+        "block_score_tc": {"bound": "tensor", "per_step": eligible * 2 * d,
+                           "what": "2*64 flop per eligible (query, block) pair of the queries that "
+                                   "see more than m blocks"},
+        "block_select": {"bound": "hbm", "per_step": nq * m * 4,
+                         "what": "4 B per selected block written (the block lists)"},
+        "inv_lists": {"bound": "hbm", "per_step": pairs * 4,
+                      "what": "4 B per selected block read (the block lists)"},
+        "token_score_tc": {"bound": "tensor", "per_step": cands * 2 * d,
+                           "what": "2*64 flop per candidate token (j <= i in a selected block)"},
+        "token_select_scratch": {"bound": "hbm", "per_step": nq * K * 4 + pairs * 4,
+                                 "what": "k int32 indices written per query + its block list read"},
+        "step": {"bound": "hbm",
+                 "per_step": nq * 2 * d + live_rows * 2 * d + nblocks * 4 * d * 2 + nq * K * 4,
+                 "what": "q and k read, representatives written and read, k int32 indices "
+                         "written per query"},
     }
+
+
+def roofline_entry(a: dict, amount: float, launch_ms: float, hbm_peak: float,
+                   tc_peak: float) -> dict:
+    """achieved = algorithmic amount per launch / launch time, against the measured peak
+    of its bound (HBM copy bandwidth, or the bf16 tensor-core GEMM rate)."""
+    if a["bound"] == "hbm":
+        ach, peak, unit = amount / (launch_ms / 1e3) / 1e9, hbm_peak, "GB/s"
+    else:
+        ach, peak, unit = amount / (launch_ms / 1e3) / 1e12, tc_peak, "TFLOP/s"
+    return {"bound": a["bound"], "achieved": round(ach, 3), "peak": peak, "unit": unit,
+            "frac": round(ach / peak, 4), "launch_ms": round(launch_ms, 4),
+            "algorithmic": a["what"], "algorithmic_per_launch": amount}
 
 
 def iou_rows(a: np.ndarray, b: np.ndarray) -> float:
@@ -299,9 +357,11 @@ def run_ours(args, world, rank):
     stream = torch.cuda.current_stream()
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
 
-    w = config_workload(args.config)
+    w_full = config_workload(args.config)
+    w, row0, row1 = local_workload(w_full, world, rank)
     B, m, K = w.B, w.m, w.topk
     nq = w.total_q
+    nq_job = w_full.total_q
     q, k = to_dev_bf16(w.q), to_dev_bf16(w.k)
     cu_q, cu_k, sl = to_dev_i32(w.cu_q), to_dev_i32(w.cu_k), to_dev_i32(w.seqlens)
     out = torch.empty(nq, K, dtype=torch.int32, device="cuda")
@@ -343,7 +403,7 @@ def run_ours(args, world, rank):
     step_ms = [a.elapsed_time(b) for a, b in ev]
     ms = max_over_ranks(sum(step_ms) / len(step_ms), world)
     launches = int(sum(v["launches"] for v in kt.values()))
-    value = job_throughput(world, nq, ms)
+    value = nq_job / (ms / 1e3)  # strong scaling: the ranks share one fixed workload
 
     # ---- end to end: host buffers through the public API --------------------------
     hq = torch.from_numpy(np.ascontiguousarray(w.q).view(np.int16)).view(torch.bfloat16).pin_memory()
@@ -370,8 +430,8 @@ def run_ours(args, world, rank):
         if i > 0:
             e2e_ms.append(a.elapsed_time(b))
     e2e = max_over_ranks(sum(e2e_ms) / len(e2e_ms), world)
-    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hcq, hck, hsl))
-    d2h = hout.numel() * hout.element_size()
+    h2d = sum_over_ranks(sum(t.numel() * t.element_size() for t in (hq, hk, hcq, hck, hsl)), world)
+    d2h = sum_over_ranks(hout.numel() * hout.element_size(), world)
 
     # ---- roofline of the dominant kernel -------------------------------------------
     alg = algorithmic(w)
@@ -383,23 +443,20 @@ def run_ours(args, world, rank):
         launch_ms = v["ms"] / v["timed"]
         launches_per_step = v["timed"] / args.steps
         amount = a["per_step"] / launches_per_step  # per launch
-        if a["bound"] == "hbm":
-            ach, peak, unit = amount / (launch_ms / 1e3) / 1e9, hbm_peak, "GB/s"
-        elif a["bound"] == "tensor":
-            ach, peak, unit = amount / (launch_ms / 1e3) / 1e12, tc_peak, "TFLOP/s"
-        else:
-            ach, peak, unit = amount / (launch_ms / 1e3) / 1e12, ALU_PEAK_TFLOPS, "TFLOP/s"
-        per_kernel[name] = {"bound": a["bound"], "achieved": round(ach, 3), "peak": peak,
-                            "unit": unit, "frac": round(ach / peak, 4),
-                            "launch_ms": round(launch_ms, 4), "algorithmic": a["what"]}
+        per_kernel[name] = roofline_entry(a, amount, launch_ms, hbm_peak, tc_peak)
+        per_kernel[name]["launches_per_step"] = launches_per_step
     dname = max((n for n in per_kernel), key=lambda n: kt[n]["ms"])
     roof = dict(per_kernel[dname])
     roof["kernel"] = dname
     t = TRAFFIC.get(dname)
-    # the stored counters are of the 128K launch: other workloads report none
-    roof["traffic"] = t[0] if t and t[1] == source_sha(t[2]) and args.config == 4 else None
-    roof["peak_source"] = (ALU_PEAK_SOURCE if roof["bound"] == "alu" else
-                           f"MEASURED_PEAKS.json ({peak_src})")
+    # stored counters hold for the 128K launch of the kernel source they were taken on
+    roof["traffic"] = (int(t[0]) if t and t[1] == source_sha(t[2]) and args.config == 4 else None)
+    if roof["traffic"] and alg[dname]["bound"] == "hbm":
+        roof["traffic_over_algorithmic"] = round(
+            roof["traffic"] / (alg[dname]["per_step"] / per_kernel[dname]["launches_per_step"]), 3)
+    roof["peak_source"] = f"MEASURED_PEAKS.json ({peak_src})"
+    step_alg = alg["step"]
+    step_roof = roofline_entry(step_alg, step_alg["per_step"], ms, hbm_peak, tc_peak)
 
     if args.dsa_steps > 0:  # profiling aid: the flat scan on the same inputs
         dout = torch.empty(nq, K, dtype=torch.int32, device="cuda")
@@ -410,11 +467,13 @@ def run_ours(args, world, rank):
         torch.cuda.synchronize()
         del dout, dws
 
-    details = {"hisa_step": {"ms": round(ms, 4), "queries_per_s": round(nq / (ms / 1e3), 1),
+    details = {"hisa_step": {"ms": round(ms, 4), "queries_per_s": round(nq_job / (ms / 1e3), 1),
+                             "rank_rows": [int(row0), int(row1)],
                              "kernels": {n: {"ms_per_step": round(v["ms"] / args.steps, 4),
                                              "launches": v["launches"]}
                                          for n, v in kt.items() if v["launches"]},
-                             "roofline_per_kernel": per_kernel}}
+                             "roofline_per_kernel": per_kernel,
+                             "roofline_step": step_roof}}
     if rank == 0 and not args.no_extras:
         details.update(extras(args, w, q, k, cu_q, cu_k, sl, out, flush, stream, hbm_peak, tc_peak))
 
@@ -422,14 +481,16 @@ def run_ours(args, world, rank):
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic",
         "config": {"workload": CONFIG_WORKLOADS[args.config], "seq_len": int(w.max_seqlen_k),
-                   "queries_per_step": nq * world,
+                   "queries_per_step": nq_job,
                    "d": 64, "B": B, "m": m, "k": K, "inputs": f"bf16 q/k, PCG64 seed {20260 + args.config}",
                    "l2": "256 MiB flush before every timed step (outside the step events)",
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
-        "e2e": {"value": round(job_throughput(world, nq, e2e), 1), "unit": UNIT,
+                   "parallelism": (f"{world} ranks, contiguous query-row shards balanced by "
+                                   "work, no collective on the data path" if world > 1
+                                   else "single GPU")},
+        "e2e": {"value": round(nq_job / (e2e / 1e3), 1), "unit": UNIT,
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                 "ms_per_step": round(e2e, 3)},
         "gpu_launches": launches,
@@ -438,7 +499,7 @@ def run_ours(args, world, rank):
         "wall_s_timed_region": round(t_wall, 3),
         "details": details,
     }
-    if rank == 0 and not args.no_cpu:
+    if rank == 0 and world == 1 and not args.no_cpu:
         line["cpu_baseline"] = cpu_baseline(w)
     return line
 
@@ -518,35 +579,99 @@ def extras(args, w4, q4, k4, cu_q4, cu_k4, sl4, out4, flush, stream, hbm_peak, t
                           "hisa_queries_per_s": round(w3.total_q / (hm3 / 1e3), 1),
                           "iou_hisa_vs_dsa_4096_rows": round(iou_rows(a3[rows3], b3[rows3]), 4),
                           "needle_recall_hisa": float(rec_h), "needle_recall_dsa": float(rec_d)}
-    # variants on the same inputs: stage 1 alone (all tokens of the best k/B blocks,
-    # i.e. no token refinement) and a fractional block budget (m = M/2)
+    # variants on the same inputs: stage 1 alone (every token of the best k/B blocks, no
+    # token refinement: hisa_block_sparse_select) and a block budget of half of the
+    # sequence's blocks (m_s = ceil(0.5 * M_s): hisa_fraction_blocks + hisa_select_varm)
     variants = {}
-    M3 = (w3.max_seqlen_k + w3.B - 1) // w3.B
-    for name, mv in (("block_sparse_only_m%d" % (w3.topk // w3.B), w3.topk // w3.B),
-                     ("hisa_half_m%d" % min(128, (M3 + 1) // 2), min(128, (M3 + 1) // 2))):
-        ov = torch.empty_like(o3)
-        wsv = torch.empty(H.hisa_select_workspace_size(w3.total_q, 1, w3.max_seqlen_k, mv, w3.topk),
-                          dtype=torch.uint8, device="cuda")
+    mb = w3.topk // w3.B
+    ob = torch.empty(w3.total_q, mb * w3.B, dtype=torch.int32, device="cuda")
+    wsb = torch.empty(H.hisa_block_sparse_workspace_size(w3.total_q, 1, w3.max_seqlen_k, mb),
+                      dtype=torch.uint8, device="cuda")
 
-        def hv():
-            H.hisa_pool_blocks(k3, ck3, sl3, w3.max_seqlen_k, reps=reps3)
-            H.hisa_select(q3, k3, reps3, cq3, ck3, sl3, w3.max_seqlen_k, mv, w3.topk, out_idx=ov,
-                          workspace=wsv)
-        hv()
-        msv = statistics.median(time_events(hv, 3, flush, stream))
-        av = ov.cpu().numpy()
-        variants[name] = {"m": mv, "ms": round(msv, 3),
-                          "iou_vs_dsa_4096_rows": round(iou_rows(av[rows3], b3[rows3]), 4),
-                          "needle_recall": float(np.mean([j in av[i] for i, j in w3.needles]))}
-        del ov, wsv
+    def hb():
+        H.hisa_pool_blocks(k3, ck3, sl3, w3.max_seqlen_k, reps=reps3)
+        H.hisa_block_sparse_select(q3, reps3, cq3, ck3, sl3, w3.max_seqlen_k, mb, out_idx=ob,
+                                   workspace=wsb)
+    hb()
+    msb = statistics.median(time_events(hb, 3, flush, stream))
+    av = ob.cpu().numpy()
+    variants[f"block_sparse_only_m{mb}"] = {
+        "entry_point": "hisa_block_sparse_select", "m": mb, "ms": round(msb, 3),
+        "iou_vs_dsa_4096_rows": round(iou_rows(av[rows3], b3[rows3]), 4),
+        "needle_recall": float(np.mean([j in av[i] for i, j in w3.needles]))}
+    del ob, wsb
+    m_max = H.HISA_MAX_M
+    ov = torch.empty_like(o3)
+    wsv = torch.empty(H.hisa_select_workspace_size(w3.total_q, 1, w3.max_seqlen_k, m_max, w3.topk),
+                      dtype=torch.uint8, device="cuda")
+    msq = torch.empty(1, dtype=torch.int32, device="cuda")
+
+    def hv():
+        H.hisa_pool_blocks(k3, ck3, sl3, w3.max_seqlen_k, reps=reps3)
+        H.hisa_fraction_blocks(ck3, sl3, 0.5, m_max, m_seq=msq)
+        H.hisa_select_varm(q3, k3, reps3, cq3, ck3, sl3, msq, w3.max_seqlen_k, m_max, w3.topk,
+                           out_idx=ov, workspace=wsv)
+    hv()
+    msv = statistics.median(time_events(hv, 3, flush, stream))
+    av = ov.cpu().numpy()
+    variants["hisa_half_blocks"] = {
+        "entry_point": "hisa_fraction_blocks(f=0.5) + hisa_select_varm", "m": int(msq.item()),
+        "ms": round(msv, 3), "iou_vs_dsa_4096_rows": round(iou_rows(av[rows3], b3[rows3]), 4),
+        "needle_recall": float(np.mean([j in av[i] for i, j in w3.needles]))}
+    del ov, wsv
     det["prefill_32k"]["variants"] = variants
     det["dsa_128k"]["hisa_speedup_over_dsa"] = None  # filled by the caller
     det["attention"] = attention_bench(w3, o3, flush, stream, hbm_peak, tc_peak)
     del q3, k3, o3, d3, ws3, dws3
     torch.cuda.empty_cache()
     det["decode"] = decode_bench(flush, stream, hbm_peak)
+    det["prefill_4096_integer"] = prefill_bench(1, flush, stream)
+    det["prefill_varlen_8seqs"] = prefill_bench(5, flush, stream)
     det["hbm_stream_ceilings"] = stream_ceilings(stream)
     return det
+
+
+def prefill_bench(cfg, flush, stream, reps=5):
+    """A prefill configuration: HISA (pool + select) and the flat scan on the same
+    inputs, their times, and HISA-vs-DSA IoU (every row, or 4096 seeded rows)."""
+    import torch
+    import sparse_attention_top_hisa_b200 as H
+    from synth import config_workload
+    w = config_workload(cfg)
+    q, k = to_dev_bf16(w.q), to_dev_bf16(w.k)
+    cq, ck, sl = to_dev_i32(w.cu_q), to_dev_i32(w.cu_k), to_dev_i32(w.seqlens)
+    reps_ = torch.zeros(w.rep_rows, 64, dtype=torch.float32, device="cuda")
+    o = torch.empty(w.total_q, w.topk, dtype=torch.int32, device="cuda")
+    d = torch.empty_like(o)
+    ws = torch.empty(H.hisa_select_workspace_size(w.total_q, w.num_seqs, w.max_seqlen_k, w.m,
+                                                  w.topk), dtype=torch.uint8, device="cuda")
+    dws = torch.empty(H.dsa_flat_workspace_size(w.total_q, w.num_seqs, w.max_seqlen_k, w.topk),
+                      dtype=torch.uint8, device="cuda")
+
+    def hisa():
+        H.hisa_pool_blocks(k, ck, sl, w.max_seqlen_k, reps=reps_)
+        H.hisa_select(q, k, reps_, cq, ck, sl, w.max_seqlen_k, w.m, w.topk, out_idx=o,
+                      workspace=ws)
+
+    def dsa():
+        H.dsa_flat_select(q, k, cq, ck, sl, w.max_seqlen_k, w.topk, out_idx=d, workspace=dws)
+    hisa()
+    dsa()
+    hm = statistics.median(time_events(hisa, reps, flush, stream))
+    dm = statistics.median(time_events(dsa, 3, flush, stream))
+    a, b = o.cpu().numpy(), d.cpu().numpy()
+    rows = (np.arange(w.total_q) if w.total_q <= 4096 else
+            np.random.Generator(np.random.PCG64(3)).choice(w.total_q, 4096, replace=False))
+    assert H.hisa_device_status() == 0
+    res = {"queries": int(w.total_q), "sequences": int(w.num_seqs),
+           "lengths": [int(x) for x in w.seqlens], "m": int(w.m), "k": int(w.topk),
+           "hisa_ms": round(hm, 4), "hisa_queries_per_s": round(w.total_q / (hm / 1e3), 1),
+           "dsa_ms": round(dm, 4), "hisa_speedup_over_dsa": round(dm / hm, 2),
+           "iou_hisa_vs_dsa": round(iou_rows(a[rows], b[rows]), 4),
+           "iou_rows": int(len(rows))}
+    del q, k, o, d, ws, dws
+    torch.cuda.empty_cache()
+    return res
 
 
 def stream_ceilings(stream, nbytes=4 << 30, reps=5):
@@ -712,23 +837,61 @@ def bf16_rows(rng, shape):
     return bf16_from_f32(rng.standard_normal(shape, dtype=np.float32))
 
 
+def _time_oracle(fn):
+    t0 = time.perf_counter()
+    fn()
+    return time.perf_counter() - t0
+
+
 def cpu_baseline(w, budget_s: float = 15.0):
-    """The oracle (unchanged) on the host cores, on a seeded sample of query rows."""
+    """The oracle (unchanged) on the host cores: a seeded sample of query rows of the
+    benchmark workload (the line's value), and the HISA and flat-DSA oracles timed on
+    every configuration (in full where that takes seconds, else on 4096 seeded rows)."""
     import oracle
+    from synth import config_workload
     n = cores()
     rng = np.random.Generator(np.random.PCG64(99))
     rows = np.sort(rng.choice(w.total_q, 512, replace=False)).astype(np.int32)
-    t0 = time.perf_counter()
-    oracle.hisa_workload(w, rows=rows, nthreads=n)
-    t1 = time.perf_counter() - t0
+    t1 = _time_oracle(lambda: oracle.hisa_workload(w, rows=rows, nthreads=n))
     target = int(min(w.total_q, max(512, 512 * budget_s / max(t1, 1e-3))))
     rows = np.sort(rng.choice(w.total_q, target, replace=False)).astype(np.int32)
-    t0 = time.perf_counter()
-    oracle.hisa_workload(w, rows=rows, nthreads=n)
-    t1 = time.perf_counter() - t0
+    t1 = _time_oracle(lambda: oracle.hisa_workload(w, rows=rows, nthreads=n))
+    per = {}
+
+    def entry(nrows, secs, full):
+        return {"rows": int(nrows), "seconds": round(secs, 3),
+                "queries_per_s": round(nrows / secs, 1), "sample": "all rows" if full else
+                "4096 seeded rows"}
+    for cfg in (1, 3, 4, 5):
+        wc = w if cfg == 4 else config_workload(cfg)
+        full = wc.total_q <= 32768
+        r = None if full else np.sort(np.random.Generator(np.random.PCG64(cfg)).choice(
+            wc.total_q, 4096, replace=False)).astype(np.int32)
+        nr = wc.total_q if full else 4096
+        per[str(cfg)] = {
+            "hisa": entry(nr, _time_oracle(lambda: oracle.hisa_workload(wc, rows=r, nthreads=n)),
+                          full),
+            "dsa": entry(nr, _time_oracle(lambda: oracle.dsa_workload(wc, rows=r, nthreads=n)),
+                         full)}
+    # decode: one step (append then select) of the 16 sequences, through the oracle's
+    # pooling of the whole caches
+    dw = config_workload(2, steps=1)
+    S = dw.num_seqs
+    kc = dw.k_cache.copy()
+    lens = dw.seqlens0.copy()
+    for s in range(S):
+        kc[int(dw.cu_k[s]) + int(lens[s])] = dw.new_keys[0, s, 0]
+    lens = lens + 1
+    cu_q = np.arange(S + 1, dtype=np.int32)
+    per["2"] = {
+        "hisa": entry(S, _time_oracle(lambda: oracle.hisa(dw.queries[0], kc, cu_q, dw.cu_k, lens,
+                                                          dw.B, dw.m, dw.topk, nthreads=n)),
+                      True),
+        "dsa": entry(S, _time_oracle(lambda: oracle.dsa(dw.queries[0], kc, cu_q, dw.cu_k, lens,
+                                                        dw.topk, nthreads=n)), True)}
     return {"value": round(target / t1, 2), "unit": UNIT, "cores": n, "kind": "oracle",
-            "sample": f"{target} seeded query rows of the 131072 (pooling over all keys each call)",
-            "seconds": round(t1, 2)}
+            "sample": f"{target} seeded query rows of the {w.total_q} (pooling over all keys each "
+                      "call)", "seconds": round(t1, 2), "per_config": per}
 
 
 # ---------------------------------------------------------------------------
@@ -755,7 +918,7 @@ def run_reference(args, world, rank):
     v = sample / (ms / 1e3)
     return {"impl": "reference", "metric": METRIC, "value": round(v, 2), "unit": UNIT,
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
+            "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "strong",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": WORKLOAD, "seq_len": 131072, "d": 64, "B": 128, "m": 64,
                        "k": 2048, "sample_rows_per_step": sample},

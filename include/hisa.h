@@ -44,7 +44,12 @@
  *   - Entry points may be called from several host threads at once: a call keeps
  *     its state in its arguments and the library's per-device lookups are atomic.
  *     The exceptions are noted where they apply (hisa_select_noalloc shares one
- *     scratch array; the timing functions are not thread-safe).
+ *     scratch array; event timing is not thread-safe, launch counting is).
+ *   - The first call of any entry point on a device looks up the addresses of the
+ *     library's device-resident words on that device (the status word and the
+ *     scratch array of hisa_select_noalloc), with that device current.  Make that
+ *     first call before any stream capture on the device; later calls may be
+ *     captured in CUDA graphs.
  *   - Every call returns a hisa_status; nothing throws across the ABI.
  *     Argument errors visible on the host are returned directly and nothing is
  *     launched.  Errors that only the device can see (a region start that is
@@ -87,7 +92,7 @@ extern "C" {
 
 #define HISA_INDEX_DIM 64
 #define HISA_BLOCK 128
-#define HISA_MAX_M 128      /* m * B candidates are held on chip per query */
+#define HISA_MAX_M 512      /* largest block budget m (m * B <= 65536 candidates per query) */
 #define HISA_MAX_TOPK 2048  /* largest k accepted by hisa_select / dsa_flat_select */
 
 typedef uint16_t hisa_bf16;  /* bf16 bit pattern */
@@ -181,6 +186,68 @@ size_t hisa_select_workspace_size(int total_q, int num_seqs, int max_seqlen_k, i
                                   int k);
 
 /*
+ * hisa_select_varm — hisa_select with a block budget per sequence.  The pages mention
+ * a fractional setting ("HISA 50%") and adaptive sparsity (idea.jsleekr.com summary
+ * and its transcript) without defining them; this library reads them as a block
+ * budget m_s per sequence, typically m_s = ceil(f * M_s) for a sequence of M_s blocks
+ * (hisa_fraction_blocks computes that on the device).
+ *
+ *   m_seq          int32 [num_seqs] (device): the budget of every sequence,
+ *                  1 <= m_seq[s] <= m_max.  A value outside that range is clamped
+ *                  and raises HISA_ERR_INVALID_ARG in the device status word.
+ *   m_max          largest budget, 1 <= m_max <= HISA_MAX_M; the row stride of
+ *                  out_blocks (entries past a row's budget are -1) and the m of the
+ *                  workspace size: hisa_select_workspace_size(..., m_max, k).
+ * Every other argument, the output and the errors are those of hisa_select; a
+ * sequence's rows equal those hisa_select gives that sequence alone with m = m_s.
+ * Budgets above 128 take a slower select that reads each score row from memory
+ * three times; the few-query cluster path takes budgets up to 128.
+ */
+hisa_status hisa_select_varm(const hisa_bf16 *q_idx, const hisa_bf16 *k_idx, const float *reps,
+                             const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
+                             const int32_t *seqlens_k, const int32_t *m_seq, int num_seqs,
+                             int total_q, int max_seqlen_k, int B, int m_max, int k,
+                             int32_t *out_idx, float *out_scores, int32_t *out_blocks, void *ws,
+                             size_t ws_bytes, hisa_stream_t stream);
+
+/*
+ * hisa_fraction_blocks — m_seq[s] = min(m_max, max(1, ceil(f * ceil(len_s / B)))) for
+ * every sequence, on the device (len_s = seqlens_k[s], or the region size when
+ * seqlens_k is NULL), for hisa_select_varm.  0 < f <= 1, 1 <= m_max <= HISA_MAX_M.
+ * A live length that does not fit its region raises HISA_ERR_INVALID_ARG in the
+ * device status word (its budget is set to 1).
+ */
+hisa_status hisa_fraction_blocks(const int32_t *cu_seqlens_k, const int32_t *seqlens_k,
+                                 int num_seqs, int B, double f, int m_max, int32_t *m_seq,
+                                 hisa_stream_t stream);
+
+/*
+ * hisa_block_sparse_select — stage 1 on its own: the block-sparse selection HISA is
+ * compared with in the Needle-in-a-Haystack paragraph of the HISA summary page.  The
+ * m blocks of every query are chosen exactly as in hisa_select (block scores, causal
+ * mask, forced blocks, top-m), and every token j <= i of them is emitted; no token is
+ * scored.  With m * B = k this is the block-sparse baseline at the same token budget.
+ *
+ *   q_idx, reps, cu_seqlens_*, seqlens_k, num_seqs, total_q, max_seqlen_k, B, m:
+ *                  as in hisa_select (no key rows are read).
+ *   out_idx (out)  int32 [total_q, m * B]: the tokens of the selected blocks in
+ *                  ascending order, -1 padded (the tail of the query's own block and
+ *                  the slots of missing blocks).
+ *   out_blocks     int32 [total_q, m] or NULL: the selected blocks, ascending.
+ *   ws, ws_bytes   device workspace of at least hisa_block_sparse_workspace_size(...)
+ *                  bytes, 256-byte aligned.
+ */
+hisa_status hisa_block_sparse_select(const hisa_bf16 *q_idx, const float *reps,
+                                     const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
+                                     const int32_t *seqlens_k, int num_seqs, int total_q,
+                                     int max_seqlen_k, int B, int m, int32_t *out_idx,
+                                     int32_t *out_blocks, void *ws, size_t ws_bytes,
+                                     hisa_stream_t stream);
+
+size_t hisa_block_sparse_workspace_size(int total_q, int num_seqs, int max_seqlen_k, int B,
+                                        int m);
+
+/*
  * dsa_flat_select — the flat DSA indexer: every causal key j <= i of the query's
  * sequence is scored with q.k and the top-k are emitted with the same ordering,
  * padding and layout as hisa_select (idea.jsleekr.com, section "DSA: 딥시크의
@@ -260,8 +327,9 @@ hisa_status hisa_device_status(int32_t *status, int clear, hisa_stream_t stream)
  *
  *   - The array exists once per device and every device that loads the library
  *     holds it until the process exits.
- *   - Batches of fewer than twice as many queries as the GPU has SMs (decode) run
- *     on a path that needs no scratch at all.  Larger batches need the scratch
+ *   - Batches of fewer than twice as many queries as the GPU has SMs (decode) whose
+ *     sequences hold at most 8192 blocks (1M tokens) and whose m is at most 128 run
+ *     on a path that needs no scratch at all.  Other batches need the scratch
  *     hisa_select_workspace_size() reports for the same arguments (about
  *     m * 516 bytes per query plus the block-score matrix), and problems whose
  *     scratch exceeds HISA_NOALLOC_SCRATCH_BYTES are rejected with
@@ -270,9 +338,8 @@ hisa_status hisa_device_status(int32_t *status, int clear, hisa_stream_t stream)
  *     in it needs to start at zero.  Calls whose kernels overlap on the GPU (on
  *     different streams, or from different host threads) race on the array and
  *     give wrong results: order them on one stream or serialise them.
- *   - The first call on a device looks up the array's device address (once per
- *     device, with that device current); make that first call before any stream
- *     capture.
+ *   - The array's device address is looked up by the first call of any entry point
+ *     on a device (see the shared conventions above).
  *   - Inputs, outputs, ordering, errors and the device status word are those of
  *     hisa_select.
  */
@@ -284,11 +351,22 @@ hisa_status hisa_select_noalloc(const hisa_bf16 *q_idx, const hisa_bf16 *k_idx, 
                                 float *out_scores, int32_t *out_blocks, hisa_stream_t stream);
 
 /*
+ * hisa_test_fault — for tests of the timeout path only (no counterpart on the pages).
+ * mode 1: the tensor-core token-scoring launches made from now on issue no loads, so
+ * that their bounded waits (about one second) run out with no copy and no MMA in
+ * flight; the launch then raises HISA_ERR_TIMEOUT in the device status word and
+ * every row of that hisa_select call is written as -1 (scores 0).  mode 0: normal
+ * operation (the default).  Process-wide, not thread-safe; returns
+ * HISA_ERR_INVALID_ARG for any other mode.
+ */
+hisa_status hisa_test_fault(int mode);
+
+/*
  * Launch accounting, for benchmarks and tests (no counterpart on the pages).
- * Every kernel launch made by this library is counted per kernel kind.  With
- * timing enabled, each launch is also bracketed by a pair of CUDA events
- * recorded on its launch stream.  Host-side state shared by all callers of the
- * process; not thread-safe; leave timing off while capturing a CUDA graph.
+ * Every kernel launch made by this library is counted per kernel kind (atomic
+ * counters).  With timing enabled, each launch is also bracketed by a pair of CUDA
+ * events recorded on its launch stream: host-side state shared by all callers of
+ * the process, not thread-safe; leave timing off while capturing a CUDA graph.
  *
  * hisa_timing_enable  — turn event timing on (1) or off (0).
  * hisa_kernel_kinds   — number of kernel kinds; hisa_kernel_name(i) names kind i.

@@ -17,11 +17,16 @@ from .binding import (  # noqa: F401
     dsa_flat_select,
     dsa_flat_workspace_size,
     hisa_append_keys,
+    hisa_block_sparse_select,
+    hisa_block_sparse_workspace_size,
     hisa_device_status,
     hisa_pool_blocks,
+    hisa_fraction_blocks,
     hisa_select,
+    hisa_select_varm,
     hisa_select_workspace_size,
     hisa_sparse_attention,
+    hisa_test_fault,
     hisa_timing_collect,
     hisa_timing_enable,
     lib,

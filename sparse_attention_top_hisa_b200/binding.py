@@ -21,7 +21,7 @@ LIB_PATH = os.path.join(_HERE, "libhisa.so")
 
 HISA_INDEX_DIM = 64
 HISA_BLOCK = 128
-HISA_MAX_M = 128
+HISA_MAX_M = 512
 HISA_MAX_TOPK = 2048
 
 STATUS = {
@@ -52,6 +52,11 @@ EXPORTED = (
     "hisa_kernel_name",
     "hisa_timing_collect",
     "hisa_select_noalloc",
+    "hisa_select_varm",
+    "hisa_fraction_blocks",
+    "hisa_block_sparse_select",
+    "hisa_block_sparse_workspace_size",
+    "hisa_test_fault",
 )
 
 
@@ -94,8 +99,16 @@ def lib() -> ctypes.CDLL:
         L.hisa_timing_collect.restype = I
         L.hisa_sparse_attention.argtypes = [P, P, P, P, P, P, I, I, I, I, ctypes.c_float, P, P,
                                             P]
+        L.hisa_select_varm.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, P, P, P, P, Z, P]
+        L.hisa_fraction_blocks.argtypes = [P, P, I, I, ctypes.c_double, I, P, P]
+        L.hisa_block_sparse_select.argtypes = [P, P, P, P, P, I, I, I, I, I, P, P, P, Z, P]
+        L.hisa_block_sparse_workspace_size.argtypes = [I, I, I, I, I]
+        L.hisa_block_sparse_workspace_size.restype = Z
+        L.hisa_test_fault.argtypes = [I]
+        L.hisa_test_fault.restype = I
         for f in ("hisa_pool_blocks", "hisa_append_keys", "hisa_select", "dsa_flat_select",
-                  "hisa_device_status", "hisa_sparse_attention"):
+                  "hisa_device_status", "hisa_sparse_attention", "hisa_select_varm",
+                  "hisa_fraction_blocks", "hisa_block_sparse_select"):
             getattr(L, f).restype = I
         _lib = L
     return _lib
@@ -211,6 +224,91 @@ def hisa_select(q_idx: torch.Tensor, k_idx: torch.Tensor, reps: torch.Tensor,
     return out_idx
 
 
+def hisa_select_varm(q_idx: torch.Tensor, k_idx: torch.Tensor, reps: torch.Tensor,
+                     cu_seqlens_q: torch.Tensor, cu_seqlens_k: torch.Tensor,
+                     seqlens_k: Optional[torch.Tensor], m_seq: torch.Tensor, max_seqlen_k: int,
+                     m_max: int, k: int, B: int = HISA_BLOCK,
+                     out_idx: Optional[torch.Tensor] = None,
+                     out_scores: Optional[torch.Tensor] = None,
+                     out_blocks: Optional[torch.Tensor] = None,
+                     workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """HISA selection with a block budget per sequence (m_seq int32 [num_seqs] on the
+    device, each in [1, m_max]); returns out_idx int32 [total_q, k]."""
+    _need(q_idx, "q_idx", torch.bfloat16, HISA_INDEX_DIM)
+    _need(k_idx, "k_idx", torch.bfloat16, HISA_INDEX_DIM)
+    _need(reps, "reps", torch.float32, HISA_INDEX_DIM)
+    _need(cu_seqlens_q, "cu_seqlens_q", torch.int32)
+    _need(cu_seqlens_k, "cu_seqlens_k", torch.int32)
+    _need(seqlens_k, "seqlens_k", torch.int32, optional=True)
+    _need(m_seq, "m_seq", torch.int32)
+    total_q, S = q_idx.shape[0], cu_seqlens_q.numel() - 1
+    if m_seq.numel() != S:
+        raise ValueError("m_seq must hold one budget per sequence")
+    if out_idx is None:
+        out_idx = torch.empty(total_q, k, dtype=torch.int32, device=q_idx.device)
+    _need(out_idx, "out_idx", torch.int32, k)
+    _need(out_scores, "out_scores", torch.float32, k, optional=True)
+    _need(out_blocks, "out_blocks", torch.int32, m_max, optional=True)
+    need = hisa_select_workspace_size(total_q, S, max_seqlen_k, m_max, k, B)
+    ws = _workspace(need, q_idx.device, workspace)
+    _check(lib().hisa_select_varm(_ptr(q_idx), _ptr(k_idx), _ptr(reps), _ptr(cu_seqlens_q),
+                                  _ptr(cu_seqlens_k), _ptr(seqlens_k), _ptr(m_seq), S, total_q,
+                                  int(max_seqlen_k), B, m_max, k, _ptr(out_idx), _ptr(out_scores),
+                                  _ptr(out_blocks), _ptr(ws), ws.numel(), _stream(stream)),
+           "hisa_select_varm")
+    return out_idx
+
+
+def hisa_fraction_blocks(cu_seqlens_k: torch.Tensor, seqlens_k: Optional[torch.Tensor], f: float,
+                         m_max: int = HISA_MAX_M, B: int = HISA_BLOCK,
+                         m_seq: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Per-sequence block budgets m_s = min(m_max, ceil(f * ceil(len_s / B))), computed on
+    the device; returns m_seq int32 [num_seqs]."""
+    _need(cu_seqlens_k, "cu_seqlens_k", torch.int32)
+    _need(seqlens_k, "seqlens_k", torch.int32, optional=True)
+    S = cu_seqlens_k.numel() - 1
+    if m_seq is None:
+        m_seq = torch.empty(S, dtype=torch.int32, device=cu_seqlens_k.device)
+    _need(m_seq, "m_seq", torch.int32)
+    _check(lib().hisa_fraction_blocks(_ptr(cu_seqlens_k), _ptr(seqlens_k), S, B, float(f), m_max,
+                                      _ptr(m_seq), _stream(stream)), "hisa_fraction_blocks")
+    return m_seq
+
+
+def hisa_block_sparse_workspace_size(total_q: int, num_seqs: int, max_seqlen_k: int, m: int,
+                                     B: int = HISA_BLOCK) -> int:
+    return int(lib().hisa_block_sparse_workspace_size(total_q, num_seqs, max_seqlen_k, B, m))
+
+
+def hisa_block_sparse_select(q_idx: torch.Tensor, reps: torch.Tensor, cu_seqlens_q: torch.Tensor,
+                             cu_seqlens_k: torch.Tensor, seqlens_k: Optional[torch.Tensor],
+                             max_seqlen_k: int, m: int, B: int = HISA_BLOCK,
+                             out_idx: Optional[torch.Tensor] = None,
+                             out_blocks: Optional[torch.Tensor] = None,
+                             workspace: Optional[torch.Tensor] = None,
+                             stream=None) -> torch.Tensor:
+    """Stage 1 alone: every causal token of the m selected blocks, ascending; returns
+    out_idx int32 [total_q, m * B]."""
+    _need(q_idx, "q_idx", torch.bfloat16, HISA_INDEX_DIM)
+    _need(reps, "reps", torch.float32, HISA_INDEX_DIM)
+    _need(cu_seqlens_q, "cu_seqlens_q", torch.int32)
+    _need(cu_seqlens_k, "cu_seqlens_k", torch.int32)
+    _need(seqlens_k, "seqlens_k", torch.int32, optional=True)
+    total_q, S = q_idx.shape[0], cu_seqlens_q.numel() - 1
+    if out_idx is None:
+        out_idx = torch.empty(total_q, m * B, dtype=torch.int32, device=q_idx.device)
+    _need(out_idx, "out_idx", torch.int32, m * B)
+    _need(out_blocks, "out_blocks", torch.int32, m, optional=True)
+    need = hisa_block_sparse_workspace_size(total_q, S, max_seqlen_k, m, B)
+    ws = _workspace(need, q_idx.device, workspace)
+    _check(lib().hisa_block_sparse_select(_ptr(q_idx), _ptr(reps), _ptr(cu_seqlens_q),
+                                          _ptr(cu_seqlens_k), _ptr(seqlens_k), S, total_q,
+                                          int(max_seqlen_k), B, m, _ptr(out_idx),
+                                          _ptr(out_blocks), _ptr(ws), ws.numel(),
+                                          _stream(stream)), "hisa_block_sparse_select")
+    return out_idx
+
+
 def dsa_flat_select(q_idx: torch.Tensor, k_idx: torch.Tensor, cu_seqlens_q: torch.Tensor,
                     cu_seqlens_k: torch.Tensor, seqlens_k: Optional[torch.Tensor],
                     max_seqlen_k: int, k: int, out_idx: Optional[torch.Tensor] = None,
@@ -242,6 +340,12 @@ def hisa_device_status(clear: bool = True, stream=None) -> int:
     _check(lib().hisa_device_status(ctypes.byref(v), 1 if clear else 0, _stream(stream)),
            "hisa_device_status")
     return int(v.value)
+
+
+def hisa_test_fault(mode: int) -> None:
+    """Tests of the timeout path only: mode 1 makes the tensor-core token-scoring launches
+    issue no loads (their bounded waits run out); 0 restores normal operation."""
+    _check(lib().hisa_test_fault(int(mode)), "hisa_test_fault")
 
 
 def hisa_timing_enable(on: bool) -> None:

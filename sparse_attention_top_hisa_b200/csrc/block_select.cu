@@ -39,37 +39,45 @@ __device__ __forceinline__ float rep_score(const QRegs &q, const float *rep) {
 }
 
 // Common front part of both kernels: locate the query, handle invalid rows and the
-// take-all case.  Returns false when the row is finished.
+// take-all case.  m is the row's block budget, m_max the row stride of dst (entries
+// m..m_max-1 are -1).  Returns false when the row is finished.
 __device__ __forceinline__ bool block_row_setup(const int32_t *cu_q, const int32_t *cu_k,
-                                                const int32_t *seqlens, int S, int row, int m,
-                                                int emax, int32_t *dst, int32_t *dst2,
-                                                int *status, QueryInfo &qi, int &own, int &E,
-                                                int lane_id, int nthreads) {
+                                                const int32_t *seqlens, const int32_t *m_seq,
+                                                int S, int row, int m_max, int emax, int32_t *dst,
+                                                int32_t *dst2, int *status, QueryInfo &qi,
+                                                int &own, int &E, int &m, int lane_id,
+                                                int nthreads) {
   qi = locate(cu_q, cu_k, seqlens, S, row, lane_id == 0 ? status : nullptr);
+  m = m_max;
   if (!qi.ok) {
-    for (int i = lane_id; i < m; i += nthreads) {
+    for (int i = lane_id; i < m_max; i += nthreads) {
       dst[i] = -1;
       if (dst2) dst2[i] = -1;
     }
     return false;
   }
+  m = seq_budget(m_seq, qi.seq, m_max, lane_id == 0 ? status : nullptr);
   own = qi.pos / BLK;
   E = own + 1;
   if (E > emax) {  // max_seqlen_k understated by the caller
     if (lane_id == 0) raise_status(status, HISA_ERR_INVALID_ARG);
-    for (int i = lane_id; i < m; i += nthreads) {
+    for (int i = lane_id; i < m_max; i += nthreads) {
       dst[i] = -1;
       if (dst2) dst2[i] = -1;
     }
     return false;
   }
   if (E <= m) {  // every eligible block is kept
-    for (int i = lane_id; i < m; i += nthreads) {
+    for (int i = lane_id; i < m_max; i += nthreads) {
       const int v = i < E ? i : -1;
       dst[i] = v;
       if (dst2) dst2[i] = v;
     }
     return false;
+  }
+  for (int i = m + lane_id; i < m_max; i += nthreads) {  // past this row's budget
+    dst[i] = -1;
+    if (dst2) dst2[i] = -1;
   }
   return true;
 }
@@ -77,7 +85,8 @@ __device__ __forceinline__ bool block_row_setup(const int32_t *cu_q, const int32
 // Many queries: one warp per query reads the keys computed on the tensor cores.
 __global__ void __launch_bounds__(BS_WARPS * 32)
 block_select_kernel(const int32_t *__restrict__ cu_q, const int32_t *__restrict__ cu_k,
-                    const int32_t *__restrict__ seqlens, int S, int total_q, int m, int emax,
+                    const int32_t *__restrict__ seqlens, const int32_t *__restrict__ m_seq,
+                    int S, int total_q, int m_max, int emax,
                     const uint32_t *__restrict__ tc_keys, int tc_stride,
                     int32_t *__restrict__ blk, int32_t *__restrict__ out_blocks,
                     int *status) {
@@ -87,12 +96,12 @@ block_select_kernel(const int32_t *__restrict__ cu_q, const int32_t *__restrict_
   if (row >= total_q) return;
   uint32_t *hist = bs_smem + (size_t)warp * 256;
   uint32_t *keys = bs_smem + BS_WARPS * 256 + (size_t)warp * emax;
-  int32_t *dst = blk + (size_t)row * m;
-  int32_t *dst2 = out_blocks ? out_blocks + (size_t)row * m : nullptr;
+  int32_t *dst = blk + (size_t)row * m_max;
+  int32_t *dst2 = out_blocks ? out_blocks + (size_t)row * m_max : nullptr;
   QueryInfo qi;
-  int own, E;
-  if (!block_row_setup(cu_q, cu_k, seqlens, S, row, m, emax, dst, dst2, status, qi, own, E, lane,
-                       32))
+  int own, E, m;
+  if (!block_row_setup(cu_q, cu_k, seqlens, m_seq, S, row, m_max, emax, dst, dst2, status, qi, own,
+                       E, m, lane, 32))
     return;
   const uint32_t *src = tc_keys + (size_t)row * tc_stride;
 #pragma unroll
@@ -124,17 +133,17 @@ constexpr int BS_CTA_THREADS = 256;
 __global__ void __launch_bounds__(BS_CTA_THREADS)
 block_select_cta_kernel(const uint16_t *__restrict__ q, const float *__restrict__ reps,
                         const int32_t *__restrict__ cu_q, const int32_t *__restrict__ cu_k,
-                        const int32_t *__restrict__ seqlens, int S, int m, int emax,
-                        int32_t *__restrict__ blk, int32_t *__restrict__ out_blocks,
-                        int *status) {
+                        const int32_t *__restrict__ seqlens, const int32_t *__restrict__ m_seq,
+                        int S, int m_max, int emax, int32_t *__restrict__ blk,
+                        int32_t *__restrict__ out_blocks, int *status) {
   extern __shared__ uint32_t bsc_smem[];
   const int row = blockIdx.x, tid = threadIdx.x;
-  int32_t *dst = blk + (size_t)row * m;
-  int32_t *dst2 = out_blocks ? out_blocks + (size_t)row * m : nullptr;
+  int32_t *dst = blk + (size_t)row * m_max;
+  int32_t *dst2 = out_blocks ? out_blocks + (size_t)row * m_max : nullptr;
   QueryInfo qi;
-  int own, E;
-  if (!block_row_setup(cu_q, cu_k, seqlens, S, row, m, emax, dst, dst2, status, qi, own, E, tid,
-                       BS_CTA_THREADS))
+  int own, E, m;
+  if (!block_row_setup(cu_q, cu_k, seqlens, m_seq, S, row, m_max, emax, dst, dst2, status, qi,
+                       own, E, m, tid, BS_CTA_THREADS))
     return;
   const int nf = min(m, 3);
   QRegs qr;
@@ -150,16 +159,18 @@ block_select_cta_kernel(const uint16_t *__restrict__ q, const float *__restrict_
 
 bool use_tc_path(int total_q, int num_sms);
 cudaError_t launch_block_score_tc(const uint16_t *q, const float *reps, const int32_t *cu_q,
-                                  const int32_t *cu_k, const int32_t *seqlens, int S,
-                                  int total_q, int max_seqlen_k, int m, uint8_t *ws,
-                                  uint32_t **scores_out, int *status, cudaStream_t st);
+                                  const int32_t *cu_k, const int32_t *seqlens,
+                                  const int32_t *m_seq, int S, int total_q, int max_seqlen_k,
+                                  int m, uint8_t *ws, uint32_t **scores_out, int *status,
+                                  cudaStream_t st);
 int block_score_stride(int max_seqlen_k);
 
 // Many queries: scores on the tensor cores (block_tc.cu), then one warp per query
 // selects.  Few queries (decode): one warp per query scores on the CUDA cores too.
 cudaError_t launch_block_select(const uint16_t *q, const float *reps, const int32_t *cu_q,
-                                const int32_t *cu_k, const int32_t *seqlens, int S,
-                                int total_q, int max_seqlen_k, int m, int32_t *blk,
+                                const int32_t *cu_k, const int32_t *seqlens,
+                                const int32_t *m_seq, int S, int total_q, int max_seqlen_k,
+                                int m, int32_t *blk,
                                 int32_t *out_blocks, uint8_t *ws, int num_sms, int *status,
                                 cudaStream_t st) {
   if (total_q == 0) return cudaSuccess;
@@ -167,8 +178,8 @@ cudaError_t launch_block_select(const uint16_t *q, const float *reps, const int3
   int tc_stride = 0;
   if (use_tc_path(total_q, num_sms)) {
     uint32_t *sc = nullptr;
-    cudaError_t e = launch_block_score_tc(q, reps, cu_q, cu_k, seqlens, S, total_q, max_seqlen_k,
-                                          m, ws, &sc, status, st);
+    cudaError_t e = launch_block_score_tc(q, reps, cu_q, cu_k, seqlens, m_seq, S, total_q,
+                                          max_seqlen_k, m, ws, &sc, status, st);
     if (e != cudaSuccess) return e;
     tc_keys = sc;
     tc_stride = block_score_stride(max_seqlen_k);
@@ -183,7 +194,7 @@ cudaError_t launch_block_select(const uint16_t *q, const float *reps, const int3
     }
     dim3 grid((total_q + BS_WARPS - 1) / BS_WARPS);
     ProfScope ps(K_BLOCK_SELECT, st);
-    block_select_kernel<<<grid, BS_WARPS * 32, smem, st>>>(cu_q, cu_k, seqlens, S, total_q, m,
+    block_select_kernel<<<grid, BS_WARPS * 32, smem, st>>>(cu_q, cu_k, seqlens, m_seq, S, total_q, m,
                                                          emax > 0 ? emax : 1, tc_keys, tc_stride,
                                                          blk, out_blocks, status);
   } else {
@@ -195,7 +206,7 @@ cudaError_t launch_block_select(const uint16_t *q, const float *reps, const int3
     }
     ProfScope ps(K_BLOCK_SELECT, st);
     block_select_cta_kernel<<<total_q, BS_CTA_THREADS, smem, st>>>(
-        q, reps, cu_q, cu_k, seqlens, S, m, emax > 0 ? emax : 1, blk, out_blocks, status);
+        q, reps, cu_q, cu_k, seqlens, m_seq, S, m, emax > 0 ? emax : 1, blk, out_blocks, status);
   }
   return cudaGetLastError();
 }

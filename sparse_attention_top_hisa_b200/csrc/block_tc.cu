@@ -70,8 +70,8 @@ block_score_tc_kernel(const __grid_constant__ CUtensorMap qmap,
                       const __grid_constant__ CUtensorMap himap,
                       const __grid_constant__ CUtensorMap lomap, const int32_t *__restrict__ cu_q,
                       const int32_t *__restrict__ cu_k, const int32_t *__restrict__ seqlens,
-                      int S, int emax, int estride, int m, uint32_t *__restrict__ scores,
-                      int *status) {
+                      const int32_t *__restrict__ m_seq, int S, int emax, int estride, int m,
+                      uint32_t *__restrict__ scores, int *status) {
   extern __shared__ uint8_t bs_smem_raw[];
   BsSmem &sm = *reinterpret_cast<BsSmem *>((reinterpret_cast<uintptr_t>(bs_smem_raw) + 1023) &
                                            ~(uintptr_t)1023);
@@ -126,7 +126,7 @@ block_score_tc_kernel(const __grid_constant__ CUtensorMap qmap,
   const bool row_ok = row_local < nr;
   const int pos = pos_first + row_local;
   const int own = pos / BLK;
-  const int nf = min(m, 3);
+  const int nf = min(seq_budget(m_seq, s, m, nullptr), 3);  // the top-m stage reports bad budgets
   uint32_t *out_row = scores + (size_t)(q0 + r0 + row_local) * estride;
   uint32_t phase = 0;
   for (int c0 = 0; c0 < e_tile; c0 += BS_TC_N, phase ^= 1u) {
@@ -214,9 +214,10 @@ size_t block_tc_workspace_bytes(int total_q, int num_seqs, int max_seqlen_k) {
 
 // Writes the dense score matrix [total_q x emax] (order-preserving keys) into ws.
 cudaError_t launch_block_score_tc(const uint16_t *q, const float *reps, const int32_t *cu_q,
-                                  const int32_t *cu_k, const int32_t *seqlens, int S,
-                                  int total_q, int max_seqlen_k, int m, uint8_t *ws,
-                                  uint32_t **scores_out, int *status, cudaStream_t st) {
+                                  const int32_t *cu_k, const int32_t *seqlens,
+                                  const int32_t *m_seq, int S, int total_q, int max_seqlen_k,
+                                  int m, uint8_t *ws, uint32_t **scores_out, int *status,
+                                  cudaStream_t st) {
   const BsPlan p = bs_plan(total_q, S, max_seqlen_k);
   const int emax = (max_seqlen_k + BLK - 1) / BLK;
   uint32_t *hi = reinterpret_cast<uint32_t *>(ws + p.off_hi);
@@ -242,8 +243,8 @@ cudaError_t launch_block_score_tc(const uint16_t *q, const float *reps, const in
   {
     ProfScope ps(K_BLOCK_SCORE_TC, st);
     block_score_tc_kernel<<<tiles, BS_TC_THREADS, BS_TC_SMEM, st>>>(
-        qmap, himap, lomap, cu_q, cu_k, seqlens, S, emax, block_score_stride(max_seqlen_k), m,
-        scores, status);
+        qmap, himap, lomap, cu_q, cu_k, seqlens, m_seq, S, emax, block_score_stride(max_seqlen_k),
+        m, scores, status);
   }
   return cudaGetLastError();
 }

@@ -135,6 +135,19 @@ __device__ __forceinline__ QueryInfo locate(const int32_t *cu_q, const int32_t *
   return r;
 }
 
+// Block budget of sequence s: m_seq[s] when a per-sequence array is given, else m_max.
+// A value outside [1, m_max] is clamped into it and raises HISA_ERR_INVALID_ARG (when
+// `status` is not null).
+__device__ __forceinline__ int seq_budget(const int32_t *m_seq, int s, int m_max, int *status) {
+  if (!m_seq) return m_max;
+  const int v = __ldg(m_seq + s);
+  if (v < 1 || v > m_max) {
+    raise_status(status, HISA_ERR_INVALID_ARG);
+    return v < 1 ? 1 : m_max;
+  }
+  return v;
+}
+
 // ---------------------------------------------------------------------------
 // block-wide exclusive scan of one value per thread (NT threads, NT % 32 == 0).
 // `warp_tot` must hold NT/32 + 1 ints of shared memory. Returns the exclusive

@@ -41,7 +41,8 @@ constexpr int DC_CTAS = 8;
 constexpr int DC_THREADS = 256;
 constexpr int DC_WARPS = DC_THREADS / 32;
 constexpr int DC_MAX_E = 8192;  // eligible blocks of one query (a 1M-token sequence)
-constexpr int DC_MAX_CAND = HISA_MAX_M * BLK / DC_CTAS;  // candidates of one CTA
+constexpr int DC_MAX_M = 128;                            // block budgets this path takes
+constexpr int DC_MAX_CAND = DC_MAX_M * BLK / DC_CTAS;    // candidates of one CTA
 constexpr int DC_KPT = DC_MAX_CAND / DC_THREADS;
 constexpr int DC_BINS = 1024;
 constexpr int DC_BIN_WORDS = DC_BINS + DC_BINS / 32;  // bucket b at word b + b / 32
@@ -74,7 +75,7 @@ struct __align__(16) DcSmem {
   uint32_t bcnt[DC_BIN_WORDS];              // D: global bucket counts
   uint32_t curs[DC_BIN_WORDS];              // D: this CTA's scatter cursors
   uint32_t whist[256 + 2 * DC_WARPS];       // B: top-m histogram and warp partials
-  int32_t blocks[HISA_MAX_M];               // B: selected blocks, ascending
+  int32_t blocks[DC_MAX_M];                 // B: selected blocks, ascending
   int pos_lo[DC_CTAS];                      // D: first output position ranked by each CTA
   int bsc[4 + DC_WARPS];                    // B: top-m scratch
   int32_t cuq[DC_LOC_MAX + 1];              // cu_seqlens_q, for the sequence lookup
@@ -116,8 +117,9 @@ struct DcPad {
 __global__ void __cluster_dims__(DC_CTAS, 1, 1) __launch_bounds__(DC_THREADS, 1)
 decode_select_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ k,
                      const float *__restrict__ reps, const int32_t *__restrict__ cu_q,
-                     const int32_t *__restrict__ cu_k, const int32_t *__restrict__ seqlens, int S,
-                     int m, int topk, int emax, int32_t *__restrict__ out_idx,
+                     const int32_t *__restrict__ cu_k, const int32_t *__restrict__ seqlens,
+                     const int32_t *__restrict__ m_seq, int S, int m_max, int topk, int emax,
+                     int32_t *__restrict__ out_idx,
                      float *__restrict__ out_scores, int32_t *__restrict__ out_blocks,
                      int *status) {
   extern __shared__ __align__(16) uint8_t dc_raw[];
@@ -134,7 +136,7 @@ decode_select_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict_
   const float NEG = -__int_as_float(0x7f800000);
   int32_t *oi = out_idx + (size_t)row * topk;
   float *os = out_scores ? out_scores + (size_t)row * topk : nullptr;
-  int32_t *ob = out_blocks ? out_blocks + (size_t)row * m : nullptr;
+  int32_t *ob = out_blocks ? out_blocks + (size_t)row * m_max : nullptr;
   DcPad pad{oi, os};
 
   // every CTA of the cluster locates the same query (the sequence lookup and the query
@@ -184,9 +186,13 @@ decode_select_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict_
     if (qi.ok && me == 0 && tid == 0) raise_status(status, HISA_ERR_INVALID_ARG);
     for (int r = me * DC_THREADS + tid; r < topk; r += DC_CTAS * DC_THREADS) pad(r);
     if (ob && me == 0)
-      for (int i = tid; i < m; i += DC_THREADS) ob[i] = -1;
+      for (int i = tid; i < m_max; i += DC_THREADS) ob[i] = -1;
     return;
   }
+  // this row's block budget; out_blocks entries past it are -1
+  const int m = seq_budget(m_seq, qi.seq, m_max, (me == 0 && tid == 0) ? status : nullptr);
+  if (ob && me == 0)
+    for (int i = m + tid; i < m_max; i += DC_THREADS) ob[i] = -1;
 
   // ---------------- stage 1: blocks ----------------
   if (E > m) {
@@ -528,16 +534,18 @@ decode_select_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict_
   for (int r = kp + me * DC_THREADS + tid; r < topk; r += DC_CTAS * DC_THREADS) pad(r);
 }
 
-// The cluster path covers every query whose eligible blocks fit DC_MAX_E.
-bool decode_path_fits(int max_seqlen_k) {
-  return (max_seqlen_k + BLK - 1) / BLK <= DC_MAX_E;
+// The cluster path covers every query whose eligible blocks fit DC_MAX_E and whose
+// block budget fits DC_MAX_M.
+bool decode_path_fits(int max_seqlen_k, int m) {
+  return (max_seqlen_k + BLK - 1) / BLK <= DC_MAX_E && m <= DC_MAX_M;
 }
 
 cudaError_t launch_decode_select(const uint16_t *q, const uint16_t *k, const float *reps,
                                  const int32_t *cu_q, const int32_t *cu_k,
-                                 const int32_t *seqlens, int S, int total_q, int max_seqlen_k,
-                                 int m, int topk, int32_t *out_idx, float *out_scores,
-                                 int32_t *out_blocks, int *status, cudaStream_t st) {
+                                 const int32_t *seqlens, const int32_t *m_seq, int S,
+                                 int total_q, int max_seqlen_k, int m, int topk,
+                                 int32_t *out_idx, float *out_scores, int32_t *out_blocks,
+                                 int *status, cudaStream_t st) {
   if (total_q == 0) return cudaSuccess;
   static std::atomic<int> attr[64];
   cudaError_t e = set_smem_once((const void *)decode_select_kernel, sizeof(DcSmem), attr);
@@ -546,7 +554,7 @@ cudaError_t launch_decode_select(const uint16_t *q, const uint16_t *k, const flo
   {
     ProfScope ps(K_DECODE_SELECT, st);
     e = launch_pdl((const void *)decode_select_kernel, dim3(total_q * DC_CTAS), dim3(DC_THREADS),
-                   sizeof(DcSmem), st, q, k, reps, cu_q, cu_k, seqlens, S, m, topk,
+                   sizeof(DcSmem), st, q, k, reps, cu_q, cu_k, seqlens, m_seq, S, m, topk,
                    emax > 0 ? emax : 1, out_idx, out_scores, out_blocks, status);
   }
   if (e != cudaSuccess) return e;

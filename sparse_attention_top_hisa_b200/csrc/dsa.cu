@@ -58,14 +58,10 @@ key_norm_kernel(const uint16_t *__restrict__ k, const int32_t *__restrict__ cu_k
   if ((threadIdx.x & 31) == 0 && nrm > 0.f) atomicMax(reinterpret_cast<int *>(kmax + s), __float_as_int(nrm));
 }
 
-struct DsaOut {
-  int32_t *idx;
-  float *scores;
+// Output index of list entry c: the key position stored beside its score.
+struct ListTok {
   const int32_t *bj;
-  __device__ void operator()(int r, int c, uint32_t u) const {
-    idx[r] = bj[c];
-    if (scores) scores[r] = key_score(u);
-  }
+  __device__ int operator()(int c) const { return bj[c]; }
 };
 
 struct DirectOut {
@@ -87,7 +83,7 @@ struct DsaPad {
 };
 
 __host__ __device__ inline size_t dsa_select_smem(int topk) {
-  return (size_t)16 * topk + sizeof(LinShared);
+  return sl_work_bytes(topk) + sizeof(SlShared);
 }
 
 __global__ void __launch_bounds__(DSA_SEL_THREADS)
@@ -98,14 +94,15 @@ dsa_select_kernel(int row0, int topk, int cap, const float *__restrict__ buf_key
   const int local = blockIdx.x, row = row0 + local;
   const int n = cnt[local];
   if (n > cap) return;  // the fallback kernel owns this row
-  uint32_t *work = reinterpret_cast<uint32_t *>(smem);
-  LinShared &sh = *reinterpret_cast<LinShared *>(smem + (size_t)16 * topk);
+  SlShared &sh = *reinterpret_cast<SlShared *>(smem + sl_work_bytes(topk));
   int32_t *oi = out_idx + (size_t)row * topk;
   float *os = out_scores ? out_scores + (size_t)row * topk : nullptr;
-  select_topk_reg<DSA_SEL_THREADS, DSA_SEL_KPT>(RowScores{buf_key + (size_t)local * cap}, n, topk,
-                                                sh, work,
-                                                DsaOut{oi, os, buf_j + (size_t)local * cap},
-                                                DsaPad{oi, os});
+  const RowScores src{buf_key + (size_t)local * cap};
+  RegCands<DSA_SEL_THREADS, DSA_SEL_KPT> cs;
+  float mx, mn;
+  cs.load(src, n, mx, mn);
+  select_topk_lin<DSA_SEL_THREADS>(cs, mx, mn, src, n, topk, sh, smem,
+                                   ListTok{buf_j + (size_t)local * cap}, oi, os);
 }
 
 __global__ void __launch_bounds__(DSA_SEL_THREADS)

@@ -25,6 +25,8 @@ enum KernelKind {
   K_BLOCK_SCORE_TC,
   K_DECODE_SELECT,
   K_SPARSE_ATTENTION,
+  K_EXPAND_BLOCKS,
+  K_FRACTION_BUDGET,
   K_NUM_KINDS
 };
 

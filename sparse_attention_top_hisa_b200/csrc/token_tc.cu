@@ -68,16 +68,16 @@ constexpr size_t TC_SMEM_BYTES = sizeof(TcSmem) + 1024;
 // more compact blocks than fit in shared memory uses global atomics directly.
 //   mode 0: add the pair counts of every key block to cnt;
 //   mode 1: reserve each key block's share of its list (cursor holds the list
-//           starts), write the entries row << 7 | slot, and record each pair's list
+//           starts), write the entries row << sb | slot, and record each pair's list
 //           position in pmap[row * m + slot] (where its scores will be).
+// Slots past a row's block budget hold -1 and are skipped.
 constexpr int INV_THREADS = 256;
 constexpr int INV_ROWS = 256;
 constexpr int INV_LOCAL_BINS = 8192;
-constexpr int INV_RB = 8;                      // rows whose block ids a warp loads at once
-constexpr int INV_SLOTS = (HISA_MAX_M + 31) / 32;  // slots per lane (m <= HISA_MAX_M)
+constexpr int INV_RB = 8;  // rows whose block ids a warp loads at once
 
 __global__ void __launch_bounds__(INV_THREADS)
-inv_lists_kernel(const int32_t *__restrict__ blk, int total_q, int m,
+inv_lists_kernel(const int32_t *__restrict__ blk, int total_q, int m, int sb,
                  const int32_t *__restrict__ cu_q, int S, int emax, int mode,
                  int *__restrict__ cnt, int *__restrict__ cursor, uint32_t *__restrict__ list,
                  int32_t *__restrict__ pmap) {
@@ -95,30 +95,31 @@ inv_lists_kernel(const int32_t *__restrict__ blk, int total_q, int m,
   const int base = s0 * emax;
   const int nbl = (s1 - s0 + 1) * emax;
   const bool local = nbl <= INV_LOCAL_BINS;
-  // walk the pairs: warp w takes rows r0 + w, r0 + w + NW, ...; lane = slot.  The
-  // block ids of INV_RB rows are loaded before any is used, so that a warp keeps that
-  // many loads in flight instead of one.
+  // walk the pairs: warp w takes rows r0 + w, r0 + w + NW, ...; lane = slot within a
+  // chunk of 32 slots.  The block ids of INV_RB rows are loaded before any is used, so
+  // that a warp keeps that many loads in flight instead of one.
   auto walk = [&](auto &&fn) {
     int s = s0;
     for (int rb = r0 + warp; rb < r1; rb += NW * INV_RB) {
-      int b[INV_RB][INV_SLOTS];
+      int sq[INV_RB];
 #pragma unroll
       for (int u = 0; u < INV_RB; u++) {
         const int row = rb + u * NW;
-#pragma unroll
-        for (int c = 0; c < INV_SLOTS; c++) {
-          const int slot = lane + 32 * c;
-          b[u][c] = (row < r1 && slot < m) ? __ldg(blk + (size_t)row * m + slot) : -1;
-        }
+        if (row < r1)
+          while (s < s1 && __ldg(cu_q + s + 1) <= row) s++;
+        sq[u] = s;
       }
+      for (int c0 = 0; c0 < m; c0 += 32) {
+        const int slot = c0 + lane;
+        int b[INV_RB];
 #pragma unroll
-      for (int u = 0; u < INV_RB; u++) {
-        const int row = rb + u * NW;
-        if (row >= r1) break;
-        while (s < s1 && __ldg(cu_q + s + 1) <= row) s++;
+        for (int u = 0; u < INV_RB; u++) {
+          const int row = rb + u * NW;
+          b[u] = (row < r1 && slot < m) ? __ldg(blk + (size_t)row * m + slot) : -1;
+        }
 #pragma unroll
-        for (int c = 0; c < INV_SLOTS; c++)
-          if (b[u][c] >= 0) fn(row, lane + 32 * c, s * emax + b[u][c]);
+        for (int u = 0; u < INV_RB; u++)
+          if (b[u] >= 0) fn(rb + u * NW, slot, sq[u] * emax + b[u]);
       }
     }
   };
@@ -128,7 +129,7 @@ inv_lists_kernel(const int32_t *__restrict__ blk, int total_q, int m,
     else
       walk([&](int row, int slot, int cb) {
         const int p = atomicAdd(cursor + cb, 1);
-        list[p] = ((uint32_t)row << 7) | (uint32_t)slot;
+        list[p] = ((uint32_t)row << sb) | (uint32_t)slot;
         pmap[(size_t)row * m + slot] = p;
       });
     return;
@@ -147,7 +148,7 @@ inv_lists_kernel(const int32_t *__restrict__ blk, int total_q, int m,
   __syncthreads();
   walk([&](int row, int slot, int cb) {
     const int p = atomicAdd(&loc[cb - base], 1);
-    list[p] = ((uint32_t)row << 7) | (uint32_t)slot;
+    list[p] = ((uint32_t)row << sb) | (uint32_t)slot;
     pmap[(size_t)row * m + slot] = p;
   });
 }
@@ -219,19 +220,20 @@ __device__ __forceinline__ TileSeq tile_seq(const TileDesc &td, int emax, const 
 }
 
 __global__ void __launch_bounds__(TC_THREADS, 1)
-token_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const uint16_t *__restrict__ q,
+token_score_tc_kernel(const uint16_t *__restrict__ q,
                       const uint16_t *__restrict__ k, const int32_t *__restrict__ cu_q,
                       const int32_t *__restrict__ cu_k, const int32_t *__restrict__ seqlens,
-                      int emax, int m, const TileDesc *__restrict__ tiles,
+                      int emax, int sb, const TileDesc *__restrict__ tiles,
                       const int *__restrict__ ntiles_ptr, const uint32_t *__restrict__ list,
-                      float *__restrict__ scratch, int *status) {
+                      float *__restrict__ scratch, int *status, int *launch_abort,
+                      int test_no_loads) {
   extern __shared__ uint8_t tc_smem_raw[];
   TcSmem &sm = *reinterpret_cast<TcSmem *>((reinterpret_cast<uintptr_t>(tc_smem_raw) + 1023) &
                                            ~(uintptr_t)1023);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
     for (int i = 0; i < TC_STAGES; i++) {
-      mbar_init(&sm.full[i], TC_LOADERS + 1);  // every loader thread + the key TMA issuer
+      mbar_init(&sm.full[i], TC_LOADERS);  // every loader thread, once its copies landed
       mbar_init(&sm.empty[i], 1);
     }
     for (int i = 0; i < 2; i++) {
@@ -240,7 +242,6 @@ token_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const uint16_t *
     }
     sm.abort = 0;
     fence_barrier_init();
-    prefetch_tmap(&kmap);
   }
   if (warp == 0) {
     tmem_alloc(&sm.tmem_base, TC_TMEM_COLS);
@@ -257,30 +258,27 @@ token_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const uint16_t *
     // ---------------- loaders: key block (TMA or cp.async) and query gather ----------------
     const int lt = tid - TC_LOAD_WARP0 * 32;
     int i = 0;
-    for (int t = blockIdx.x; t < ntiles; t += gridDim.x, i++) {
+    // test_no_loads (tests of the timeout path only): the loaders issue nothing, so the
+    // MMA thread's first wait runs out with no copy and no MMA in flight
+    for (int t = test_no_loads ? ntiles : blockIdx.x; t < ntiles; t += gridDim.x, i++) {
       const int s = i % TC_STAGES;
       const TileDesc td = tiles[t];  // fetched while the stage drains
       const TileSeq ts = tile_seq(td, emax, cu_q, cu_k, seqlens);
-      if (i >= TC_STAGES && !mbar_wait(&sm.empty[s], (uint32_t)(((i / TC_STAGES) & 1) ^ 1), status)) {
+      if (i >= TC_STAGES &&
+          !mbar_wait(&sm.empty[s], (uint32_t)(((i / TC_STAGES) & 1) ^ 1), status, abort_flag)) {
         *abort_flag = 1;
+        atomicExch(launch_abort, 1);
         break;
       }
       if (*abort_flag) break;
-      const int live = ts.len - ts.b * BLK;
+      const int live = min(BLK, ts.len - ts.b * BLK);
       const uint32_t sq = smem_u32(sm.q[s]), sk = smem_u32(sm.k[s]);
-      if (lt == 0) {
-        if (live >= BLK) {
-          mbar_arrive_expect_tx(&sm.full[s], BLK * ROW_BYTES);
-          tma_load_2d(sm.k[s], &kmap, &sm.full[s], 0, ts.kbase + ts.b * BLK);
-        } else {
-          mbar_arrive(&sm.full[s]);
-        }
-      }
-      if (live < BLK) {  // partial last block: only the rows that exist (the rest is masked)
-        for (int x = lt; x < live * 8; x += TC_LOADERS) {
-          const int r = x >> 3, c = x & 7;
-          cp_async_16(sk + sw128_offset(r, c), k + (size_t)(ts.kbase + ts.b * BLK + r) * D + c * 8);
-        }
+      // the key block, by cp.async like the queries, so that one wait_all covers every
+      // copy a loader has in flight; a partial last block loads only the rows that
+      // exist (the others are masked)
+      for (int x = lt; x < live * 8; x += TC_LOADERS) {
+        const int r = x >> 3, c = x & 7;
+        cp_async_16(sk + sw128_offset(r, c), k + (size_t)(ts.kbase + ts.b * BLK + r) * D + c * 8);
       }
       // the selecting queries, in chunks of 32 rows (chunk c is loaded by loader warp
       // c % TC_LOAD_WARPS): one coalesced read of the chunk's list entries, then lane l
@@ -304,7 +302,7 @@ token_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const uint16_t *
               const int rl = i2 * 4 + (lane >> 3), row = c * 32 + rl, piece = lane & 7;
               const uint32_t e = __shfl_sync(0xffffffffu, ent[j], rl);
               if (row < td.n)
-                cp_async_16(sq + sw128_offset(row, piece), q + (size_t)(e >> 7) * D + piece * 8);
+                cp_async_16(sq + sw128_offset(row, piece), q + (size_t)(e >> sb) * D + piece * 8);
             }
           }
         }
@@ -318,7 +316,7 @@ token_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const uint16_t *
         mbar_arrive(&sm.full[(i - 1) % TC_STAGES]);
       }
     }
-    if (i > 0) {  // the last tile issued (nothing is pending after an abort's break)
+    if (i > 0) {  // the last tile issued; after an abort, every copy still lands first
       cp_async_wait_all();
       fence_proxy_async_smem();
       if (!*abort_flag) mbar_arrive(&sm.full[(i - 1) % TC_STAGES]);
@@ -333,6 +331,7 @@ token_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const uint16_t *
         if (!mbar_wait(&sm.full[s], (uint32_t)((i / TC_STAGES) & 1), status) ||
             (i >= 2 && !mbar_wait(&sm.acc_empty[a], (uint32_t)(((i >> 1) & 1) ^ 1), status))) {
           *abort_flag = 1;
+          atomicExch(launch_abort, 1);  // the select pads every row of this launch
           break;
         }
         if (*abort_flag) break;
@@ -346,6 +345,9 @@ token_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const uint16_t *
         umma_commit(&sm.empty[s]);
         umma_commit(&sm.acc_full[a]);
       }
+      // before the CTA frees TMEM, the last issued product (and so every earlier one)
+      // has completed, also when the loop above gave up
+      if (i > 0) mbar_wait(&sm.acc_full[(i - 1) & 1], (uint32_t)(((i - 1) >> 1) & 1), status);
     }
     __syncwarp();
   } else {
@@ -366,8 +368,9 @@ token_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const uint16_t *
         const int c = c_beg + 32 * j + lane;
         ej[j] = c < c_end ? __ldg(list + td.list_off + c) : 0u;
       }
-      if (!mbar_wait(&sm.acc_full[a], (uint32_t)((i >> 1) & 1), status)) {
+      if (!mbar_wait(&sm.acc_full[a], (uint32_t)((i >> 1) & 1), status, abort_flag)) {
         *abort_flag = 1;
+        atomicExch(launch_abort, 1);
         break;
       }
       tc_fence_after();
@@ -387,7 +390,7 @@ token_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const uint16_t *
             for (int u = 0; u < 32; u++) {
               const uint32_t e = __shfl_sync(0xffffffffu, ej[j], u);
               if (c0 + u < c_end) {
-                const int row = (int)(e >> 7);
+                const int row = (int)(e >> sb);
                 scratch[(size_t)(td.list_off + c0 + u) * BLK + r] =
                     row >= rlim ? __uint_as_float(v[u]) : NEG;
               }
@@ -455,8 +458,8 @@ TcPlan tc_plan(int total_q, int num_seqs, int max_seqlen_k, int m) {
   const long long pairs = (long long)total_q * m;
   p.max_tiles = (int)(pairs / TC_N + p.nb + 1);
   size_t off = 0;
-  p.off_cnt = off;
-  off = a256(off + (size_t)p.nb * 4);
+  p.off_cnt = off;  // nb counters, then the launch's abort word
+  off = a256(off + (size_t)(p.nb + 1) * 4);
   p.off_cursor = off;
   off = a256(off + (size_t)p.nb * 4);
   p.off_ntiles = off;
@@ -480,11 +483,15 @@ size_t tc_workspace_bytes(int total_q, int num_seqs, int max_seqlen_k, int m) {
 // Scores every selected (query, block) pair into ws's score buffer (one 128-score
 // segment per list entry; *pmap_out[row * m + slot] names the segment of each pair),
 // ready for the select kernel.
+// Tests of the timeout path only (hisa_test_fault): launches made while it is set
+// issue no loads.
+std::atomic<int> g_test_no_loads{0};
+
 cudaError_t launch_token_score_tc(const uint16_t *q, const uint16_t *k, const int32_t *cu_q,
                                   const int32_t *cu_k, const int32_t *seqlens, int S,
                                   int total_q, int max_seqlen_k, int m, const int32_t *blk,
                                   uint8_t *ws, float **scores_out, const int32_t **pmap_out,
-                                  int num_sms, int *status, cudaStream_t st) {
+                                  int **abort_out, int num_sms, int *status, cudaStream_t st) {
   const TcPlan p = tc_plan(total_q, S, max_seqlen_k, m);
   const int emax = (max_seqlen_k + BLK - 1) / BLK;
   int *cnt = reinterpret_cast<int *>(ws + p.off_cnt);
@@ -496,14 +503,15 @@ cudaError_t launch_token_score_tc(const uint16_t *q, const uint16_t *k, const in
   int32_t *pmap = reinterpret_cast<int32_t *>(ws + p.off_pmap);
   *scores_out = scores;
   *pmap_out = pmap;
-  CUtensorMap kmap;
-  if (!make_key_tensor_map(&kmap, k)) return cudaErrorInvalidValue;
-  cudaError_t e = cudaMemsetAsync(cnt, 0, (size_t)p.nb * 4, st);
+  int *launch_abort = cnt + p.nb;
+  *abort_out = launch_abort;
+  cudaError_t e = cudaMemsetAsync(cnt, 0, (size_t)(p.nb + 1) * 4, st);
   if (e != cudaSuccess) return e;
   const int grid = (total_q + INV_ROWS - 1) / INV_ROWS;
+  const int sb = m > 128 ? 9 : 7;  // slot bits of a list entry (row << sb | slot)
   {
     ProfScope ps(K_INV_LISTS, st);
-    inv_lists_kernel<<<grid, INV_THREADS, 0, st>>>(blk, total_q, m, cu_q, S, emax, 0, cnt, cursor, list,
+    inv_lists_kernel<<<grid, INV_THREADS, 0, st>>>(blk, total_q, m, sb, cu_q, S, emax, 0, cnt, cursor, list,
                                                    pmap);
   }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -514,7 +522,7 @@ cudaError_t launch_token_score_tc(const uint16_t *q, const uint16_t *k, const in
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   {
     ProfScope ps(K_INV_LISTS, st);
-    inv_lists_kernel<<<grid, INV_THREADS, 0, st>>>(blk, total_q, m, cu_q, S, emax, 1, cnt, cursor, list,
+    inv_lists_kernel<<<grid, INV_THREADS, 0, st>>>(blk, total_q, m, sb, cu_q, S, emax, 1, cnt, cursor, list,
                                                    pmap);
   }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -524,7 +532,8 @@ cudaError_t launch_token_score_tc(const uint16_t *q, const uint16_t *k, const in
   {
     ProfScope ps(K_TOKEN_SCORE_TC, st);
     token_score_tc_kernel<<<num_sms, TC_THREADS, TC_SMEM_BYTES, st>>>(
-        kmap, q, k, cu_q, cu_k, seqlens, emax, m, tiles, ntiles, list, scores, status);
+        q, k, cu_q, cu_k, seqlens, emax, sb, tiles, ntiles, list, scores, status,
+        launch_abort, g_test_no_loads.load(std::memory_order_relaxed));
   }
   return cudaGetLastError();
 }

@@ -139,3 +139,44 @@ def check_block_band(w, rows, gpu_blocks, ora_blocks, ora_reps):
                 problems.append((row, "block", b))
                 break
     assert not problems, f"block sets: {len(problems)} rows fail the band rule, e.g. {problems[:5]}"
+
+
+def query_positions(w) -> np.ndarray:
+    """Sequence-local position of every query row (the last q_len positions)."""
+    out = np.empty(w.total_q, np.int64)
+    for s in range(w.num_seqs):
+        a, b = int(w.cu_q[s]), int(w.cu_q[s + 1])
+        L = int(w.seqlens[s])
+        out[a:b] = np.arange(L - (b - a), L)
+    return out
+
+
+def check_rows_structure(w, idx: np.ndarray, sc: np.ndarray, flat: bool, chunk: int = 16384):
+    """Every row, checked on the device: -1 only as a suffix; 0 <= j <= i; no duplicate
+    index; scores non-increasing with equal scores in ascending index; and exactly
+    min(k, c_i) valid entries, c_i the candidate count (i + 1 for the flat scan;
+    (min(m, own + 1) - 1) * B + i % B + 1 for HISA, whose own block is always selected
+    and whose other selected blocks lie wholly before the query)."""
+    pos_all = query_positions(w)
+    own = pos_all // w.B
+    cand = pos_all + 1 if flat else (np.minimum(w.m, own + 1) - 1) * w.B + pos_all % w.B + 1
+    want = np.minimum(w.topk, cand)
+    for r0 in range(0, idx.shape[0], chunk):
+        r1 = min(idx.shape[0], r0 + chunk)
+        I = torch.from_numpy(np.ascontiguousarray(idx[r0:r1])).cuda().long()
+        S = torch.from_numpy(np.ascontiguousarray(sc[r0:r1])).cuda()
+        pos = torch.from_numpy(pos_all[r0:r1]).cuda()
+        valid = I >= 0
+        assert not bool((I < -1).any()), "index below -1"
+        assert not bool((valid[:, 1:] & ~valid[:, :-1]).any()), "-1 before a valid entry"
+        assert not bool(((I > pos[:, None]) & valid).any()), "index after the query"
+        nv = valid.sum(dim=1).cpu().numpy()
+        assert np.array_equal(nv, want[r0:r1]), "valid count differs from min(k, candidates)"
+        srt = torch.sort(I, dim=1).values
+        assert not bool(((srt[:, 1:] == srt[:, :-1]) & (srt[:, 1:] >= 0)).any()), "duplicate"
+        v2 = valid[:, 1:]
+        assert not bool(((S[:, 1:] > S[:, :-1]) & v2).any()), "scores increase along a row"
+        assert not bool(((S[:, 1:] == S[:, :-1]) & v2 & (I[:, 1:] < I[:, :-1])).any()), \
+            "equal scores out of index order"
+        del I, S, pos, valid, srt
+    torch.cuda.empty_cache()

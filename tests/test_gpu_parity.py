@@ -11,8 +11,8 @@ import pytest
 import torch
 
 import oracle
-from parity import (OnDevice, check_block_band, check_token_band, dev_bf16, dev_i32,
-                    exact_scores, sample_rows)
+from parity import (OnDevice, check_block_band, check_rows_structure, check_token_band, dev_bf16,
+                    dev_i32, exact_scores, sample_rows)
 from synth import (bf16_from_f32, config_workload, decode_workload, gaussian_prefill,
                    integer_prefill, varlen_prefill)
 
@@ -252,7 +252,7 @@ def _gauss_hisa_check(w, n_rows, seed):
                                       rows=rows)
     check_token_band(w, rows, idx[rows], sc[rows], r_idx, r_sc, "hisa")
     # every row, not just the sampled ones, is structurally valid
-    assert np.all((idx >= -1))
+    check_rows_structure(w, idx, sc, flat=False)
     return idx, sc, bl
 
 
@@ -262,6 +262,7 @@ def _gauss_dsa_check(w, n_rows, seed):
     rows = sample_rows(w, n_rows, seed)
     o_idx, o_sc = oracle.dsa_workload(w, rows=rows)
     check_token_band(w, rows, idx[rows], sc[rows], o_idx, o_sc, "dsa")
+    check_rows_structure(w, idx, sc, flat=True)
     return idx
 
 
