@@ -698,8 +698,9 @@ def stream_ceilings(stream, nbytes=4 << 30, reps=5):
 
 def decode_bench(flush, stream, hbm_peak, n_states=4, steps=256):
     """16 sequences x 32768 keys; each step appends one key per sequence and selects
-    for one query per sequence. Steps rotate over n_states independent decode states
-    (4 x 67.6 MB of key cache > L2) and the 256 steps run as one CUDA graph."""
+    for one query per sequence (hisa_decode_step: one launch per step). Steps rotate
+    over n_states independent decode states (4 x 67.6 MB of key cache > L2) and the 256
+    steps run as one CUDA graph."""
     import torch
     import sparse_attention_top_hisa_b200 as H
     from synth import config_workload
@@ -719,11 +720,11 @@ def decode_bench(flush, stream, hbm_peak, n_states=4, steps=256):
     qs = to_dev_bf16(dw.queries.reshape(steps * S, 64)).view(steps, S, 64)
     ws = torch.empty(H.hisa_select_workspace_size(S, S, cap, m, K), dtype=torch.uint8, device="cuda")
 
-    def run_steps():
+    def run_steps():  # one launch per step: append and select fused (hisa_decode_step)
         for i in range(steps):
             kc, lens, reps, out = states[i % n_states]
-            H.hisa_append_keys(kc, reps, cu_k, lens, newk[i])
-            H.hisa_select(qs[i], kc, reps, cu_q, cu_k, lens, cap, m, K, out_idx=out, workspace=ws)
+            H.hisa_decode_step(kc, reps, cu_k, lens, newk[i].view(S, 64), qs[i], cap, m, K,
+                               out_idx=out)
 
     def reset():
         for kc, lens, reps, out in states:

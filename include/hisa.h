@@ -186,6 +186,31 @@ size_t hisa_select_workspace_size(int total_q, int num_seqs, int max_seqlen_k, i
                                   int k);
 
 /*
+ * hisa_decode_step — one decode step of a batch in one launch: the KV-cache update of
+ * hisa_append_keys with one new key per sequence (the representative of the block
+ * that receives it is refreshed, HISA summary page, paragraph on KV-cache maintenance)
+ * and hisa_select for one query per sequence, placed at the new key's position.  The
+ * outputs, the cache, the representatives and the lengths equal those of
+ * hisa_append_keys(n_new = 1) followed by hisa_select with cu_seqlens_q = 0, 1, ...,
+ * num_seqs, bit for bit.
+ *
+ *   k_cache, reps, cu_seqlens_k, seqlens_k (in/out)   as in hisa_append_keys.
+ *   new_keys       bf16 [num_seqs, 64]: the key appended to each sequence.
+ *   q_idx          bf16 [num_seqs, 64]: the query of each sequence.
+ *   max_seqlen_k   >= every length after the append; at most 8192 blocks (the
+ *                  few-query path), else HISA_ERR_NOT_IMPLEMENTED.
+ *   m, k, out_idx, out_scores, out_blocks   as in hisa_select (m <= 128 here).
+ * A sequence whose region cannot take one more key is left unchanged, its row is
+ * written as -1 and HISA_ERR_CAPACITY is raised in the device status word.  No
+ * workspace.
+ */
+hisa_status hisa_decode_step(hisa_bf16 *k_cache, float *reps, const int32_t *cu_seqlens_k,
+                             int32_t *seqlens_k, const hisa_bf16 *new_keys,
+                             const hisa_bf16 *q_idx, int num_seqs, int max_seqlen_k, int B, int m,
+                             int k, int32_t *out_idx, float *out_scores, int32_t *out_blocks,
+                             hisa_stream_t stream);
+
+/*
  * hisa_select_varm — hisa_select with a block budget per sequence.  The pages mention
  * a fractional setting ("HISA 50%") and adaptive sparsity (idea.jsleekr.com summary
  * and its transcript) without defining them; this library reads them as a block

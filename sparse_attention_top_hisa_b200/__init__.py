@@ -19,6 +19,7 @@ from .binding import (  # noqa: F401
     hisa_append_keys,
     hisa_block_sparse_select,
     hisa_block_sparse_workspace_size,
+    hisa_decode_step,
     hisa_device_status,
     hisa_pool_blocks,
     hisa_fraction_blocks,

@@ -57,6 +57,7 @@ EXPORTED = (
     "hisa_block_sparse_select",
     "hisa_block_sparse_workspace_size",
     "hisa_test_fault",
+    "hisa_decode_step",
 )
 
 
@@ -104,6 +105,8 @@ def lib() -> ctypes.CDLL:
         L.hisa_block_sparse_select.argtypes = [P, P, P, P, P, I, I, I, I, I, P, P, P, Z, P]
         L.hisa_block_sparse_workspace_size.argtypes = [I, I, I, I, I]
         L.hisa_block_sparse_workspace_size.restype = Z
+        L.hisa_decode_step.argtypes = [P, P, P, P, P, P, I, I, I, I, I, P, P, P, P]
+        L.hisa_decode_step.restype = I
         L.hisa_test_fault.argtypes = [I]
         L.hisa_test_fault.restype = I
         for f in ("hisa_pool_blocks", "hisa_append_keys", "hisa_select", "dsa_flat_select",
@@ -221,6 +224,35 @@ def hisa_select(q_idx: torch.Tensor, k_idx: torch.Tensor, reps: torch.Tensor,
                              _ptr(cu_seqlens_k), _ptr(seqlens_k), S, total_q, int(max_seqlen_k),
                              B, m, k, _ptr(out_idx), _ptr(out_scores), _ptr(out_blocks), _ptr(ws),
                              ws.numel(), _stream(stream)), "hisa_select")
+    return out_idx
+
+
+def hisa_decode_step(k_cache: torch.Tensor, reps: torch.Tensor, cu_seqlens_k: torch.Tensor,
+                     seqlens_k: torch.Tensor, new_keys: torch.Tensor, q_idx: torch.Tensor,
+                     max_seqlen_k: int, m: int, k: int, B: int = HISA_BLOCK,
+                     out_idx: Optional[torch.Tensor] = None,
+                     out_scores: Optional[torch.Tensor] = None,
+                     out_blocks: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """One decode step in one launch: append new_keys [S, 64] (one per sequence) and select
+    for q_idx [S, 64] at the new positions; returns out_idx int32 [S, k]."""
+    _need(k_cache, "k_cache", torch.bfloat16, HISA_INDEX_DIM)
+    _need(reps, "reps", torch.float32, HISA_INDEX_DIM)
+    _need(cu_seqlens_k, "cu_seqlens_k", torch.int32)
+    _need(seqlens_k, "seqlens_k", torch.int32)
+    _need(new_keys, "new_keys", torch.bfloat16)
+    _need(q_idx, "q_idx", torch.bfloat16, HISA_INDEX_DIM)
+    S = cu_seqlens_k.numel() - 1
+    if new_keys.numel() != S * HISA_INDEX_DIM or q_idx.shape[0] != S:
+        raise ValueError("new_keys and q_idx need one row per sequence")
+    if out_idx is None:
+        out_idx = torch.empty(S, k, dtype=torch.int32, device=q_idx.device)
+    _need(out_idx, "out_idx", torch.int32, k)
+    _need(out_scores, "out_scores", torch.float32, k, optional=True)
+    _need(out_blocks, "out_blocks", torch.int32, m, optional=True)
+    _check(lib().hisa_decode_step(_ptr(k_cache), _ptr(reps), _ptr(cu_seqlens_k), _ptr(seqlens_k),
+                                  _ptr(new_keys), _ptr(q_idx), S, int(max_seqlen_k), B, m, k,
+                                  _ptr(out_idx), _ptr(out_scores), _ptr(out_blocks),
+                                  _stream(stream)), "hisa_decode_step")
     return out_idx
 
 

@@ -51,7 +51,9 @@ cudaError_t launch_decode_select(const uint16_t *q, const uint16_t *k, const flo
                                  const int32_t *seqlens, const int32_t *m_seq, int S,
                                  int total_q, int max_seqlen_k, int m, int topk,
                                  int32_t *out_idx, float *out_scores, int32_t *out_blocks,
-                                 int *status, cudaStream_t st);
+                                 int *status, cudaStream_t st, uint16_t *append_kc = nullptr,
+                                 float *append_reps = nullptr, int32_t *append_seqlens = nullptr,
+                                 const uint16_t *new_keys = nullptr);
 }  // namespace hisa
 
 using namespace hisa;
@@ -272,8 +274,10 @@ hisa_status select_args(const hisa_bf16 *q_idx, const hisa_bf16 *k_idx, const fl
       !aligned(m_seq, 4) || !aligned(out_idx, 4) || !aligned(out_scores, 4) ||
       !aligned(out_blocks, 4))
     return HISA_ERR_UNALIGNED;
-  // list entries hold row << 7 | slot (m <= 128) or row << 9 | slot
+  // list entries hold row << 7 | slot (m <= 128) or row << 9 | slot, and list positions
+  // (rows rounded up to a whole chunk, times m) are int32
   if (total_q >= (m > 128 ? (1 << 23) : (1 << 25))) return HISA_ERR_INVALID_ARG;
+  if ((long long)(total_q + 65536) * m >= (1ll << 31)) return HISA_ERR_INVALID_ARG;
   return HISA_OK;
 }
 
@@ -347,6 +351,31 @@ hisa_status hisa_select_varm(const hisa_bf16 *q_idx, const hisa_bf16 *k_idx, con
   return select_with_workspace(q_idx, k_idx, reps, cu_seqlens_q, cu_seqlens_k, seqlens_k, m_seq,
                                num_seqs, total_q, max_seqlen_k, B, m_max, k, out_idx,
                                out_scores, out_blocks, ws, ws_bytes, stream);
+}
+
+hisa_status hisa_decode_step(hisa_bf16 *k_cache, float *reps, const int32_t *cu_seqlens_k,
+                             int32_t *seqlens_k, const hisa_bf16 *new_keys,
+                             const hisa_bf16 *q_idx, int num_seqs, int max_seqlen_k, int B, int m,
+                             int k, int32_t *out_idx, float *out_scores, int32_t *out_blocks,
+                             hisa_stream_t stream) {
+  if (B != HISA_BLOCK || m < 1 || m > HISA_MAX_M || k < 1 || k > HISA_MAX_TOPK ||
+      num_seqs < 0 || max_seqlen_k < 0)
+    return HISA_ERR_INVALID_ARG;
+  if (num_seqs == 0) return HISA_OK;
+  if (!k_cache || !reps || !cu_seqlens_k || !seqlens_k || !new_keys || !q_idx || !out_idx)
+    return HISA_ERR_INVALID_ARG;
+  if (!aligned(k_cache, 16) || !aligned(reps, 16) || !aligned(new_keys, 16) ||
+      !aligned(q_idx, 16) || !aligned(cu_seqlens_k, 4) || !aligned(seqlens_k, 4) ||
+      !aligned(out_idx, 4) || !aligned(out_scores, 4) || !aligned(out_blocks, 4))
+    return HISA_ERR_UNALIGNED;
+  if (!decode_path_fits(max_seqlen_k, m)) return HISA_ERR_NOT_IMPLEMENTED;
+  int *st = status_word();
+  if (!st) return HISA_ERR_CUDA;
+  return from_cuda(launch_decode_select(q_idx, k_cache, reps, nullptr, cu_seqlens_k, seqlens_k,
+                                        nullptr, num_seqs, num_seqs, max_seqlen_k, m, k, out_idx,
+                                        out_scores, out_blocks, st,
+                                        static_cast<cudaStream_t>(stream), k_cache, reps,
+                                        seqlens_k, new_keys));
 }
 
 hisa_status hisa_fraction_blocks(const int32_t *cu_seqlens_k, const int32_t *seqlens_k,

@@ -48,6 +48,7 @@ constexpr int DC_BINS = 1024;
 constexpr int DC_BIN_WORDS = DC_BINS + DC_BINS / 32;  // bucket b at word b + b / 32
 constexpr int DC_MAXK = HISA_MAX_TOPK;
 constexpr int DC_LOC_MAX = 1024;  // sequences looked up cooperatively (else by binary search)
+constexpr int DC_WARP_TOPM_E = 1024;  // eligible blocks up to which one warp runs the top-m
 constexpr size_t LIN_BLK_SCRATCH_MAX = (size_t)LIN_BLK_CAP * 8 + DC_MAX_E;
 static_assert(DC_KPT * DC_THREADS == DC_MAX_CAND, "candidates split evenly");
 
@@ -114,21 +115,25 @@ struct DcPad {
   }
 };
 
-__global__ void __cluster_dims__(DC_CTAS, 1, 1) __launch_bounds__(DC_THREADS, 1)
-decode_select_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ k,
-                     const float *__restrict__ reps, const int32_t *__restrict__ cu_q,
-                     const int32_t *__restrict__ cu_k, const int32_t *__restrict__ seqlens,
-                     const int32_t *__restrict__ m_seq, int S, int m_max, int topk, int emax,
-                     int32_t *__restrict__ out_idx,
-                     float *__restrict__ out_scores, int32_t *__restrict__ out_blocks,
-                     int *status) {
-  extern __shared__ __align__(16) uint8_t dc_raw[];
-  DcSmem &sm = *reinterpret_cast<DcSmem *>(dc_raw);
-  // Launched as a programmatic dependent of the previous kernel on the stream (when
-  // the stream allows it): nothing is read before that kernel has completed, and the
-  // next kernel may begin launching at once (it waits the same way).
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+// The append of a fused decode step (hisa_decode_step); all null otherwise.  The new
+// key of sequence s is new_keys[s]; the step appends it at position seqlens[s] and the
+// query of row s sits there.
+struct DcAppend {
+  uint16_t *kc;              // the key cache (written: the new row)
+  float *reps;               // the representatives (written: the new key's block)
+  int32_t *seqlens;          // live lengths (written: + 1)
+  const uint16_t *new_keys;  // [num_seqs, 64]
+};
+
+__device__ void decode_select_body(DcSmem &sm, const DcAppend &ap, const uint16_t *__restrict__ q,
+                                   const uint16_t *__restrict__ k, const float *__restrict__ reps,
+                                   const int32_t *__restrict__ cu_q,
+                                   const int32_t *__restrict__ cu_k,
+                                   const int32_t *__restrict__ seqlens,
+                                   const int32_t *__restrict__ m_seq, int S, int m_max, int topk,
+                                   int emax, int32_t *__restrict__ out_idx,
+                                   float *__restrict__ out_scores,
+                                   int32_t *__restrict__ out_blocks, int *status) {
   cg::cluster_group cl = cg::this_cluster();
   const int me = (int)cl.block_rank();
   const int row = blockIdx.x / DC_CTAS;
@@ -143,7 +148,32 @@ decode_select_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict_
   // row in one memory round trip, the sequence's region in a second); nothing below
   // this early exit has touched another CTA's shared memory
   QueryInfo qi;
-  if (S <= DC_LOC_MAX) {
+  if (ap.new_keys) {
+    // fused step: row s is sequence s, whose query sits at the position of its new key
+    if (tid < D / 8) sm.qrow[tid] = __ldg(reinterpret_cast<const uint4 *>(q + (size_t)row * D) + tid);
+    if (tid == 0) {
+      sm.seqinfo[1] = cu_k[row];
+      sm.seqinfo[2] = cu_k[row + 1];
+      sm.seqinfo[3] = ap.seqlens[row];
+    }
+    __syncthreads();
+    const int k0 = sm.seqinfo[1], k1 = sm.seqinfo[2], len0 = sm.seqinfo[3];
+    qi.seq = row;
+    qi.kbase = k0;
+    qi.len = len0 + 1;
+    qi.pos = len0;
+    qi.ok = true;
+    if (k0 % BLK != 0) {
+      if (me == 0 && tid == 0) raise_status(status, HISA_ERR_UNALIGNED);
+      qi.ok = false;
+    } else if (len0 < 0 || len0 > k1 - k0) {
+      if (me == 0 && tid == 0) raise_status(status, HISA_ERR_INVALID_ARG);
+      qi.ok = false;
+    } else if (len0 + 1 > k1 - k0) {
+      if (me == 0 && tid == 0) raise_status(status, HISA_ERR_CAPACITY);
+      qi.ok = false;
+    }
+  } else if (S <= DC_LOC_MAX) {
     for (int i = tid; i <= S; i += DC_THREADS) sm.cuq[i] = __ldg(cu_q + i);
     if (tid < D / 8) sm.qrow[tid] = __ldg(reinterpret_cast<const uint4 *>(q + (size_t)row * D) + tid);
     if (tid == 0) sm.seqinfo[0] = -1;
@@ -258,11 +288,19 @@ decode_select_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict_
     }
     __syncthreads();
     static_assert(sizeof(sm.u2) >= LIN_BLK_SCRATCH_MAX, "top-m scratch fits the staging area");
-    if (!cta_select_blocks_lin<DC_THREADS>(sm.u1.allkeys, E, own, m, sm.blocks,
-                                           me == 0 ? ob : nullptr, sm.whist, sm.warp_tot,
-                                           sm.bsc, reinterpret_cast<uint8_t *>(&sm.u2)))
+    if (E <= DC_WARP_TOPM_E) {
+      // few blocks: one warp selects (radix digits over a per-warp histogram, no CTA
+      // barrier between the rounds) while the others wait once
+      if (warp == 0)
+        warp_select_blocks(sm.u1.allkeys, E, own, m, sm.blocks, me == 0 ? ob : nullptr, sm.whist,
+                           false);
+      __syncthreads();
+    } else if (!cta_select_blocks_lin<DC_THREADS>(sm.u1.allkeys, E, own, m, sm.blocks,
+                                                  me == 0 ? ob : nullptr, sm.whist, sm.warp_tot,
+                                                  sm.bsc, reinterpret_cast<uint8_t *>(&sm.u2))) {
       cta_select_blocks<DC_THREADS>(sm.u1.allkeys, E, own, m, sm.blocks,
                                     me == 0 ? ob : nullptr, sm.whist, sm.warp_tot, sm.bsc);
+    }
   } else {
     for (int i = tid; i < m; i += DC_THREADS) {
       const int v = i < E ? i : -1;
@@ -308,7 +346,11 @@ decode_select_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict_
           const int j = sm.blocks[me * bp + (lk >> 7)] * BLK + (lk & 127);
           live[p] = j <= qi.pos;
           if (live[p]) {
-            const uint4 *kr = reinterpret_cast<const uint4 *>(kseq + (size_t)j * D) + quarter * 2;
+            // a fused step's new key is read from the step's input (the cache row is
+            // written at the end of the step)
+            const uint16_t *krow = (ap.new_keys && j == qi.pos) ? ap.new_keys + (size_t)row * D
+                                                                : kseq + (size_t)j * D;
+            const uint4 *kr = reinterpret_cast<const uint4 *>(krow) + quarter * 2;
             a[p] = __ldg(kr);
             b[p] = __ldg(kr + 1);
           }
@@ -534,6 +576,61 @@ decode_select_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict_
   for (int r = kp + me * DC_THREADS + tid; r < topk; r += DC_CTAS * DC_THREADS) pad(r);
 }
 
+// The append of a fused step, by CTA 0 of the row's cluster once its selection is done
+// (every CTA of the cluster read the old length long before): the new key row is
+// written, the block that receives it is summed again in increasing row order exactly
+// like the pooling kernels (bit-identical to a fresh pool), and the length grows by one.
+__device__ void decode_append_tail(DcSmem &sm, const DcAppend &ap, const int32_t *cu_k, int s) {
+  const int tid = threadIdx.x;
+  __syncthreads();
+  const int k0 = cu_k[s], k1 = cu_k[s + 1];
+  const int len0 = ap.seqlens[s];
+  if (k0 % BLK != 0 || len0 < 0 || len0 + 1 > k1 - k0) return;  // reported by the body
+  const int b = len0 / BLK, count = len0 - b * BLK + 1;
+  const uint4 *src = reinterpret_cast<const uint4 *>(ap.new_keys + (size_t)s * D);
+  uint4 *rows = reinterpret_cast<uint4 *>(ap.kc + (size_t)k0 * D);
+  uint4 *stage = reinterpret_cast<uint4 *>(&sm.u2);  // 16 KB: the block's rows
+  for (int i = tid; i < count * 8; i += DC_THREADS) {
+    const int r = b * BLK + (i >> 3);
+    stage[i] = r < len0 ? rows[(size_t)r * 8 + (i & 7)] : src[i & 7];
+  }
+  if (tid < 8) rows[(size_t)len0 * 8 + tid] = src[tid];
+  __syncthreads();
+  if (tid < 32) {
+    const uint32_t *w = reinterpret_cast<const uint32_t *>(stage);
+    float a = 0.f, c = 0.f;
+    for (int t = 0; t < count; t++) {
+      const uint32_t x = w[t * 32 + tid];
+      a += bf_lo(x);
+      c += bf_hi(x);
+    }
+    const float cnt = (float)count;
+    reinterpret_cast<float2 *>(ap.reps + (size_t)(k0 / BLK + b) * D)[tid] =
+        make_float2(__fdiv_rn(a, cnt), __fdiv_rn(c, cnt));
+  }
+  if (tid == 0) ap.seqlens[s] = len0 + 1;
+}
+
+__global__ void __cluster_dims__(DC_CTAS, 1, 1) __launch_bounds__(DC_THREADS, 1)
+decode_select_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ k,
+                     const float *__restrict__ reps, const int32_t *__restrict__ cu_q,
+                     const int32_t *__restrict__ cu_k, const int32_t *__restrict__ seqlens,
+                     const int32_t *__restrict__ m_seq, int S, int m_max, int topk, int emax,
+                     int32_t *__restrict__ out_idx, float *__restrict__ out_scores,
+                     int32_t *__restrict__ out_blocks, DcAppend ap, int *status) {
+  extern __shared__ __align__(16) uint8_t dc_raw[];
+  DcSmem &sm = *reinterpret_cast<DcSmem *>(dc_raw);
+  // Launched as a programmatic dependent of the previous kernel on the stream (when
+  // the stream allows it): nothing is read before that kernel has completed, and the
+  // next kernel may begin launching at once (it waits the same way).
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  decode_select_body(sm, ap, q, k, reps, cu_q, cu_k, seqlens, m_seq, S, m_max, topk, emax,
+                     out_idx, out_scores, out_blocks, status);
+  if (ap.new_keys && cg::this_cluster().block_rank() == 0)
+    decode_append_tail(sm, ap, cu_k, blockIdx.x / DC_CTAS);
+}
+
 // The cluster path covers every query whose eligible blocks fit DC_MAX_E and whose
 // block budget fits DC_MAX_M.
 bool decode_path_fits(int max_seqlen_k, int m) {
@@ -545,17 +642,20 @@ cudaError_t launch_decode_select(const uint16_t *q, const uint16_t *k, const flo
                                  const int32_t *seqlens, const int32_t *m_seq, int S,
                                  int total_q, int max_seqlen_k, int m, int topk,
                                  int32_t *out_idx, float *out_scores, int32_t *out_blocks,
-                                 int *status, cudaStream_t st) {
+                                 int *status, cudaStream_t st, uint16_t *append_kc,
+                                 float *append_reps, int32_t *append_seqlens,
+                                 const uint16_t *new_keys) {
   if (total_q == 0) return cudaSuccess;
   static std::atomic<int> attr[64];
   cudaError_t e = set_smem_once((const void *)decode_select_kernel, sizeof(DcSmem), attr);
   if (e != cudaSuccess) return e;
   const int emax = (max_seqlen_k + BLK - 1) / BLK;
+  const DcAppend ap{append_kc, append_reps, append_seqlens, new_keys};
   {
     ProfScope ps(K_DECODE_SELECT, st);
     e = launch_pdl((const void *)decode_select_kernel, dim3(total_q * DC_CTAS), dim3(DC_THREADS),
                    sizeof(DcSmem), st, q, k, reps, cu_q, cu_k, seqlens, m_seq, S, m, topk,
-                   emax > 0 ? emax : 1, out_idx, out_scores, out_blocks, status);
+                   emax > 0 ? emax : 1, out_idx, out_scores, out_blocks, ap, status);
   }
   if (e != cudaSuccess) return e;
   return cudaGetLastError();

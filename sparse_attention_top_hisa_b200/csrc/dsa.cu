@@ -26,7 +26,7 @@ namespace hisa {
 constexpr int DSA_Q = 128;   // queries per filter CTA
 constexpr int DSA_SEL_THREADS = 256;
 constexpr int DSA_SEL_KPT = 16;  // candidate lists hold at most 256 * 16 keys
-constexpr int DSA_FB_CTAS = 16;
+constexpr int DSA_FB_CTAS = 64;
 
 __global__ void __launch_bounds__(256)
 key_norm_kernel(const uint16_t *__restrict__ k, const int32_t *__restrict__ cu_k,
@@ -119,30 +119,45 @@ dsa_fallback_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__
   int *tmp_c = reinterpret_cast<int *>(smem + (size_t)12 * topk);
   SelectShared &sh = *reinterpret_cast<SelectShared *>(smem + (size_t)16 * topk);
   uint32_t *keys = scratch + (size_t)blockIdx.x * scratch_stride;
-  for (int local = blockIdx.x; local < nrows; local += gridDim.x) {
-    if (cnt[local] <= cap) continue;
-    const int row = row0 + local;
-    const QueryInfo qi = locate(cu_q, cu_k, seqlens, S, row, nullptr);
-    if (!qi.ok) continue;
-    if ((size_t)qi.pos + 1 > scratch_stride) {  // max_seqlen_k understated by the caller
-      if (threadIdx.x == 0) raise_status(status, HISA_ERR_INVALID_ARG);
-      continue;
-    }
-    QRegs qr;
-    load_q(qr, q + (size_t)row * D);
-    const uint4 *kseq = reinterpret_cast<const uint4 *>(k + (size_t)qi.kbase * D);
-    for (int j = threadIdx.x; j <= qi.pos; j += DSA_SEL_THREADS) {
-      uint4 w[8];
-#pragma unroll
-      for (int c = 0; c < 8; c++) w[c] = __ldg(kseq + (size_t)j * 8 + c);
-      keys[j] = score_key(token_score(qr, w));
+  __shared__ int ovf[DSA_SEL_THREADS];
+  __shared__ int novf;
+  // rows are checked DSA_SEL_THREADS at a time (one per thread) and the overflowing
+  // ones, usually none, are then taken one after another by the whole CTA
+  for (int base = blockIdx.x * DSA_SEL_THREADS; base < nrows;
+       base += gridDim.x * DSA_SEL_THREADS) {
+    if (threadIdx.x == 0) novf = 0;
+    __syncthreads();
+    {
+      const int local = base + threadIdx.x;
+      if (local < nrows && cnt[local] > cap) ovf[atomicAdd(&novf, 1)] = local;
     }
     __syncthreads();
-    int32_t *oi = out_idx + (size_t)row * topk;
-    float *os = out_scores ? out_scores + (size_t)row * topk : nullptr;
-    select_topk<DSA_SEL_THREADS>([&](int c) { return keys[c]; }, qi.pos + 1, topk, sh, sel_key,
-                                 sel_c, tmp_key, tmp_c,
-                                 DirectOut{oi, os}, DsaPad{oi, os});
+    const int nov = novf;
+    for (int e = 0; e < nov; e++) {
+      const int local = ovf[e];
+      const int row = row0 + local;
+      const QueryInfo qi = locate(cu_q, cu_k, seqlens, S, row, nullptr);
+      if (!qi.ok) continue;  // uniform: every thread sees the same row
+      if ((size_t)qi.pos + 1 > scratch_stride) {  // max_seqlen_k understated by the caller
+        if (threadIdx.x == 0) raise_status(status, HISA_ERR_INVALID_ARG);
+        continue;
+      }
+      QRegs qr;
+      load_q(qr, q + (size_t)row * D);
+      const uint4 *kseq = reinterpret_cast<const uint4 *>(k + (size_t)qi.kbase * D);
+      for (int j = threadIdx.x; j <= qi.pos; j += DSA_SEL_THREADS) {
+        uint4 w[8];
+#pragma unroll
+        for (int c = 0; c < 8; c++) w[c] = __ldg(kseq + (size_t)j * 8 + c);
+        keys[j] = score_key(token_score(qr, w));
+      }
+      __syncthreads();
+      int32_t *oi = out_idx + (size_t)row * topk;
+      float *os = out_scores ? out_scores + (size_t)row * topk : nullptr;
+      select_topk<DSA_SEL_THREADS>([&](int c) { return keys[c]; }, qi.pos + 1, topk, sh, sel_key,
+                                   sel_c, tmp_key, tmp_c, DirectOut{oi, os}, DsaPad{oi, os});
+    }
+    __syncthreads();
   }
 }
 

@@ -6,10 +6,12 @@
 // a 128 x 128 fp32 TMEM accumulator whose lane i is query i.  Thread i of the CTA owns
 // query i, so the per-query state of the two-pass filter stays in the thread:
 //   pass 1: every score of the query is counted in one of DSA_TC_NB buckets linear over
-//           [-R, R] (R = |q| |k|max, so every score falls inside); b* is the bucket
-//           holding the k-th best score;
-//   pass 2: the scores are recomputed and every candidate in a bucket <= b* is appended,
-//           in token order, to the query's candidate list (a superset of its top-k).
+//           [-R, R] (R = |q| |k|max, so every score falls inside), or over [0, R] for a
+//           query with more than 4k candidates; b* is the bucket holding the k-th best
+//           score;
+//   pass 2: the scores are recomputed and every score above a threshold just under the
+//           lower edge of b* is appended, in token order, to the query's candidate list
+//           (a superset of its top-k).
 // Warp-specialised: a producer warp streams the key blocks through a two-stage
 // TMA ring (a sequence's partial last block comes by guarded cp.async) and issues
 // the MMAs into two TMEM accumulators; four epilogue warps drain them.  Full/empty
@@ -42,7 +44,7 @@ __device__ __forceinline__ int dsa_bucket(float s, float R, float inv) {
   return min(max(b, 0), DSA_TC_NB - 1);
 }
 
-__global__ void __launch_bounds__(DSA_TC_THREADS, 1)
+__global__ void __launch_bounds__(DSA_TC_THREADS, 2)
 dsa_filter_tc_kernel(const __grid_constant__ CUtensorMap qmap,
                      const __grid_constant__ CUtensorMap kmap, const uint16_t *__restrict__ k,
                      const int32_t *__restrict__ cu_q, const int32_t *__restrict__ cu_k,
@@ -179,10 +181,19 @@ dsa_filter_tc_kernel(const __grid_constant__ CUtensorMap qmap,
         }
       }
       R = sqrtf(qq) * __ldg(kmax + s) * (1.0f + 1.0f / 1024.0f);
-      inv = R > 0.f ? (float)DSA_TC_NB / (2.0f * R) : 0.f;
     }
     const int pos = len - qlen + (row - q0);
+    if (active) {
+      // A query with more than 4k candidates keeps under a quarter of them, so for a
+      // score distribution symmetric about 0 its k-th best score is well above 0: the
+      // buckets then cover [0, R] (twice as fine) and lower scores share the last one.
+      // A k-th score below 0 only makes that last bucket the boundary one: every
+      // candidate is kept, the list overflows and the exact fallback takes the row.
+      const float lo = pos + 1 > 4 * topk ? 0.f : -R;
+      inv = R > 0.f ? (float)DSA_TC_NB / (R - lo) : 0.f;
+    }
     int bstar = DSA_TC_NB - 1, count = 0;
+    float thr = -__int_as_float(0x7f800000);  // pass 2 keeps the scores >= thr
     float *bk = buf_key + (size_t)(row - row0) * cap;
     int32_t *bj = buf_j + (size_t)(row - row0) * cap;
     for (int it = 0; it < steps; it++) {
@@ -200,6 +211,11 @@ dsa_filter_tc_kernel(const __grid_constant__ CUtensorMap qmap,
             break;
           }
         }
+        // every score of buckets 0..b* is above R - (b* + 1) / inv; the threshold sits a
+        // little lower, so that rounding can only add candidates (the select is exact
+        // over any superset of the top-k)
+        if (bstar < DSA_TC_NB - 1 && inv > 0.f)
+          thr = R - (float)(bstar + 1) / inv - R * (1.0f / 65536.0f);
       }
       const int jmax = active ? pos - b * BLK : -1;  // keys 0..jmax of this block are causal
       for (int c0 = 0; c0 < BLK; c0 += 16) {
@@ -214,7 +230,7 @@ dsa_filter_tc_kernel(const __grid_constant__ CUtensorMap qmap,
 #pragma unroll
             for (int u = 0; u < 16; u++) {
               const float sc = __uint_as_float(v[u]);
-              if (dsa_bucket(sc, R, inv) <= bstar) {
+              if (sc >= thr) {
                 if (count < cap) {
                   bk[count] = sc;
                   bj[count] = b * BLK + c0 + u;
@@ -231,7 +247,7 @@ dsa_filter_tc_kernel(const __grid_constant__ CUtensorMap qmap,
               const int bb = dsa_bucket(sc, R, inv);
               if (!pass2) {
                 atomicAdd(&hist[bb], 1u);
-              } else if (bb <= bstar) {
+              } else if (sc >= thr) {
                 if (count < cap) {
                   bk[count] = sc;
                   bj[count] = b * BLK + c0 + u;

@@ -245,8 +245,9 @@ namespace hisa {
 //     their bucket's slots; each bucket's cursor then marks its end, which is the
 //     next bucket's start;
 //  5. every survivor counts the members of its own bucket that beat it (score desc,
-//     candidate asc); its bucket start plus that count is its output slot, and the
-//     slots below kp are kept (b* keeps its best kp - start(b*));
+//     then output index asc, so candidates need not come in index order); its bucket
+//     start plus that count is its output slot, and the slots below kp are kept (b*
+//     keeps its best kp - start(b*));
 //  6. the staged row (token index, score) is written with coalesced stores.
 // Every step is predicated rather than branched, so that a warp's candidates share
 // one instruction stream.  A b* with more members than fit past the k-th slot
@@ -525,9 +526,14 @@ __device__ void select_topk_lin(const Cands &cs, float mx, float mn, const Src &
       const int b = map(x);
       const int st = b ? (int)off[sl_slot(b - 1)] : 0, en = (int)off[sl_slot(b)];
       int r = st;
+      int tk = -1;  // this candidate's output index, looked up only for an equal score
       for (int t = st; t < en; t++) {
         const float y = sv_s[t];
-        r += (y > x) || (y == x && (int)sv_c[t] < c);
+        if (y == x && t != p) {
+          if (tk < 0) tk = tok(c);
+          r += tok((int)sv_c[t]) < tk;
+        }
+        r += y > x;
       }
       if (r < kp) {
         st_j[r] = tok(c);
@@ -565,248 +571,210 @@ __device__ void select_topk_lin(const Cands &cs, float mx, float mn, const Src &
 namespace hisa {
 
 // ---------------------------------------------------------------------------
-// Exact top-k of a row made of whole 128-score segments (the token stage: one segment
-// per selected block), candidates in registers.
+// Exact top-k through linear score buckets, candidates held in registers (the
+// token stage).
 //
-// The steps of select_topk_lin, shaped for this row layout:
-//  * register group j of warp w is segment j * NT/32 + w (four scores per lane), so
-//    the segment lookups and the "is this the query's own block" test are uniform
-//    across the warp;
-//  * the number of candidates is known from the block list (the caller passes it),
-//    so the buckets need not count every candidate: the buckets cover
-//    [hi - span, hi] with span = (hi - lo) * min(1, 2.4 k / n) -- with k a quarter of
-//    n the k-th best score lies well inside it for bell-shaped rows, so the buckets
-//    are about twice as fine where the output is -- and only scores inside the span
-//    are counted; the last bucket takes the rest (its count is the remainder) and
-//    -inf is never counted.  Exactness never depends on the span: a k-th score below
-//    it only makes the last bucket the boundary one, whose members then all survive
-//    (or, past the survivor space, take the radix route);
-//  * survivors are scattered as (score, token) pairs, so that ranking needs no
-//    lookup, and each counts the higher scores of its bucket four at a time (the
-//    survivor array is followed by -inf pads, and later buckets only hold lower
-//    scores, so reading past the bucket's end never changes a count); equal scores
-//    compare tokens (blocks are ascending, so token order is candidate order).
-constexpr int SG_BINS = 4096;
-constexpr int SG_LAST = SG_BINS - 1;   // scores below the span (and the remainder count)
-constexpr int SG_WORDS = SG_BINS + 4;  // + the -inf bin, rounded to 16 bytes
+// Input: n raw fp32 scores in candidate (= token) order, -inf marking a position
+// that is not a candidate (finite scores are the contract).  Each of the NT threads
+// loads KPT of them once (coalesced 16-byte loads; candidate c = ((i/4)*NT +
+// thread)*4 + i%4) and keeps them in registers.  Then:
+// 1. max/min and count of the candidate scores (fused with the load);
+// 2. histogram over LIN_BINS buckets linear in the score between max and min
+//    (bucket 0 holds the highest scores).  The bucket map is monotone in the score,
+//    so bucket order is score order;
+// 3. one scan gives every bucket its output offset and finds the bucket b* that
+//    holds the k-th best score;
+// 4. candidates in buckets before b* are scattered to their bucket's output range,
+//    those in b* are gathered apart, each as a 64-bit (key, ~index) composite whose
+//    unsigned order is the output order (score desc, index asc);
+// 5. the b* candidates are ranked exactly and the best k - |buckets before b*| of
+//    them fill the end of the output;
+// 6. every other survivor is ranked within its own bucket (a handful of elements for
+//    continuous scores) and written to its final slot.
+// A boundary bucket with more than k members (heavy ties) sends the query through
+// the radix routine above instead, reading the scores again.
 
-struct SgShared {
+constexpr int LIN_BINS = 2048;
+// Bucket b lives at word b + b / 32 of the count arrays: a thread scanning eight
+// consecutive buckets then touches 32 distinct banks across its warp.
+constexpr int LIN_WORDS = LIN_BINS + LIN_BINS / 32;
+__device__ __forceinline__ int lin_slot(int b) { return b + (b >> 5); }
+
+struct LinShared {
   union {
     SelectShared radix;
     struct {
-      uint32_t off[SG_WORDS];  // counts, then first slots, then (after the scatter) ends
+      uint32_t cnt[LIN_WORDS];
+      uint32_t off[LIN_WORDS];
       int warp_tot[33];
+      int wn[32];
       float wmx[32], wmn[32];
-      int misc[4];
+      uint32_t misc[8];
     } lin;
   };
 };
 
-// Working bytes: staged indices int32[k] | staged scores f32[k] | survivors
-// (f32 score, i32 token)[cap + 4]; the radix route reuses them as its four lists.
-__host__ __device__ inline int sg_cap(int k) { return (k + SL_SLACK + 7) & ~7; }
-__host__ __device__ inline size_t sg_work_bytes(int k) {
-  const size_t a = (size_t)8 * k + (size_t)8 * (sg_cap(k) + 4);
-  const size_t b = (size_t)16 * k;
-  return ((a > b ? a : b) + 15) & ~(size_t)15;
+__device__ __forceinline__ int lin_bucket(float s, float smax, float inv) {
+  const int b = __float2int_rz((smax - s) * inv);
+  return min(max(b, 0), LIN_BINS - 1);
 }
 
-// bucket(x) = min(round((hi - x) * inv), SG_LAST) for a finite x <= hi, and SG_BINS
-// for -inf: the sum of the multiply-add is then +inf (or NaN when inv = 0), whose bit
-// pattern lies at least 2^29 above that of 2^23 while every finite sum lies far below,
-// so bit 29 of the difference separates the two.
-struct SgMap {
-  float hi, inv;
-  __device__ __forceinline__ int operator()(float x) const {
-    const float t = fmaf(hi - x, inv, 8388608.0f);
-    const uint32_t u = (uint32_t)__float_as_int(t) - 0x4B000000u;
-    return (int)min(u, (uint32_t)SG_LAST) + (int)(u >> 29);
-  }
-};
-
-// f: KPT scores per thread (group j of warp w = segment j * NW + w; lane l holds its
-// scores 4l..4l+3), -inf past the row.  nseg: segments in the row (only the last may
-// hold -inf); nvalid: its finite scores.  seg_base(s): the first score of segment s
-// in memory (the radix route reads the row again); seg_tok[s]: the token of its first
-// score (shared memory).  k >= 1; nseg * 128 <= 65536.
-template <int NT, int KPT, class SegBase>
-__device__ void select_topk_seg(const float (&f)[KPT], int nseg, int nvalid, int k, SgShared &sh,
-                                uint8_t *work, SegBase seg_base, const int32_t *seg_tok,
-                                int32_t *out_idx, float *out_scores) {
-  static_assert(SG_BINS % NT == 0 && NT % 32 == 0 && KPT % 4 == 0, "layout");
-  constexpr int NW = NT / 32;
-  constexpr int PER = SG_BINS / NT;
+// sc: the n raw scores (RowScores or SegScores; four consecutive candidates never
+// straddle a segment).  work: 4*k words (2*k uint64) of shared scratch.
+template <int NT, int KPT, class Src, class Out, class Pad>
+__device__ void select_topk_reg(Src sc, int n, int k, LinShared &sh, uint32_t *work, Out out,
+                                Pad pad) {
+  static_assert(KPT % 4 == 0, "scores are loaded four at a time");
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const float NEG = neg_inf();
-  const int n = nseg * 128;
-  int32_t *st_j = reinterpret_cast<int32_t *>(work);
-  float *st_s = reinterpret_cast<float *>(work + (size_t)4 * k);
-  const int cap = sg_cap(k);
-  float2 *sv = reinterpret_cast<float2 *>(work + (size_t)8 * k);  // (score, token bits)
-  uint32_t *off = sh.lin.off;
+  constexpr int NW = NT / 32;
+  uint64_t *surv = reinterpret_cast<uint64_t *>(work);      // k survivors
+  uint64_t *bnd = reinterpret_cast<uint64_t *>(work) + k;   // up to k boundary members
+  const float NEG = -__int_as_float(0x7f800000);             // -inf
 
-  // 1. max and min (only the own block, the last segment, can hold -inf)
+  float f[KPT];
   float mx = NEG, mn = -NEG;
+  int nv = 0;
 #pragma unroll
   for (int j = 0; j < KPT / 4; j++) {
-    const int s = j * NW + warp;
+    const int c0 = (j * NT + tid) * 4;
+    float4 v = make_float4(NEG, NEG, NEG, NEG);
+    if (c0 + 3 < n) {
+      v = sc.ld4(c0);
+    } else if (c0 < n) {
+      v.x = sc.ld1(c0);
+      if (c0 + 1 < n) v.y = sc.ld1(c0 + 1);
+      if (c0 + 2 < n) v.z = sc.ld1(c0 + 2);
+    }
+    f[4 * j] = v.x;
+    f[4 * j + 1] = v.y;
+    f[4 * j + 2] = v.z;
+    f[4 * j + 3] = v.w;
 #pragma unroll
-    for (int e = 0; e < 4; e++) mx = fmaxf(mx, f[4 * j + e]);
-    if (s < nseg - 1) {
-#pragma unroll
-      for (int e = 0; e < 4; e++) mn = fminf(mn, f[4 * j + e]);
-    } else if (s == nseg - 1) {
-#pragma unroll
-      for (int e = 0; e < 4; e++)
-        if (f[4 * j + e] != NEG) mn = fminf(mn, f[4 * j + e]);
+    for (int e = 0; e < 4; e++) {
+      const float x = f[4 * j + e];
+      if (x != NEG) {
+        mx = fmaxf(mx, x);
+        mn = fminf(mn, x);
+        nv++;
+      }
     }
   }
+  auto cand = [&](int i) { return ((i >> 2) * NT + tid) * 4 + (i & 3); };
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    nv += __shfl_xor_sync(0xffffffffu, nv, o);
   }
   if (lane == 0) {
     sh.lin.wmx[warp] = mx;
     sh.lin.wmn[warp] = mn;
+    sh.lin.wn[warp] = nv;
   }
-  for (int i = tid; i < SG_WORDS / 4; i += NT)
-    reinterpret_cast<uint4 *>(off)[i] = make_uint4(0u, 0u, 0u, 0u);
-  if (tid == 0) {
-    sh.lin.misc[0] = -1;
-    sh.lin.misc[1] = 0;
-    sh.lin.misc[2] = 0;
-  }
+  for (int i = tid; i < LIN_WORDS; i += NT) sh.lin.cnt[i] = 0u;
   __syncthreads();
   mx = NEG;
   mn = -NEG;
+  nv = 0;
 #pragma unroll
   for (int w = 0; w < NW; w++) {
     mx = fmaxf(mx, sh.lin.wmx[w]);
     mn = fminf(mn, sh.lin.wmn[w]);
+    nv += sh.lin.wn[w];
   }
-  const float frac = fminf(1.f, 2.4f * (float)k / (float)n);
-  const float span = (mx - mn) * frac;
-  const SgMap map{mx, (mn < mx && span > 0.f) ? (float)SG_LAST / span : 0.f};
+  const int nvalid = nv;
+  const float smax = mx;
+  const float range = mx - mn;
+  const float inv = (nvalid > 0 && range > 0.f) ? (float)LIN_BINS / range : 0.f;
 
-  // 2. histogram of the scores inside the span
+  // 2. histogram
 #pragma unroll
-  for (int i = 0; i < KPT; i++) {
-    const int b = map(f[i]);
-    if (b < SG_LAST) atomicAdd(&off[b], 1u);
-  }
+  for (int i = 0; i < KPT; i++)
+    if (f[i] != NEG) atomicAdd(&sh.lin.cnt[lin_slot(lin_bucket(f[i], smax, inv))], 1u);
   __syncthreads();
 
-  // 3. first slots and b* (thread t owns buckets PER t .. PER t + PER - 1, read four at
-  // a time; the last bucket's count is what the others leave of nvalid)
+  // 3. offsets and the boundary bucket
   const int kp = min(k, nvalid);
   {
-    uint4 *off4 = reinterpret_cast<uint4 *>(off) + tid * (PER / 4);
+    constexpr int per = LIN_BINS / NT;
+    uint32_t h[per];
     int local = 0;
 #pragma unroll
-    for (int i = 0; i < PER / 4; i++) {
-      const uint4 v = off4[i];
-      local += (int)(v.x + v.y + v.z + v.w);
+    for (int i = 0; i < per; i++) {
+      h[i] = sh.lin.cnt[lin_slot(tid * per + i)];
+      local += (int)h[i];
     }
     int total;
     int run = block_exclusive_scan<NT>(local, sh.lin.warp_tot, &total);
+    if (tid == 0) {
+      sh.lin.misc[3] = LIN_BINS;  // no boundary bucket when every candidate survives
+      sh.lin.misc[4] = (uint32_t)kp;
+      sh.lin.misc[5] = 0u;        // boundary fill counter
+    }
+    __syncthreads();
 #pragma unroll
-    for (int i = 0; i < PER / 4; i++) {
-      const uint4 v = off4[i];
-      uint32_t h[4] = {v.x, v.y, v.z, v.w};
-      if (tid == NT - 1 && i == PER / 4 - 1) h[3] = (uint32_t)(nvalid - total);
-      uint32_t o[4];
-#pragma unroll
-      for (int e = 0; e < 4; e++) {
-        if (run < kp && run + (int)h[e] >= kp) {
-          sh.lin.misc[0] = tid * PER + 4 * i + e;
-          sh.lin.misc[1] = run;
-          sh.lin.misc[2] = (int)h[e];
-        }
-        o[e] = (uint32_t)run;
-        run += (int)h[e];
+    for (int i = 0; i < per; i++) {
+      const int b = tid * per + i;
+      if (nvalid > k && run < k && run + (int)h[i] >= k) {
+        sh.lin.misc[3] = (uint32_t)b;
+        sh.lin.misc[4] = (uint32_t)run;
       }
-      off4[i] = make_uint4(o[0], o[1], o[2], o[3]);
+      sh.lin.off[lin_slot(b)] = (uint32_t)run;
+      sh.lin.cnt[lin_slot(b)] = (uint32_t)run;  // becomes the scatter cursor
+      run += (int)h[i];
     }
   }
   __syncthreads();
-  const int bstar = sh.lin.misc[0];
-  const int nsurv = bstar >= 0 ? sh.lin.misc[1] + sh.lin.misc[2] : 0;
+  const int bstar = (int)sh.lin.misc[3];
+  const int above = (int)sh.lin.misc[4];  // survivors in buckets before b*
+  const int need = kp - above;             // survivors taken from b*
 
-  if (nsurv > cap) {
-    // heavy ties at the boundary: the radix route (its lists reuse the working bytes)
+  // 4. scatter
+#pragma unroll
+  for (int i = 0; i < KPT; i++) {
+    if (f[i] != NEG) {
+      const int b = lin_bucket(f[i], smax, inv);
+      if (b < bstar) {
+        const uint32_t slot = atomicAdd(&sh.lin.cnt[lin_slot(b)], 1u);
+        surv[slot] = rank_key(f[i], cand(i));
+      } else if (b == bstar) {
+        const uint32_t e = atomicAdd(&sh.lin.misc[5], 1u);
+        if (e < (uint32_t)k) bnd[e] = rank_key(f[i], cand(i));
+      }
+    }
+  }
+  __syncthreads();
+  const int nbnd = (int)sh.lin.misc[5];
+  if (nbnd > k) {  // heavy ties at the boundary: exact radix route
     __syncthreads();
     auto key = [&](int c) -> uint32_t {
-      const float x = seg_base(c >> 7)[c & 127];
+      const float x = sc.ld1(c);
       return x != NEG ? score_key(x) : 0u;
     };
-    auto tok = [&](int c) { return seg_tok[c >> 7] + (c & 127); };
-    select_topk<NT>(key, n, k, sh.radix, reinterpret_cast<uint32_t *>(work),
-                    reinterpret_cast<int *>(work + (size_t)4 * k),
-                    reinterpret_cast<uint32_t *>(work + (size_t)8 * k),
-                    reinterpret_cast<int *>(work + (size_t)12 * k),
-                    StageOut<decltype(tok)>{st_j, st_s, tok}, StagePad{st_j, st_s});
-  } else {
-    // 4. scatter the survivors (buckets 0..b*) as (score, token) to their buckets
-#pragma unroll
-    for (int j = 0; j < KPT / 4; j++) {
-      const int s = j * NW + warp;
-      const int t0 = (s < nseg ? seg_tok[s] : 0) + lane * 4;
-#pragma unroll
-      for (int e = 0; e < 4; e++) {
-        const float x = f[4 * j + e];
-        const int b = map(x);
-        if (b <= bstar) {
-          const uint32_t p = atomicAdd(&off[b], 1u);
-          if (p < (uint32_t)cap) sv[p] = make_float2(x, __int_as_float(t0 + e));
-        }
-      }
-    }
-    if (tid < 4) sv[nsurv + tid] = make_float2(NEG, 0.f);  // pads read by the last bucket
-    __syncthreads();
-    // 5. rank within the bucket; bucket b spans [end(b - 1), end(b))
-    for (int p = tid; p < nsurv; p += NT) {
-      const float2 me = sv[p];
-      const float x = me.x;
-      const int tk = __float_as_int(me.y);
-      const int b = map(x);
-      const int st = b ? (int)off[b - 1] : 0, en = (int)off[b];
-      int r = st;
-      for (int t = st; t < en; t += 4) {
-        const float2 y0 = sv[t], y1 = sv[t + 1], y2 = sv[t + 2], y3 = sv[t + 3];
-        r += (y0.x > x) + (y1.x > x) + (y2.x > x) + (y3.x > x);
-        // equal scores: the lower token first (past the bucket's end no score is equal)
-        r += (y0.x == x && __float_as_int(y0.y) < tk) + (y1.x == x && __float_as_int(y1.y) < tk) +
-             (y2.x == x && __float_as_int(y2.y) < tk) + (y3.x == x && __float_as_int(y3.y) < tk);
-      }
-      if (r < kp) {
-        st_j[r] = tk;
-        st_s[r] = x;
-      }
-    }
-    for (int r = kp + tid; r < k; r += NT) {
-      st_j[r] = -1;
-      st_s[r] = 0.f;
-    }
-    __syncthreads();
+    select_topk<NT>(key, n, k, sh.radix, work, reinterpret_cast<int *>(work + k), work + 2 * k,
+                    reinterpret_cast<int *>(work + 3 * k), out, pad);
+    return;
   }
 
-  // 6. the row, with coalesced stores
-  const bool vec = (k & 3) == 0 && (reinterpret_cast<uintptr_t>(out_idx) & 15) == 0 &&
-                   (reinterpret_cast<uintptr_t>(out_scores) & 15) == 0;
-  if (vec) {
-    const int k4 = k >> 2;
-    for (int r = tid; r < k4; r += NT) {
-      reinterpret_cast<int4 *>(out_idx)[r] = reinterpret_cast<const int4 *>(st_j)[r];
-      if (out_scores)
-        reinterpret_cast<float4 *>(out_scores)[r] = reinterpret_cast<const float4 *>(st_s)[r];
-    }
-  } else {
-    for (int r = tid; r < k; r += NT) {
-      out_idx[r] = st_j[r];
-      if (out_scores) out_scores[r] = st_s[r];
+  // 5. the boundary bucket, ranked exactly
+  if (need > 0) {
+    for (int e = tid; e < nbnd; e += NT) {
+      const uint64_t me = bnd[e];
+      int rank = 0;
+      for (int t = 0; t < nbnd; t++) rank += bnd[t] > me;
+      if (rank < need) out(above + rank, (int)~(uint32_t)me, (uint32_t)(me >> 32));
     }
   }
+  // 6. everything above the boundary, ranked within its own bucket
+  for (int s = tid; s < above; s += NT) {
+    const uint64_t me = surv[s];
+    const int b = lin_bucket(key_score((uint32_t)(me >> 32)), smax, inv);
+    const int st = (int)sh.lin.off[lin_slot(b)], en = (int)sh.lin.cnt[lin_slot(b)];
+    int rank = 0;
+    for (int t = st; t < en; t++) rank += surv[t] > me;
+    out(st + rank, (int)~(uint32_t)me, (uint32_t)(me >> 32));
+  }
+  for (int r = kp + tid; r < k; r += NT) pad(r);
   __syncthreads();
 }
 

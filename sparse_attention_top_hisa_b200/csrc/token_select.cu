@@ -78,8 +78,8 @@ struct BlockTok {
 __host__ __device__ inline size_t token_smem_bytes(int m, int topk) {
   return sl_work_bytes(topk) + sizeof(SlShared) + (size_t)m * 8;
 }
-__host__ __device__ inline size_t token_seg_smem_bytes(int m, int topk) {
-  return sg_work_bytes(topk) + sizeof(SgShared) + (size_t)m * 12;
+__host__ __device__ inline size_t token_reg_smem_bytes(int m, int topk) {
+  return (size_t)16 * topk + sizeof(LinShared) + (size_t)m * 8;
 }
 
 __global__ void __launch_bounds__(TS_THREADS)
@@ -111,9 +111,10 @@ template <int NT>
 __device__ __forceinline__ int select_row_setup(const int32_t *cu_q, const int32_t *cu_k,
                                                 const int32_t *seqlens, const int32_t *m_seq,
                                                 int S, int m, int topk, const int32_t *blk,
-                                                const int32_t *pmap, const int *launch_abort,
-                                                int row, int32_t *oi, float *os, int32_t *sblk,
-                                                int32_t *sseg, int *pos_out = nullptr) {
+                                                const int32_t *pmap, int list_base,
+                                                const int *launch_abort, int row, int32_t *oi,
+                                                float *os, int32_t *sblk, int32_t *sseg,
+                                                int *pos_out = nullptr) {
   const QueryInfo qi = locate(cu_q, cu_k, seqlens, S, row, nullptr);
   // a scoring launch that gave up a wait left its score rows incomplete: pad every row
   if (!qi.ok || (launch_abort && *launch_abort)) {
@@ -127,64 +128,62 @@ __device__ __forceinline__ int select_row_setup(const int32_t *cu_q, const int32
   const int nsel = min(seq_budget(m_seq, qi.seq, m, nullptr), qi.pos / BLK + 1);
   for (int i = threadIdx.x; i < nsel; i += NT) {
     sblk[i] = blk[(size_t)row * m + i];
-    if (pmap) sseg[i] = pmap[(size_t)row * m + i];
+    if (pmap) sseg[i] = pmap[(size_t)row * m + i] - list_base;  // segment in the chunk buffer
   }
   if (pos_out) *pos_out = qi.pos;
   __syncthreads();
   return nsel * BLK;
 }
 
-// One CTA per query: exact top-k of the query's score row, held in registers as whole
-// 128-score segments (NT * KPT >= m * 128), by select_topk_seg.  pmap non-null: the
-// segment of slot i is pmap[row * m + i] of the score buffer; else the row's
-// segments are contiguous.  MINB CTAs are meant to share an SM.
-template <int NT, int KPT, int MINB>
-__global__ void __launch_bounds__(NT, MINB)
-token_select_seg_kernel(const int32_t *__restrict__ cu_q, const int32_t *__restrict__ cu_k,
-                        const int32_t *__restrict__ seqlens, const int32_t *__restrict__ m_seq,
-                        int S, int m, int topk, const int32_t *__restrict__ blk,
-                        const float *__restrict__ scratch, const int32_t *__restrict__ pmap,
-                        const int *__restrict__ launch_abort, int32_t *__restrict__ out_idx,
-                        float *__restrict__ out_scores) {
+struct TokenOut {
+  int32_t *idx;
+  float *scores;
+  const int32_t *blkrow;
+  __device__ void operator()(int r, int c, uint32_t u) const {
+    idx[r] = blkrow[c >> 7] * BLK + (c & 127);
+    if (scores) scores[r] = key_score(u);
+  }
+};
+
+struct RowPad {
+  int32_t *idx;
+  float *scores;
+  __device__ void operator()(int r) const {
+    idx[r] = -1;
+    if (scores) scores[r] = 0.f;
+  }
+};
+
+// One CTA per query: exact top-k of the query's score row, KPT candidates per thread
+// held in registers (NT * KPT >= m * 128), by select_topk_reg.  pmap non-null: the
+// segment of slot i is pmap[row * m + i] - list_base of the score buffer; else the
+// row's segments are contiguous.
+template <int NT, int KPT>
+__global__ void __launch_bounds__(NT, 1024 / NT)
+token_select_scratch_kernel(const int32_t *__restrict__ cu_q, const int32_t *__restrict__ cu_k,
+                            const int32_t *__restrict__ seqlens, const int32_t *__restrict__ m_seq,
+                            int S, int m, int topk, const int32_t *__restrict__ blk,
+                            const float *__restrict__ scratch, const int32_t *__restrict__ pmap,
+                            int list_base, const int *__restrict__ launch_abort, int row0,
+                            int32_t *__restrict__ out_idx, float *__restrict__ out_scores) {
   extern __shared__ __align__(16) uint8_t smem[];
-  uint8_t *work = smem;
-  const size_t wb = sg_work_bytes(topk);
-  SgShared &sh = *reinterpret_cast<SgShared *>(smem + wb);
-  int32_t *sblk = reinterpret_cast<int32_t *>(smem + wb + sizeof(SgShared));
+  uint32_t *work = reinterpret_cast<uint32_t *>(smem);
+  LinShared &sh = *reinterpret_cast<LinShared *>(smem + (size_t)16 * topk);
+  int32_t *sblk = reinterpret_cast<int32_t *>(smem + (size_t)16 * topk + sizeof(LinShared));
   int32_t *sseg = sblk + m;
-  const int row = blockIdx.x;
+  const int row = row0 + blockIdx.x;
   int32_t *oi = out_idx + (size_t)row * topk;
   float *os = out_scores ? out_scores + (size_t)row * topk : nullptr;
-  int pos = 0;
   const int n = select_row_setup<NT>(cu_q, cu_k, seqlens, m_seq, S, m, topk, blk, pmap,
-                                     launch_abort, row, oi, os, sblk, sseg, &pos);
+                                     list_base, launch_abort, row, oi, os, sblk, sseg);
   if (n == 0) return;
-  const int nseg = n >> 7;
-  // the selected blocks before the own one are whole and precede the query; the own
-  // block (the last) holds its tokens up to the query's position
-  const int nvalid = (nseg - 1) * BLK + pos % BLK + 1;
-  const float *rowbase = scratch + (size_t)row * m * BLK;
-  auto seg_base = [&](int sg) -> const float * {
-    return pmap ? scratch + (size_t)sseg[sg] * BLK : rowbase + (size_t)sg * BLK;
-  };
-  constexpr int NW = NT / 32;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const float NEG = neg_inf();
-  float f[KPT];
-#pragma unroll
-  for (int j = 0; j < KPT / 4; j++) {
-    const int sg = j * NW + warp;  // uniform across the warp
-    float4 v = make_float4(NEG, NEG, NEG, NEG);
-    if (sg < nseg) v = *reinterpret_cast<const float4 *>(seg_base(sg) + lane * 4);
-    f[4 * j] = v.x;
-    f[4 * j + 1] = v.y;
-    f[4 * j + 2] = v.z;
-    f[4 * j + 3] = v.w;
-  }
-  // token of the first score of every selected block (the block list, scaled)
-  for (int i = threadIdx.x; i < nseg; i += NT) sseg[m + i] = sblk[i] * BLK;
-  __syncthreads();
-  select_topk_seg<NT, KPT>(f, nseg, nvalid, topk, sh, work, seg_base, sseg + m, oi, os);
+  const TokenOut out{oi, os, sblk};
+  const RowPad pad{oi, os};
+  if (pmap)  // scores of slot i in segment sseg[i] of the buffer
+    select_topk_reg<NT, KPT>(SegScores{scratch, sseg}, n, topk, sh, work, out, pad);
+  else       // one contiguous score row per query
+    select_topk_reg<NT, KPT>(RowScores{scratch + (size_t)row * m * BLK}, n, topk, sh, work, out,
+                             pad);
 }
 
 // The same for rows longer than the registers hold (m > 128): every pass of the
@@ -195,19 +194,19 @@ token_select_mem_kernel(const int32_t *__restrict__ cu_q, const int32_t *__restr
                         const int32_t *__restrict__ seqlens, const int32_t *__restrict__ m_seq,
                         int S, int m, int topk, const int32_t *__restrict__ blk,
                         const float *__restrict__ scratch, const int32_t *__restrict__ pmap,
-                        const int *__restrict__ launch_abort, int32_t *__restrict__ out_idx,
-                        float *__restrict__ out_scores) {
+                        int list_base, const int *__restrict__ launch_abort, int row0,
+                        int32_t *__restrict__ out_idx, float *__restrict__ out_scores) {
   extern __shared__ __align__(16) uint8_t smem[];
   uint8_t *work = smem;
   const size_t wb = sl_work_bytes(topk);
   SlShared &sh = *reinterpret_cast<SlShared *>(smem + wb);
   int32_t *sblk = reinterpret_cast<int32_t *>(smem + wb + sizeof(SlShared));
   int32_t *sseg = sblk + m;
-  const int row = blockIdx.x;
+  const int row = row0 + blockIdx.x;
   int32_t *oi = out_idx + (size_t)row * topk;
   float *os = out_scores ? out_scores + (size_t)row * topk : nullptr;
   const int n = select_row_setup<NT>(cu_q, cu_k, seqlens, m_seq, S, m, topk, blk, pmap,
-                                     launch_abort, row, oi, os, sblk, sseg);
+                                     list_base, launch_abort, row, oi, os, sblk, sseg);
   if (n == 0) return;
   float mx, mn;
   if (pmap) {
@@ -228,11 +227,6 @@ static bool token_use_split(int total_q, int num_sms) { return !use_tc_path(tota
 
 size_t tc_workspace_bytes(int total_q, int num_seqs, int max_seqlen_k, int m);
 size_t block_tc_workspace_bytes(int total_q, int num_seqs, int max_seqlen_k);
-cudaError_t launch_token_score_tc(const uint16_t *q, const uint16_t *k, const int32_t *cu_q,
-                                  const int32_t *cu_k, const int32_t *seqlens, int S,
-                                  int total_q, int max_seqlen_k, int m, const int32_t *blk,
-                                  uint8_t *ws, float **scores_out, const int32_t **pmap_out,
-                                  int **abort_out, int num_sms, int *status, cudaStream_t st);
 
 size_t token_scratch_bytes(int total_q, int num_seqs, int max_seqlen_k, int m, int num_sms) {
   if (token_use_split(total_q, num_sms)) return (size_t)total_q * m * BLK * 4;
@@ -244,21 +238,66 @@ size_t token_scratch_bytes(int total_q, int num_seqs, int max_seqlen_k, int m, i
 
 template <class Kern>
 static cudaError_t launch_select(Kern kern, int nt, size_t smem, std::atomic<int> *attr,
-                                 int total_q, cudaStream_t st, const int32_t *cu_q,
+                                 int nrows, cudaStream_t st, const int32_t *cu_q,
                                  const int32_t *cu_k, const int32_t *seqlens,
                                  const int32_t *m_seq, int S, int m, int topk,
                                  const int32_t *blk, const float *scores, const int32_t *pmap,
-                                 const int *launch_abort, int32_t *out_idx, float *out_scores) {
+                                 int list_base, const int *launch_abort, int row0,
+                                 int32_t *out_idx, float *out_scores) {
   cudaError_t e = set_smem_once((const void *)kern, smem, attr);
   if (e != cudaSuccess) return e;
   ProfScope ps(K_TOKEN_SELECT_SCRATCH, st);
-  kern<<<total_q, nt, smem, st>>>(cu_q, cu_k, seqlens, m_seq, S, m, topk, blk, scores, pmap,
-                                  launch_abort, out_idx, out_scores);
+  kern<<<nrows, nt, smem, st>>>(cu_q, cu_k, seqlens, m_seq, S, m, topk, blk, scores, pmap,
+                                list_base, launch_abort, row0, out_idx, out_scores);
   return cudaGetLastError();
 }
 
-// m is the row stride of blk (the largest block budget); m_seq (nullable) the budget
-// of each sequence.
+// The exact select of query rows [row0, row0 + nrows): m is the row stride of blk (the
+// largest block budget), m_seq (nullable) the budget of each sequence.  pmap non-null:
+// the segment of slot i of a row is pmap[row * m + i] - list_base of `scores`; else
+// every row's segments are contiguous (row stride m * 128).  split: few queries
+// (wider CTAs).
+cudaError_t launch_select_rows(const int32_t *cu_q, const int32_t *cu_k, const int32_t *seqlens,
+                               const int32_t *m_seq, int S, int m, int topk, const int32_t *blk,
+                               const float *scores, const int32_t *pmap, int list_base,
+                               const int *launch_abort, int row0, int nrows, bool split,
+                               int32_t *out_idx, float *out_scores, cudaStream_t st) {
+  if (nrows <= 0) return cudaSuccess;
+#define HISA_SELECT_ARGS nrows, st, cu_q, cu_k, seqlens, m_seq, S, m, topk, blk, scores, pmap, \
+                         list_base, launch_abort, row0, out_idx, out_scores
+  const int n = m * BLK;
+  const size_t smem_reg = token_reg_smem_bytes(m, topk);
+  if (split && n <= 1024 * 8) {  // few queries: a wider CTA per query shortens each selection
+    static std::atomic<int> attr[64];
+    return launch_select(token_select_scratch_kernel<1024, 8>, 1024, smem_reg, attr, HISA_SELECT_ARGS);
+  }
+  if (split && n <= 1024 * 16) {
+    static std::atomic<int> attr[64];
+    return launch_select(token_select_scratch_kernel<1024, 16>, 1024, smem_reg, attr, HISA_SELECT_ARGS);
+  }
+  if (n <= 256 * 32) {
+    static std::atomic<int> attr[64];
+    return launch_select(token_select_scratch_kernel<256, 32>, 256, smem_reg, attr, HISA_SELECT_ARGS);
+  }
+  if (n <= 512 * 32) {
+    static std::atomic<int> attr[64];
+    return launch_select(token_select_scratch_kernel<512, 32>, 512, smem_reg, attr, HISA_SELECT_ARGS);
+  }
+  {  // m > 128: the score row is read from memory on every pass
+    static std::atomic<int> attr[64];
+    return launch_select(token_select_mem_kernel<1024>, 1024, token_smem_bytes(m, topk), attr,
+                         HISA_SELECT_ARGS);
+  }
+#undef HISA_SELECT_ARGS
+}
+
+cudaError_t launch_token_stage_tc(const uint16_t *q, const uint16_t *k, const int32_t *cu_q,
+                                  const int32_t *cu_k, const int32_t *seqlens,
+                                  const int32_t *m_seq, int S, int total_q, int max_seqlen_k,
+                                  int m, int topk, const int32_t *blk, uint8_t *ws, int num_sms,
+                                  int32_t *out_idx, float *out_scores, int *status,
+                                  cudaStream_t st);
+
 cudaError_t launch_token_select(const uint16_t *q, const uint16_t *k, const int32_t *cu_q,
                                 const int32_t *cu_k, const int32_t *seqlens,
                                 const int32_t *m_seq, int S, int total_q, int max_seqlen_k,
@@ -266,51 +305,25 @@ cudaError_t launch_token_select(const uint16_t *q, const uint16_t *k, const int3
                                 int32_t *out_idx, float *out_scores, int *status,
                                 cudaStream_t st) {
   if (total_q == 0) return cudaSuccess;
-  cudaError_t e;
+  if (!token_use_split(total_q, num_sms))
+    return launch_token_stage_tc(q, k, cu_q, cu_k, seqlens, m_seq, S, total_q, max_seqlen_k, m,
+                                 topk, blk, ws, num_sms, out_idx, out_scores, status, st);
+  // few queries: spread each query's blocks over enough CTAs to cover the SMs about twice
   float *scores = reinterpret_cast<float *>(ws);
-  const int32_t *pmap = nullptr;  // contiguous score rows unless the tensor-core path maps them
-  int *launch_abort = nullptr;    // set by a scoring launch whose bounded wait ran out
-  const bool split = token_use_split(total_q, num_sms);
-  if (split) {
-    // spread each query's blocks over enough CTAs to cover the SMs about twice
-    int splits = (2 * num_sms + total_q - 1) / total_q;
-    splits = splits < 1 ? 1 : (splits > m ? m : splits);
-    int slots = (m + splits - 1) / splits;
-    slots = (slots + 1) & ~1;  // whole staging rounds
-    splits = (m + slots - 1) / slots;
-    {
-      ProfScope ps(K_TOKEN_SCORE_SPLIT, st);
-      token_score_split_kernel<<<dim3(total_q, splits), TS_THREADS, 0, st>>>(
-          q, k, cu_q, cu_k, seqlens, m_seq, S, m, blk, slots, scores);
-    }
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  } else {
-    e = launch_token_score_tc(q, k, cu_q, cu_k, seqlens, S, total_q, max_seqlen_k, m, blk, ws,
-                              &scores, &pmap, &launch_abort, num_sms, status, st);
-    if (e != cudaSuccess) return e;
+  int splits = (2 * num_sms + total_q - 1) / total_q;
+  splits = splits < 1 ? 1 : (splits > m ? m : splits);
+  int slots = (m + splits - 1) / splits;
+  slots = (slots + 1) & ~1;  // whole staging rounds
+  splits = (m + slots - 1) / slots;
+  {
+    ProfScope ps(K_TOKEN_SCORE_SPLIT, st);
+    token_score_split_kernel<<<dim3(total_q, splits), TS_THREADS, 0, st>>>(
+        q, k, cu_q, cu_k, seqlens, m_seq, S, m, blk, slots, scores);
   }
-  const size_t smem = token_smem_bytes(m, topk);
-#define HISA_SELECT_ARGS total_q, st, cu_q, cu_k, seqlens, m_seq, S, m, topk, blk, scores, pmap, \
-                         launch_abort, out_idx, out_scores
-  const int n = m * BLK;
-  const size_t smem_seg = token_seg_smem_bytes(m, topk);
-  if (split && n <= 1024 * 8) {  // few queries: a wider CTA per query shortens each selection
-    static std::atomic<int> attr[64];
-    return launch_select(token_select_seg_kernel<1024, 8, 1>, 1024, smem_seg, attr, HISA_SELECT_ARGS);
-  }
-  if (n <= 512 * 16) {
-    static std::atomic<int> attr[64];
-    return launch_select(token_select_seg_kernel<512, 16, 2>, 512, smem_seg, attr, HISA_SELECT_ARGS);
-  }
-  if (n <= 1024 * 16) {
-    static std::atomic<int> attr[64];
-    return launch_select(token_select_seg_kernel<1024, 16, 1>, 1024, smem_seg, attr, HISA_SELECT_ARGS);
-  }
-  {  // m > 128: the score row is read from memory on every pass
-    static std::atomic<int> attr[64];
-    return launch_select(token_select_mem_kernel<1024>, 1024, smem, attr, HISA_SELECT_ARGS);
-  }
-#undef HISA_SELECT_ARGS
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_select_rows(cu_q, cu_k, seqlens, m_seq, S, m, topk, blk, scores, nullptr, 0,
+                            nullptr, 0, total_q, true, out_idx, out_scores, st);
 }
 
 }  // namespace hisa

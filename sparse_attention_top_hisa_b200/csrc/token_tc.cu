@@ -62,8 +62,9 @@ constexpr size_t TC_SMEM_BYTES = sizeof(TcSmem) + 1024;
 // ---------------------------------------------------------------------------
 // inverted lists
 
-// The (query, slot) pairs of a range of INV_ROWS consecutive query rows are first
-// aggregated per compact key block in shared memory, so that global atomics are
+// Query rows are processed in chunks (see tc_chunking); the lists are kept per (chunk,
+// compact key block).  The (query, slot) pairs of a range of INV_ROWS consecutive query
+// rows are first aggregated per compact key block in shared memory, so that global atomics are
 // issued once per (CTA, key block) instead of once per pair.  A CTA whose rows span
 // more compact blocks than fit in shared memory uses global atomics directly.
 //   mode 0: add the pair counts of every key block to cnt;
@@ -77,8 +78,8 @@ constexpr int INV_LOCAL_BINS = 8192;
 constexpr int INV_RB = 8;  // rows whose block ids a warp loads at once
 
 __global__ void __launch_bounds__(INV_THREADS)
-inv_lists_kernel(const int32_t *__restrict__ blk, int total_q, int m, int sb,
-                 const int32_t *__restrict__ cu_q, int S, int emax, int mode,
+inv_lists_kernel(const int32_t *__restrict__ blk, int total_q, int m, int sb, int chunk_rows,
+                 int nb, const int32_t *__restrict__ cu_q, int S, int emax, int mode,
                  int *__restrict__ cnt, int *__restrict__ cursor, uint32_t *__restrict__ list,
                  int32_t *__restrict__ pmap) {
   __shared__ int loc[INV_LOCAL_BINS];
@@ -92,7 +93,10 @@ inv_lists_kernel(const int32_t *__restrict__ blk, int total_q, int m, int sb,
   }
   __syncthreads();
   const int s0 = seq_range[0], s1 = seq_range[1];
-  const int base = s0 * emax;
+  // the counters of a chunk of query rows follow those of the previous chunk; a CTA's
+  // rows lie in one chunk (chunk_rows is a multiple of INV_ROWS)
+  const int cbase = (r0 / chunk_rows) * nb;
+  const int base = cbase + s0 * emax;
   const int nbl = (s1 - s0 + 1) * emax;
   const bool local = nbl <= INV_LOCAL_BINS;
   // walk the pairs: warp w takes rows r0 + w, r0 + w + NW, ...; lane = slot within a
@@ -119,7 +123,7 @@ inv_lists_kernel(const int32_t *__restrict__ blk, int total_q, int m, int sb,
         }
 #pragma unroll
         for (int u = 0; u < INV_RB; u++)
-          if (b[u] >= 0) fn(rb + u * NW, slot, sq[u] * emax + b[u]);
+          if (b[u] >= 0) fn(rb + u * NW, slot, cbase + sq[u] * emax + b[u]);
       }
     }
   };
@@ -155,10 +159,18 @@ inv_lists_kernel(const int32_t *__restrict__ blk, int total_q, int m, int sb,
 
 constexpr int SCAN_THREADS = 1024;
 
+// One CTA per chunk of query rows: list offsets of the chunk's key blocks (the chunk's
+// list region starts at list_stride * chunk) and its tile descriptors (tile region at
+// tile_stride * chunk), and the chunk's tile count.
 __global__ void __launch_bounds__(SCAN_THREADS)
-inv_scan_kernel(const int *__restrict__ cnt, int nb, int *__restrict__ cursor,
-                TileDesc *__restrict__ tiles, int *__restrict__ ntiles) {
+inv_scan_kernel(const int *__restrict__ cnt, int nb, long long list_stride, int tile_stride,
+                int *__restrict__ cursor, TileDesc *__restrict__ tiles,
+                int *__restrict__ ntiles) {
   __shared__ int warp_tot[SCAN_THREADS / 32 + 1];
+  const int chunk = blockIdx.x;
+  cnt += (size_t)chunk * nb;
+  cursor += (size_t)chunk * nb;
+  tiles += (size_t)chunk * tile_stride;
   const int per = (nb + SCAN_THREADS - 1) / SCAN_THREADS;
   const int b0 = threadIdx.x * per, b1 = min(nb, b0 + per);
   int sc = 0, st = 0;
@@ -168,11 +180,11 @@ inv_scan_kernel(const int *__restrict__ cnt, int nb, int *__restrict__ cursor,
     st += (c + TC_N - 1) / TC_N;
   }
   int total_c, total_t;
-  int oc = block_exclusive_scan<SCAN_THREADS>(sc, warp_tot, &total_c);
+  int oc = (int)(list_stride * chunk) + block_exclusive_scan<SCAN_THREADS>(sc, warp_tot, &total_c);
   int ot = block_exclusive_scan<SCAN_THREADS>(st, warp_tot, &total_t);
   // Tile descriptors: the warp writes its lanes' blocks one after another, 32
-  // descriptors per store instruction (one block can own hundreds of tiles: block 0
-  // is selected by every query).
+  // descriptors per store instruction (one block can own several tiles: block 0 is
+  // selected by every query).
   const int lane = threadIdx.x & 31;
   for (int j = 0; j < per; j++) {
     const int i = b0 + j;
@@ -197,7 +209,7 @@ inv_scan_kernel(const int *__restrict__ cnt, int nb, int *__restrict__ cursor,
     oc += c;
     ot += nt;
   }
-  if (threadIdx.x == 0) *ntiles = total_t;
+  if (threadIdx.x == 0) ntiles[chunk] = total_t;
 }
 
 // ---------------------------------------------------------------------------
@@ -225,8 +237,8 @@ token_score_tc_kernel(const uint16_t *__restrict__ q,
                       const int32_t *__restrict__ cu_k, const int32_t *__restrict__ seqlens,
                       int emax, int sb, const TileDesc *__restrict__ tiles,
                       const int *__restrict__ ntiles_ptr, const uint32_t *__restrict__ list,
-                      float *__restrict__ scratch, int *status, int *launch_abort,
-                      int test_no_loads) {
+                      int list_base, float *__restrict__ scratch, int *status,
+                      int *launch_abort, int test_no_loads) {
   extern __shared__ uint8_t tc_smem_raw[];
   TcSmem &sm = *reinterpret_cast<TcSmem *>((reinterpret_cast<uintptr_t>(tc_smem_raw) + 1023) &
                                            ~(uintptr_t)1023);
@@ -391,7 +403,7 @@ token_score_tc_kernel(const uint16_t *__restrict__ q,
               const uint32_t e = __shfl_sync(0xffffffffu, ej[j], u);
               if (c0 + u < c_end) {
                 const int row = (int)(e >> sb);
-                scratch[(size_t)(td.list_off + c0 + u) * BLK + r] =
+                scratch[(size_t)(td.list_off - list_base + c0 + u) * BLK + r] =
                     row >= rlim ? __uint_as_float(v[u]) : NEG;
               }
             }
@@ -444,9 +456,39 @@ bool make_key_tensor_map(CUtensorMap *map, const uint16_t *k) {
   return make_rows_tensor_map(map, k, (uint64_t)1 << 31, BLK);
 }
 
+// Stage 2 can run over chunks of consecutive query rows, scoring then selecting one chunk
+// at a time, with a score buffer of one chunk; each chunk's list region, tile
+// descriptors and counters sit at fixed offsets, so no scan across chunks is needed.
+// Chunks sized for L2 (tens of MB of scores) were measured slower than one chunk: each
+// scoring and selecting launch pays its ramp and tail, which outweighed the HBM traffic
+// saved (10.2 ms against 5.7 ms per 131072-query step with 1024-row chunks).  So the
+// whole batch is one chunk unless its score buffer would exceed kChunkScoreBytes.
+constexpr size_t kChunkScoreBytes = (size_t)64 << 30;
+
+struct TcChunks {
+  int rows;     // query rows per chunk (a multiple of INV_ROWS)
+  int nchunks;
+};
+
+TcChunks tc_chunking(int total_q, int m) {
+  TcChunks c;
+  long long rows = (long long)(kChunkScoreBytes / ((size_t)m * BLK * 4));
+  rows = rows / INV_ROWS * INV_ROWS;
+  if (rows < INV_ROWS) rows = INV_ROWS;
+  const long long whole = ((long long)total_q + INV_ROWS - 1) / INV_ROWS * INV_ROWS;
+  if (rows > whole) rows = whole > 0 ? whole : INV_ROWS;
+  c.rows = (int)rows;
+  c.nchunks = (int)((total_q + rows - 1) / rows);
+  if (c.nchunks < 1) c.nchunks = 1;
+  return c;
+}
+
 struct TcPlan {
   size_t off_cnt, off_cursor, off_ntiles, off_tiles, off_list, off_pmap, off_scores, total;
-  int nb, max_tiles;
+  int nb;            // counters per chunk (sequences x blocks)
+  int tile_stride;   // tile descriptors reserved per chunk
+  long long list_stride;  // list entries reserved per chunk (rows x m)
+  TcChunks ch;
 };
 
 static size_t a256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -454,24 +496,27 @@ static size_t a256(size_t x) { return (x + 255) & ~(size_t)255; }
 TcPlan tc_plan(int total_q, int num_seqs, int max_seqlen_k, int m) {
   TcPlan p;
   const int emax = (max_seqlen_k + BLK - 1) / BLK;
+  p.ch = tc_chunking(total_q, m);
   p.nb = (num_seqs > 0 ? num_seqs : 1) * (emax > 0 ? emax : 1);
+  p.list_stride = (long long)p.ch.rows * m;
+  p.tile_stride = (int)(p.list_stride / TC_N + p.nb + 1);
   const long long pairs = (long long)total_q * m;
-  p.max_tiles = (int)(pairs / TC_N + p.nb + 1);
+  const size_t nbt = (size_t)p.nb * p.ch.nchunks;
   size_t off = 0;
-  p.off_cnt = off;  // nb counters, then the launch's abort word
-  off = a256(off + (size_t)(p.nb + 1) * 4);
+  p.off_cnt = off;  // every chunk's counters, then the launch's abort word
+  off = a256(off + (nbt + 1) * 4);
   p.off_cursor = off;
-  off = a256(off + (size_t)p.nb * 4);
+  off = a256(off + nbt * 4);
   p.off_ntiles = off;
-  off = a256(off + 4);
+  off = a256(off + (size_t)p.ch.nchunks * 4);
   p.off_tiles = off;
-  off = a256(off + (size_t)p.max_tiles * sizeof(TileDesc));
+  off = a256(off + (size_t)p.tile_stride * p.ch.nchunks * sizeof(TileDesc));
   p.off_list = off;
-  off = a256(off + (size_t)pairs * 4);
+  off = a256(off + (size_t)p.list_stride * p.ch.nchunks * 4);
   p.off_pmap = off;
   off = a256(off + (size_t)pairs * 4);
-  p.off_scores = off;
-  off = a256(off + (size_t)pairs * BLK * 4);
+  p.off_scores = off;  // one chunk's score segments
+  off = a256(off + (size_t)p.list_stride * BLK * 4);
   p.total = off;
   return p;
 }
@@ -480,62 +525,111 @@ size_t tc_workspace_bytes(int total_q, int num_seqs, int max_seqlen_k, int m) {
   return tc_plan(total_q, num_seqs, max_seqlen_k, m).total;
 }
 
-// Scores every selected (query, block) pair into ws's score buffer (one 128-score
-// segment per list entry; *pmap_out[row * m + slot] names the segment of each pair),
-// ready for the select kernel.
 // Tests of the timeout path only (hisa_test_fault): launches made while it is set
 // issue no loads.
 std::atomic<int> g_test_no_loads{0};
 
-cudaError_t launch_token_score_tc(const uint16_t *q, const uint16_t *k, const int32_t *cu_q,
-                                  const int32_t *cu_k, const int32_t *seqlens, int S,
-                                  int total_q, int max_seqlen_k, int m, const int32_t *blk,
-                                  uint8_t *ws, float **scores_out, const int32_t **pmap_out,
-                                  int **abort_out, int num_sms, int *status, cudaStream_t st) {
-  const TcPlan p = tc_plan(total_q, S, max_seqlen_k, m);
-  const int emax = (max_seqlen_k + BLK - 1) / BLK;
-  int *cnt = reinterpret_cast<int *>(ws + p.off_cnt);
-  int *cursor = reinterpret_cast<int *>(ws + p.off_cursor);
-  int *ntiles = reinterpret_cast<int *>(ws + p.off_ntiles);
-  TileDesc *tiles = reinterpret_cast<TileDesc *>(ws + p.off_tiles);
-  uint32_t *list = reinterpret_cast<uint32_t *>(ws + p.off_list);
-  float *scores = reinterpret_cast<float *>(ws + p.off_scores);
-  int32_t *pmap = reinterpret_cast<int32_t *>(ws + p.off_pmap);
-  *scores_out = scores;
-  *pmap_out = pmap;
-  int *launch_abort = cnt + p.nb;
-  *abort_out = launch_abort;
-  cudaError_t e = cudaMemsetAsync(cnt, 0, (size_t)(p.nb + 1) * 4, st);
+// The chunked stage 2 of the tensor-core path, as carved from ws.
+struct TcStage {
+  TcPlan p;
+  int emax, sb;
+  int *cnt, *cursor, *ntiles, *launch_abort;
+  TileDesc *tiles;
+  uint32_t *list;
+  int32_t *pmap;
+  float *scores;
+};
+
+TcStage tc_stage(int total_q, int S, int max_seqlen_k, int m, uint8_t *ws) {
+  TcStage t;
+  t.p = tc_plan(total_q, S, max_seqlen_k, m);
+  t.emax = (max_seqlen_k + BLK - 1) / BLK;
+  t.sb = m > 128 ? 9 : 7;  // slot bits of a list entry (row << sb | slot)
+  t.cnt = reinterpret_cast<int *>(ws + t.p.off_cnt);
+  t.cursor = reinterpret_cast<int *>(ws + t.p.off_cursor);
+  t.ntiles = reinterpret_cast<int *>(ws + t.p.off_ntiles);
+  t.tiles = reinterpret_cast<TileDesc *>(ws + t.p.off_tiles);
+  t.list = reinterpret_cast<uint32_t *>(ws + t.p.off_list);
+  t.pmap = reinterpret_cast<int32_t *>(ws + t.p.off_pmap);
+  t.scores = reinterpret_cast<float *>(ws + t.p.off_scores);
+  t.launch_abort = t.cnt + (size_t)t.p.nb * t.p.ch.nchunks;
+  return t;
+}
+
+// Every chunk's (query, slot) lists and tile descriptors.
+cudaError_t launch_token_lists(const TcStage &t, const int32_t *cu_q, int S, int total_q, int m,
+                               const int32_t *blk, cudaStream_t st) {
+  const size_t nbt = (size_t)t.p.nb * t.p.ch.nchunks;
+  cudaError_t e = cudaMemsetAsync(t.cnt, 0, (nbt + 1) * 4, st);
   if (e != cudaSuccess) return e;
   const int grid = (total_q + INV_ROWS - 1) / INV_ROWS;
-  const int sb = m > 128 ? 9 : 7;  // slot bits of a list entry (row << sb | slot)
   {
     ProfScope ps(K_INV_LISTS, st);
-    inv_lists_kernel<<<grid, INV_THREADS, 0, st>>>(blk, total_q, m, sb, cu_q, S, emax, 0, cnt, cursor, list,
-                                                   pmap);
+    inv_lists_kernel<<<grid, INV_THREADS, 0, st>>>(blk, total_q, m, t.sb, t.p.ch.rows, t.p.nb,
+                                                   cu_q, S, t.emax, 0, t.cnt, t.cursor, t.list,
+                                                   t.pmap);
   }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   {
     ProfScope ps(K_INV_SCAN, st);
-    inv_scan_kernel<<<1, SCAN_THREADS, 0, st>>>(cnt, p.nb, cursor, tiles, ntiles);
+    inv_scan_kernel<<<t.p.ch.nchunks, SCAN_THREADS, 0, st>>>(t.cnt, t.p.nb, t.p.list_stride,
+                                                              t.p.tile_stride, t.cursor, t.tiles,
+                                                              t.ntiles);
   }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   {
     ProfScope ps(K_INV_LISTS, st);
-    inv_lists_kernel<<<grid, INV_THREADS, 0, st>>>(blk, total_q, m, sb, cu_q, S, emax, 1, cnt, cursor, list,
-                                                   pmap);
-  }
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  static std::atomic<int> attr[64];
-  if ((e = set_smem_once((const void *)token_score_tc_kernel, TC_SMEM_BYTES, attr)) != cudaSuccess)
-    return e;
-  {
-    ProfScope ps(K_TOKEN_SCORE_TC, st);
-    token_score_tc_kernel<<<num_sms, TC_THREADS, TC_SMEM_BYTES, st>>>(
-        q, k, cu_q, cu_k, seqlens, emax, sb, tiles, ntiles, list, scores, status,
-        launch_abort, g_test_no_loads.load(std::memory_order_relaxed));
+    inv_lists_kernel<<<grid, INV_THREADS, 0, st>>>(blk, total_q, m, t.sb, t.p.ch.rows, t.p.nb,
+                                                   cu_q, S, t.emax, 1, t.cnt, t.cursor, t.list,
+                                                   t.pmap);
   }
   return cudaGetLastError();
+}
+
+// Scores the selected (query, block) pairs of one chunk into the chunk score buffer:
+// the segment of list entry p is segment p - chunk * list_stride.
+cudaError_t launch_token_score_chunk(const TcStage &t, int chunk, const uint16_t *q,
+                                     const uint16_t *k, const int32_t *cu_q, const int32_t *cu_k,
+                                     const int32_t *seqlens, int num_sms, int *status,
+                                     cudaStream_t st) {
+  static std::atomic<int> attr[64];
+  cudaError_t e = set_smem_once((const void *)token_score_tc_kernel, TC_SMEM_BYTES, attr);
+  if (e != cudaSuccess) return e;
+  ProfScope ps(K_TOKEN_SCORE_TC, st);
+  token_score_tc_kernel<<<num_sms, TC_THREADS, TC_SMEM_BYTES, st>>>(
+      q, k, cu_q, cu_k, seqlens, t.emax, t.sb, t.tiles + (size_t)chunk * t.p.tile_stride,
+      t.ntiles + chunk, t.list, (int)(t.p.list_stride * chunk), t.scores, status, t.launch_abort,
+      g_test_no_loads.load(std::memory_order_relaxed));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_select_rows(const int32_t *cu_q, const int32_t *cu_k, const int32_t *seqlens,
+                               const int32_t *m_seq, int S, int m, int topk, const int32_t *blk,
+                               const float *scores, const int32_t *pmap, int list_base,
+                               const int *launch_abort, int row0, int nrows, bool split,
+                               int32_t *out_idx, float *out_scores, cudaStream_t st);
+
+// Stage 2 on the tensor-core path: every chunk's lists, then per chunk its scores and
+// the exact select of its rows (stream order keeps one chunk's segments in the buffer).
+cudaError_t launch_token_stage_tc(const uint16_t *q, const uint16_t *k, const int32_t *cu_q,
+                                  const int32_t *cu_k, const int32_t *seqlens,
+                                  const int32_t *m_seq, int S, int total_q, int max_seqlen_k,
+                                  int m, int topk, const int32_t *blk, uint8_t *ws, int num_sms,
+                                  int32_t *out_idx, float *out_scores, int *status,
+                                  cudaStream_t st) {
+  const TcStage t = tc_stage(total_q, S, max_seqlen_k, m, ws);
+  cudaError_t e = launch_token_lists(t, cu_q, S, total_q, m, blk, st);
+  if (e != cudaSuccess) return e;
+  for (int c = 0; c < t.p.ch.nchunks; c++) {
+    e = launch_token_score_chunk(t, c, q, k, cu_q, cu_k, seqlens, num_sms, status, st);
+    if (e != cudaSuccess) return e;
+    const int row0 = c * t.p.ch.rows;
+    e = launch_select_rows(cu_q, cu_k, seqlens, m_seq, S, m, topk, blk, t.scores, t.pmap,
+                           (int)(t.p.list_stride * c), t.launch_abort, row0,
+                           min(t.p.ch.rows, total_q - row0), false, out_idx, out_scores, st);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 }  // namespace hisa

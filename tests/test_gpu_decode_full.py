@@ -146,3 +146,70 @@ def test_decode_four_rotating_states_in_a_graph():
         assert torch.equal(fresh, st.reps)
         _oracle_check(dwl, host_k, host_len, dwl.queries[last], outs[last].cpu().numpy(),
                       scs[last].cpu().numpy(), bls[last].cpu().numpy(), f"state {r} last step")
+
+
+def test_fused_decode_step_equals_append_then_select():
+    """hisa_decode_step (append and select in one launch) against hisa_append_keys followed
+    by hisa_select, bit for bit, over 200 steps that cross a block boundary (32768 +
+    128 keys), eagerly and captured in a graph; and the capacity error."""
+    h = H()
+    dwl = config_workload(2, steps=200)
+    S, cap = dwl.num_seqs, dwl.capacity
+    cu_k = dev_i32(dwl.cu_k)
+    cu_q = dev_i32(np.arange(S + 1))
+    a, b = _State(dwl), _State(dwl)
+    newk = dev_bf16(dwl.new_keys.reshape(dwl.steps, S, 64))
+    qs = dev_bf16(dwl.queries.reshape(-1, 64)).view(dwl.steps, S, 64)
+    ws = torch.empty(h.hisa_select_workspace_size(S, S, cap, dwl.m, dwl.topk), dtype=torch.uint8,
+                     device="cuda")
+    outs = [torch.empty(S, dwl.topk, dtype=torch.int32, device="cuda") for _ in range(4)]
+    scs = [torch.empty(S, dwl.topk, dtype=torch.float32, device="cuda") for _ in range(2)]
+    bls = [torch.empty(S, dwl.m, dtype=torch.int32, device="cuda") for _ in range(2)]
+
+    def separate(i):
+        h.hisa_append_keys(a.kc, a.reps, cu_k, a.lens, newk[i].view(S, 1, 64))
+        h.hisa_select(qs[i], a.kc, a.reps, cu_q, cu_k, a.lens, cap, dwl.m, dwl.topk,
+                      out_idx=outs[0], out_scores=scs[0], out_blocks=bls[0], workspace=ws)
+
+    def fused(i):
+        h.hisa_decode_step(b.kc, b.reps, cu_k, b.lens, newk[i], qs[i], cap, dwl.m, dwl.topk,
+                           out_idx=outs[1], out_scores=scs[1], out_blocks=bls[1])
+
+    for i in range(150):
+        separate(i)
+        fused(i)
+        if i % 10 == 9 or i in (127, 128, 129):
+            torch.cuda.synchronize()
+            assert torch.equal(outs[0], outs[1]), i
+            assert torch.equal(scs[0], scs[1]), i
+            assert torch.equal(bls[0], bls[1]), i
+    torch.cuda.synchronize()
+    assert h.hisa_device_status() == 0
+    assert torch.equal(a.lens, b.lens) and torch.equal(a.kc, b.kc) and torch.equal(a.reps, b.reps)
+    # the last 50 steps of the fused path captured in a graph on a side stream
+    g = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(g, stream=side):
+            for i in range(150, 200):
+                h.hisa_decode_step(b.kc, b.reps, cu_k, b.lens, newk[i], qs[i], cap, dwl.m,
+                                   dwl.topk, out_idx=outs[3])
+    torch.cuda.current_stream().wait_stream(side)
+    g.replay()
+    for i in range(150, 200):
+        separate(i)
+    torch.cuda.synchronize()
+    assert torch.equal(outs[0], outs[3])
+    assert torch.equal(a.lens, b.lens) and torch.equal(a.kc, b.kc) and torch.equal(a.reps, b.reps)
+    fresh = h.hisa_pool_blocks(b.kc, cu_k, b.lens, cap)
+    assert torch.equal(fresh, b.reps)
+    del g
+    # a sequence whose region is full: left unchanged, row -1, HISA_ERR_CAPACITY
+    full = dev_i32(np.full(S, cap, np.int32))
+    before = b.kc.clone()
+    out = h.hisa_decode_step(b.kc, b.reps, cu_k, full, newk[0], qs[0], cap, dwl.m, dwl.topk)
+    st = h.hisa_device_status(clear=True)
+    assert st & (1 << 7)
+    assert bool((out == -1).all()) and torch.equal(b.kc, before)
+    assert bool((full == cap).all())
