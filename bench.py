@@ -60,7 +60,12 @@ L2_FLUSH_BYTES = 256 << 20
 # the 131072-token prefill, from an ncu capture of that kernel alone on the 32768-token
 # prefill scaled by the selected (query, block) pairs of the two launches, with the
 # sha256 prefix of the kernel's sources at capture time (a changed source voids it).
-TRAFFIC = {"token_select_scratch": (5241752391, "741119f642a38df2", ("token_select.cu", "select.cuh"))}
+TRAFFIC = {
+    # 32K: 957.4 MB read + 252.3 MB written, 1839104 pairs; 128K: 8130560 pairs
+    "token_select_scratch": (5348312699, "56dc02620c2223cf", ("token_select.cu", "select.cuh")),
+    # 32K: 21.2 MB read + 878.1 MB written
+    "token_score_tc": (3975557505, "8ed7b49db83627bf", ("token_tc.cu",)),
+}
 
 
 def parse_args():
@@ -445,15 +450,18 @@ def run_ours(args, world, rank):
         amount = a["per_step"] / launches_per_step  # per launch
         per_kernel[name] = roofline_entry(a, amount, launch_ms, hbm_peak, tc_peak)
         per_kernel[name]["launches_per_step"] = launches_per_step
+    for name, e in per_kernel.items():
+        t = TRAFFIC.get(name)
+        # stored counters hold for the 128K launch of the kernel source they were taken on
+        e["traffic"] = (int(t[0]) if t and t[1] == source_sha(t[2]) and args.config == 4
+                        and world == 1 else None)
+        if e["traffic"]:
+            e["traffic_GBs"] = round(e["traffic"] / (e["launch_ms"] * 1e6), 1)
+            if alg[name]["bound"] == "hbm":
+                e["traffic_over_algorithmic"] = round(e["traffic"] / e["algorithmic_per_launch"], 3)
     dname = max((n for n in per_kernel), key=lambda n: kt[n]["ms"])
     roof = dict(per_kernel[dname])
     roof["kernel"] = dname
-    t = TRAFFIC.get(dname)
-    # stored counters hold for the 128K launch of the kernel source they were taken on
-    roof["traffic"] = (int(t[0]) if t and t[1] == source_sha(t[2]) and args.config == 4 else None)
-    if roof["traffic"] and alg[dname]["bound"] == "hbm":
-        roof["traffic_over_algorithmic"] = round(
-            roof["traffic"] / (alg[dname]["per_step"] / per_kernel[dname]["launches_per_step"]), 3)
     roof["peak_source"] = f"MEASURED_PEAKS.json ({peak_src})"
     step_alg = alg["step"]
     step_roof = roofline_entry(step_alg, step_alg["per_step"], ms, hbm_peak, tc_peak)
@@ -940,12 +948,11 @@ def decode_profile(steps):
     kc, lens = to_dev_bf16(dw.k_cache), to_dev_i32(dw.seqlens0)
     reps = H.hisa_pool_blocks(kc, cu_k, lens, cap)
     out = torch.empty(S, K, dtype=torch.int32, device="cuda")
-    ws = torch.empty(H.hisa_select_workspace_size(S, S, cap, m, K), dtype=torch.uint8, device="cuda")
     newk = to_dev_bf16(dw.new_keys)
     qs = to_dev_bf16(dw.queries.reshape(steps * S, 64)).view(steps, S, 64)
-    for i in range(steps):
-        H.hisa_append_keys(kc, reps, cu_k, lens, newk[i])
-        H.hisa_select(qs[i], kc, reps, cu_q, cu_k, lens, cap, m, K, out_idx=out, workspace=ws)
+    for i in range(steps):  # the fused step the decode benchmark times
+        H.hisa_decode_step(kc, reps, cu_k, lens, newk[i].reshape(S, 64), qs[i], cap, m, K,
+                           out_idx=out)
     # then the attention step over the last selection (16 heads, width 128)
     rng = np.random.Generator(np.random.PCG64(31))
     ka = to_dev_bf16(bf16_rows(rng, (S * cap, 128)))
