@@ -8,16 +8,18 @@
 // Schedule (the score matrix is never materialised):
 //   1. key_norm_kernel: per sequence the largest key norm |k|max, so that every
 //      score of query q lies in [-R, R] with R = |q| |k|max (Cauchy-Schwarz).
-//   2. dsa_filter_tc_kernel (dsa_tc.cu): one thread per query, 128 queries per
-//      CTA, scores on the tensor cores.  Pass 1 histograms the scores into linear
-//      buckets over [-R, R] (bucket 0 = highest); the bucket holding the k-th best
-//      score is b*.  Pass 2 recomputes the scores and appends every candidate in
-//      buckets <= b* (a superset of the top-k, in token order) to the query's
-//      candidate list.  Bucketing is monotone in the score, so the superset
-//      property holds exactly whatever the rounding.
+//   2. dsa_filter_tc_kernel (dsa_tc.cu): two threads per query, 128 queries per
+//      CTA, scores on the tensor cores.  Pass 1 histograms the scores (of every key
+//      block, or of every eighth for long tiles) into linear buckets over [-R, R]
+//      (bucket 0 = highest) and picks the bucket b* that holds the k-th best score
+//      (or an estimate of a threshold a little under it).  Pass 2 recomputes the
+//      scores and appends every candidate in buckets <= b* to the query's candidate
+//      list.  Bucketing is monotone in the score, so with at least k entries the
+//      list is a superset of the top-k whatever the rounding.
 //   3. dsa_select_kernel: exact top-k of each candidate list (shared routine).
-//   4. dsa_fallback_kernel: a row whose list overflowed its capacity (many equal
-//      scores) is redone exactly from a full score row in scratch memory.
+//   4. dsa_fallback_kernel: a row whose list overflowed its capacity or came out
+//      short (a sampled threshold set too high), or whose boundary holds heavy ties,
+//      is redone exactly from a full score row in scratch memory.
 #include "prof.cuh"
 #include "select.cuh"
 
@@ -88,7 +90,7 @@ __host__ __device__ inline size_t dsa_select_smem(int topk) {
 
 __global__ void __launch_bounds__(DSA_SEL_THREADS)
 dsa_select_kernel(int row0, int topk, int cap, const float *__restrict__ buf_key,
-                  const int32_t *__restrict__ buf_j, const int32_t *__restrict__ cnt,
+                  const int32_t *__restrict__ buf_j, int32_t *__restrict__ cnt,
                   int32_t *__restrict__ out_idx, float *__restrict__ out_scores) {
   extern __shared__ __align__(16) uint8_t smem[];
   const int local = blockIdx.x, row = row0 + local;
@@ -101,8 +103,12 @@ dsa_select_kernel(int row0, int topk, int cap, const float *__restrict__ buf_key
   RegCands<DSA_SEL_THREADS, DSA_SEL_KPT> cs;
   float mx, mn;
   cs.load(src, n, mx, mn);
-  select_topk_lin<DSA_SEL_THREADS>(cs, mx, mn, src, n, topk, sh, smem,
-                                   ListTok{buf_j + (size_t)local * cap}, oi, os);
+  // the lists are not in token order, so heavy ties at the boundary (the radix route,
+  // which breaks ties by list position) are left to the fallback kernel, launched next
+  if (!select_topk_lin<DSA_SEL_THREADS, false>(cs, mx, mn, src, n, topk, sh, smem,
+                                               ListTok{buf_j + (size_t)local * cap}, oi, os) &&
+      threadIdx.x == 0)
+    cnt[local] = cap + 1;
 }
 
 __global__ void __launch_bounds__(DSA_SEL_THREADS)

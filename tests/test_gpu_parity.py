@@ -227,6 +227,30 @@ def test_equal_keys_degenerate():
     assert np.array_equal(h_idx, o_h)
 
 
+def test_dsa_sampled_threshold_too_high_takes_the_fallback():
+    """Long tiles estimate their pass-2 threshold from every eighth key block.  Here those
+    blocks hold keys aligned with the queries and every other block keys opposed to them,
+    so the estimate lands far above the true k-th score, the candidate lists come out
+    short, and the rows must go through the exact fallback.  Integer inputs: bit-exact."""
+    L, k = 12000, 2048
+    rng = np.random.default_rng(812)
+    w = varlen_prefill([L], 3, m=8, topk=k, integer=True)
+    u = rng.integers(-2, 3, size=64).astype(np.float32)
+    u[u == 0] = 1.0
+    q = u + rng.integers(-1, 2, size=(L, 64))
+    blk = np.arange(L) // 128
+    sign = np.where(blk % 8 == 0, 1.0, -1.0)[:, None]
+    kk = sign * u + rng.integers(-1, 2, size=(L, 64))
+    w.q[:] = bf16_from_f32(q.astype(np.float32))
+    w.k[:L] = bf16_from_f32(kk.astype(np.float32))
+    dw = OnDevice(w)
+    idx, sc = run_dsa(dw, k)
+    o_idx, o_sc = oracle.dsa_workload(w)
+    assert np.array_equal(idx, o_idx)
+    valid = o_idx >= 0
+    assert np.array_equal(sc[valid].astype(np.float64), o_sc[valid])
+
+
 def test_hisa_equals_dsa_when_every_block_is_selected():
     """m >= number of blocks: HISA is the flat scan, bit for bit, on Gaussian inputs too."""
     w = gaussian_prefill(4096 + 77, 5, m=64, topk=512)
