@@ -61,8 +61,8 @@ L2_FLUSH_BYTES = 256 << 20
 # prefill scaled by the selected (query, block) pairs of the two launches, with the
 # sha256 prefix of the kernel's sources at capture time (a changed source voids it).
 TRAFFIC = {
-    # 32K: 957.4 MB read + 252.3 MB written, 1839104 pairs; 128K: 8130560 pairs
-    "token_select_scratch": (5348312699, "56dc02620c2223cf", ("token_select.cu", "select.cuh")),
+    # 32K: 957.4 MB read + 252.4 MB written, 1839104 pairs; 128K: 8130560 pairs
+    "token_select_scratch": (5348619405, "45365b5016604859", ("token_select.cu", "select.cuh")),
     # 32K: 21.2 MB read + 878.1 MB written
     "token_score_tc": (3975557505, "8ed7b49db83627bf", ("token_tc.cu",)),
 }

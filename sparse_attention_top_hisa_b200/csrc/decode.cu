@@ -125,7 +125,42 @@ struct DcAppend {
   const uint16_t *new_keys;  // [num_seqs, 64]
 };
 
-__device__ void decode_select_body(DcSmem &sm, const DcAppend &ap, const uint16_t *__restrict__ q,
+// The append of a fused step for sequence s (k0: its region start, len0: its live
+// length before the step), by threads t of nt: the rows of the block that receives
+// the new key are staged, the new key row is written, the block is summed again in
+// increasing row order exactly like the pooling kernels (bit-identical to a fresh
+// pool), and the length grows by one.  sync(): a barrier over the nt threads.
+template <class Sync>
+__device__ void decode_append_block(uint4 *stage, const DcAppend &ap, int k0, int len0, int s,
+                                    int t, int nt, Sync sync) {
+  const int b = len0 / BLK, count = len0 - b * BLK + 1;
+  const uint4 *src = reinterpret_cast<const uint4 *>(ap.new_keys + (size_t)s * D);
+  uint4 *rows = reinterpret_cast<uint4 *>(ap.kc + (size_t)k0 * D);
+  for (int i = t; i < count * 8; i += nt) {
+    const int r = b * BLK + (i >> 3);
+    stage[i] = r < len0 ? rows[(size_t)r * 8 + (i & 7)] : src[i & 7];
+  }
+  if (t < 8) rows[(size_t)len0 * 8 + t] = src[t];
+  sync();
+  if (t < 32) {
+    const uint32_t *w = reinterpret_cast<const uint32_t *>(stage);
+    float a = 0.f, c = 0.f;
+    for (int r = 0; r < count; r++) {
+      const uint32_t x = w[r * 32 + t];
+      a += bf_lo(x);
+      c += bf_hi(x);
+    }
+    const float cnt = (float)count;
+    reinterpret_cast<float2 *>(ap.reps + (size_t)(k0 / BLK + b) * D)[t] =
+        make_float2(__fdiv_rn(a, cnt), __fdiv_rn(c, cnt));
+  }
+  if (t == 0) ap.seqlens[s] = len0 + 1;
+}
+
+// appended: set when a fused step's append was done here (by warps 1..7 of CTA 0 while
+// warp 0 selects the blocks); otherwise the kernel appends after the selection.
+__device__ void decode_select_body(DcSmem &sm, const DcAppend &ap, bool &appended,
+                                   const uint16_t *__restrict__ q,
                                    const uint16_t *__restrict__ k, const float *__restrict__ reps,
                                    const int32_t *__restrict__ cu_q,
                                    const int32_t *__restrict__ cu_k,
@@ -291,9 +326,19 @@ __device__ void decode_select_body(DcSmem &sm, const DcAppend &ap, const uint16_
     if (E <= DC_WARP_TOPM_E) {
       // few blocks: one warp selects (radix digits over a per-warp histogram, no CTA
       // barrier between the rounds) while the others wait once
-      if (warp == 0)
+      const bool append_here = ap.new_keys && me == 0;
+      if (warp == 0) {
         warp_select_blocks(sm.u1.allkeys, E, own, m, sm.blocks, me == 0 ? ob : nullptr, sm.whist,
                            false);
+      } else if (append_here) {
+        // meanwhile the fused step's append (every CTA of the cluster read the old length
+        // before the cluster barrier above; the selection reads neither the new key's
+        // cache row nor its block's representative, the block being forced)
+        decode_append_block(reinterpret_cast<uint4 *>(&sm.u2), ap, qi.kbase, qi.pos, row,
+                            tid - 32, DC_THREADS - 32,
+                            [] { asm volatile("bar.sync 1, %0;" ::"n"(DC_THREADS - 32) : "memory"); });
+      }
+      appended = append_here;  // every thread of the CTA, warp 0 included
       __syncthreads();
     } else if (!cta_select_blocks_lin<DC_THREADS>(sm.u1.allkeys, E, own, m, sm.blocks,
                                                   me == 0 ? ob : nullptr, sm.whist, sm.warp_tot,
@@ -577,38 +622,15 @@ __device__ void decode_select_body(DcSmem &sm, const DcAppend &ap, const uint16_
 }
 
 // The append of a fused step, by CTA 0 of the row's cluster once its selection is done
-// (every CTA of the cluster read the old length long before): the new key row is
-// written, the block that receives it is summed again in increasing row order exactly
-// like the pooling kernels (bit-identical to a fresh pool), and the length grows by one.
+// (every CTA of the cluster read the old length long before), when the selection did
+// not already do it beside its block top-m.
 __device__ void decode_append_tail(DcSmem &sm, const DcAppend &ap, const int32_t *cu_k, int s) {
-  const int tid = threadIdx.x;
   __syncthreads();
   const int k0 = cu_k[s], k1 = cu_k[s + 1];
   const int len0 = ap.seqlens[s];
   if (k0 % BLK != 0 || len0 < 0 || len0 + 1 > k1 - k0) return;  // reported by the body
-  const int b = len0 / BLK, count = len0 - b * BLK + 1;
-  const uint4 *src = reinterpret_cast<const uint4 *>(ap.new_keys + (size_t)s * D);
-  uint4 *rows = reinterpret_cast<uint4 *>(ap.kc + (size_t)k0 * D);
-  uint4 *stage = reinterpret_cast<uint4 *>(&sm.u2);  // 16 KB: the block's rows
-  for (int i = tid; i < count * 8; i += DC_THREADS) {
-    const int r = b * BLK + (i >> 3);
-    stage[i] = r < len0 ? rows[(size_t)r * 8 + (i & 7)] : src[i & 7];
-  }
-  if (tid < 8) rows[(size_t)len0 * 8 + tid] = src[tid];
-  __syncthreads();
-  if (tid < 32) {
-    const uint32_t *w = reinterpret_cast<const uint32_t *>(stage);
-    float a = 0.f, c = 0.f;
-    for (int t = 0; t < count; t++) {
-      const uint32_t x = w[t * 32 + tid];
-      a += bf_lo(x);
-      c += bf_hi(x);
-    }
-    const float cnt = (float)count;
-    reinterpret_cast<float2 *>(ap.reps + (size_t)(k0 / BLK + b) * D)[tid] =
-        make_float2(__fdiv_rn(a, cnt), __fdiv_rn(c, cnt));
-  }
-  if (tid == 0) ap.seqlens[s] = len0 + 1;
+  decode_append_block(reinterpret_cast<uint4 *>(&sm.u2), ap, k0, len0, s, threadIdx.x, DC_THREADS,
+                      [] { __syncthreads(); });
 }
 
 __global__ void __cluster_dims__(DC_CTAS, 1, 1) __launch_bounds__(DC_THREADS, 1)
@@ -625,9 +647,10 @@ decode_select_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict_
   // next kernel may begin launching at once (it waits the same way).
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  decode_select_body(sm, ap, q, k, reps, cu_q, cu_k, seqlens, m_seq, S, m_max, topk, emax,
-                     out_idx, out_scores, out_blocks, status);
-  if (ap.new_keys && cg::this_cluster().block_rank() == 0)
+  bool appended = false;
+  decode_select_body(sm, ap, appended, q, k, reps, cu_q, cu_k, seqlens, m_seq, S, m_max, topk,
+                     emax, out_idx, out_scores, out_blocks, status);
+  if (ap.new_keys && !appended && cg::this_cluster().block_rank() == 0)
     decode_append_tail(sm, ap, cu_k, blockIdx.x / DC_CTAS);
 }
 

@@ -619,9 +619,11 @@ struct LinShared {
   };
 };
 
+// rint((smax - s) * inv) clamped to the last bucket, through the 2^23 magic number
+// instead of a float-to-int conversion: smax - s >= 0, so the sum stays in [2^23, 2^24)
+// where a float's bits count in units of one; monotone (non-increasing) in s.
 __device__ __forceinline__ int lin_bucket(float s, float smax, float inv) {
-  const int b = __float2int_rz((smax - s) * inv);
-  return min(max(b, 0), LIN_BINS - 1);
+  return min(__float_as_int(fmaf(smax - s, inv, 8388608.0f)) - 0x4B000000, LIN_BINS - 1);
 }
 
 // sc: the n raw scores (RowScores or SegScores; four consecutive candidates never
@@ -690,7 +692,8 @@ __device__ void select_topk_reg(Src sc, int n, int k, LinShared &sh, uint32_t *w
   const int nvalid = nv;
   const float smax = mx;
   const float range = mx - mn;
-  const float inv = (nvalid > 0 && range > 0.f) ? (float)LIN_BINS / range : 0.f;
+  float inv = (nvalid > 0 && range > 0.f) ? (float)LIN_BINS / range : 0.f;
+  if (!isfinite(inv)) inv = 0.f;  // a range too narrow to divide: one bucket, radix route
 
   // 2. histogram
 #pragma unroll
@@ -775,290 +778,6 @@ __device__ void select_topk_reg(Src sc, int n, int k, LinShared &sh, uint32_t *w
     const uint64_t me = surv[s];
     const int b = lin_bucket(key_score((uint32_t)(me >> 32)), smax, inv);
     const int st = (int)sh.lin.off[lin_slot(b)], en = (int)sh.lin.cnt[lin_slot(b)];
-    int rank = 0;
-    for (int t = st; t < en; t++) rank += surv[t] > me;
-    out(st + rank, (int)~(uint32_t)me, (uint32_t)(me >> 32));
-  }
-  for (int r = kp + tid; r < k; r += NT) pad(r);
-  __syncthreads();
-}
-
-}  // namespace hisa
-
-namespace hisa {
-
-// ---------------------------------------------------------------------------
-// Exact top-k in two bucket levels, candidates held in registers (the token stage).
-//
-// Input as for select_topk_reg: n raw fp32 scores in candidate (= token) order, -inf
-// marking a position that is not a candidate; NT threads load KPT of them each
-// (candidate c = ((i/4)*NT + thread)*4 + i%4) and keep them in registers.  Then:
-// 1. max/min and count of the candidate scores (fused with the load);
-// 2. level 1: histogram over DN_BINS1 buckets linear in the score between max and
-//    min (bucket 0 holds the highest scores); one scan finds the bucket b1 that holds
-//    the k-th best score, so the candidates of buckets 0..b1 (k plus part of one
-//    bucket) contain the top-k;
-// 3. those candidates are compacted into a dense list in shared memory: every thread
-//    counts its own, one block scan gives each thread its offset;
-// 4. level 2, over the dense list only: histogram over DN_BINS2 buckets linear
-//    between the max and the lower edge of b1, one scan for the bucket offsets and
-//    the bucket b2 that holds the k-th best score;
-// 5. list entries of buckets before b2 are scattered to their bucket's output range,
-//    those of b2 are gathered apart, each as a 64-bit (key, ~candidate) composite
-//    whose unsigned order is the output order (score desc, candidate asc);
-// 6. the b2 members are ranked exactly and the best fill the end of the output;
-//    every other entry is ranked within its own bucket and written to its slot.
-// The per-candidate work of the long passes (2, 3) is a bucket or a compare and a
-// count; the scatter and ranking run densely over about k entries.  A level-1
-// boundary bucket too large for the list, or a level-2 boundary bucket too large for
-// its array (heavy ties), sends the query through the radix routine above instead,
-// reading the scores again.
-constexpr int DN_BINS1 = 512;
-constexpr int DN_BINS2 = 2048;
-constexpr int DN_WORDS2 = DN_BINS2 + DN_BINS2 / 32;  // bucket b at word b + b / 32
-constexpr int DN_LIST_EXTRA = 512;                   // dense list capacity: k + this
-constexpr int DN_BND_CAP = 256;                      // level-2 boundary members
-__device__ __forceinline__ int dn_slot(int b) { return b + (b >> 5); }
-
-struct DnSmall {
-  uint32_t h1[DN_BINS1];
-  uint32_t e2[DN_WORDS2];  // level-2 counts, then bucket offsets, then bucket ends
-  int warp_tot[33];
-  int wn[32];
-  float wmx[32], wmn[32];
-  int misc[8];
-};
-
-// Shared bytes of select_topk_dense for k outputs.  Layout: dense list (score,
-// candidate) x (k + DN_LIST_EXTRA) | survivors u64 x k | boundary u64 x DN_BND_CAP |
-// DnSmall; the radix route reuses the first 16 k bytes as its four lists and puts its
-// SelectShared right after them.
-__host__ __device__ inline size_t dn_small_offset(int k) {
-  return (size_t)8 * (k + DN_LIST_EXTRA) + (size_t)8 * k + (size_t)8 * DN_BND_CAP;
-}
-__host__ __device__ inline size_t dn_bytes(int k) {
-  const size_t a = dn_small_offset(k) + sizeof(DnSmall);
-  const size_t b = (size_t)16 * k + sizeof(SelectShared);
-  return ((a > b ? a : b) + 15) & ~(size_t)15;
-}
-
-__device__ __forceinline__ int dn_bucket(float s, float smax, float inv, int nb) {
-  const int b = __float2int_rz((smax - s) * inv);
-  return min(max(b, 0), nb - 1);
-}
-
-// sc: the n raw scores (RowScores or SegScores).  smem: dn_bytes(k) bytes of shared
-// memory, 16-byte aligned.  Called by all NT threads; contains __syncthreads().
-template <int NT, int KPT, class Src, class Out, class Pad>
-__device__ void select_topk_dense(Src sc, int n, int k, uint8_t *smem, Out out, Pad pad) {
-  static_assert(KPT % 4 == 0 && KPT <= 32, "scores are loaded four at a time, one bit each");
-  static_assert(DN_BINS1 % NT == 0 && DN_BINS2 % NT == 0, "whole buckets per thread");
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  constexpr int NW = NT / 32;
-  const int capd = k + DN_LIST_EXTRA;
-  uint2 *dl = reinterpret_cast<uint2 *>(smem);                               // dense list
-  uint64_t *surv = reinterpret_cast<uint64_t *>(smem + (size_t)8 * capd);    // k survivors
-  uint64_t *bnd = surv + k;                                                  // b2 members
-  DnSmall &sh = *reinterpret_cast<DnSmall *>(smem + dn_small_offset(k));
-  const float NEG = -__int_as_float(0x7f800000);  // -inf
-
-  // 1. load, max / min / count
-  float f[KPT];
-  float mx = NEG, mn = -NEG;
-  int nv = 0;
-#pragma unroll
-  for (int j = 0; j < KPT / 4; j++) {
-    const int c0 = (j * NT + tid) * 4;
-    float4 v = make_float4(NEG, NEG, NEG, NEG);
-    if (c0 + 3 < n) {
-      v = sc.ld4(c0);
-    } else if (c0 < n) {
-      v.x = sc.ld1(c0);
-      if (c0 + 1 < n) v.y = sc.ld1(c0 + 1);
-      if (c0 + 2 < n) v.z = sc.ld1(c0 + 2);
-    }
-    f[4 * j] = v.x;
-    f[4 * j + 1] = v.y;
-    f[4 * j + 2] = v.z;
-    f[4 * j + 3] = v.w;
-#pragma unroll
-    for (int e = 0; e < 4; e++) {
-      const float x = f[4 * j + e];
-      if (x != NEG) {
-        mx = fmaxf(mx, x);
-        mn = fminf(mn, x);
-        nv++;
-      }
-    }
-  }
-  auto cand = [&](int i) { return ((i >> 2) * NT + tid) * 4 + (i & 3); };
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-    nv += __shfl_xor_sync(0xffffffffu, nv, o);
-  }
-  if (lane == 0) {
-    sh.wmx[warp] = mx;
-    sh.wmn[warp] = mn;
-    sh.wn[warp] = nv;
-  }
-  for (int i = tid; i < DN_BINS1; i += NT) sh.h1[i] = 0u;
-  for (int i = tid; i < DN_WORDS2; i += NT) sh.e2[i] = 0u;
-  if (tid == 0) sh.misc[5] = 0;  // level-2 boundary fill counter
-  __syncthreads();
-  mx = NEG;
-  mn = -NEG;
-  nv = 0;
-#pragma unroll
-  for (int w = 0; w < NW; w++) {
-    mx = fmaxf(mx, sh.wmx[w]);
-    mn = fminf(mn, sh.wmn[w]);
-    nv += sh.wn[w];
-  }
-  const int nvalid = nv, kp = min(k, nvalid);
-  const float smax = mx, range = mx - mn;
-  const float inv1 = range > 0.f ? (float)DN_BINS1 / range : 0.f;
-
-  auto radix_route = [&]() {
-    __syncthreads();  // every thread is done with the dense layout
-    auto key = [&](int c) -> uint32_t {
-      const float x = sc.ld1(c);
-      return x != NEG ? score_key(x) : 0u;
-    };
-    uint32_t *w = reinterpret_cast<uint32_t *>(smem);
-    SelectShared &rs = *reinterpret_cast<SelectShared *>(smem + (size_t)16 * k);
-    select_topk<NT>(key, n, k, rs, w, reinterpret_cast<int *>(w + k), w + 2 * k,
-                    reinterpret_cast<int *>(w + 3 * k), out, pad);
-  };
-  if (nvalid == 0) {
-    for (int r = tid; r < k; r += NT) pad(r);
-    __syncthreads();
-    return;
-  }
-  if (!(range > 0.f) || !isfinite(inv1)) {  // every candidate score equal
-    radix_route();
-    return;
-  }
-
-  // 2. level 1
-#pragma unroll
-  for (int i = 0; i < KPT; i++)
-    if (f[i] != NEG) atomicAdd(&sh.h1[dn_bucket(f[i], smax, inv1, DN_BINS1)], 1u);
-  __syncthreads();
-  {
-    constexpr int PER = DN_BINS1 / NT;
-    uint32_t h[PER];
-    int local = 0;
-#pragma unroll
-    for (int i = 0; i < PER; i++) {
-      h[i] = sh.h1[tid * PER + i];
-      local += (int)h[i];
-    }
-    int total;
-    int run = block_exclusive_scan<NT>(local, sh.warp_tot, &total);
-#pragma unroll
-    for (int i = 0; i < PER; i++) {
-      if (run < kp && run + (int)h[i] >= kp) {  // exactly one bucket
-        sh.misc[0] = tid * PER + i;
-        sh.misc[1] = run + (int)h[i];
-      }
-      run += (int)h[i];
-    }
-  }
-  __syncthreads();
-  const int b1 = sh.misc[0], nd = sh.misc[1];  // candidates in buckets 0..b1
-  if (nd > capd) {  // a level-1 bucket too crowded for the list
-    radix_route();
-    return;
-  }
-
-  // 3. compaction of buckets 0..b1 (every thread's candidates in a contiguous run)
-  uint32_t keep = 0u;
-  int mine = 0;
-#pragma unroll
-  for (int i = 0; i < KPT; i++) {
-    const bool kp_i = f[i] != NEG && dn_bucket(f[i], smax, inv1, DN_BINS1) <= b1;
-    keep |= (uint32_t)kp_i << i;
-    mine += kp_i;
-  }
-  {
-    int total;
-    int at = block_exclusive_scan<NT>(mine, sh.warp_tot, &total);
-#pragma unroll
-    for (int i = 0; i < KPT; i++)
-      if ((keep >> i) & 1u) dl[at++] = make_uint2(__float_as_uint(f[i]), (uint32_t)cand(i));
-  }
-  // level-2 buckets run from the top score to the lower edge of b1; rounding can put
-  // a list entry a little past either end, where the clamp keeps the order
-  const float inv2 = (float)DN_BINS2 * inv1 / (float)(b1 + 1);
-  __syncthreads();
-  if (!isfinite(inv2)) {  // a range too narrow for the finer buckets
-    radix_route();
-    return;
-  }
-
-  // 4. level 2 over the list
-  for (int e = tid; e < nd; e += NT)
-    atomicAdd(&sh.e2[dn_slot(dn_bucket(__uint_as_float(dl[e].x), smax, inv2, DN_BINS2))], 1u);
-  __syncthreads();
-  {
-    constexpr int PER = DN_BINS2 / NT;
-    uint32_t h[PER];
-    int local = 0;
-#pragma unroll
-    for (int i = 0; i < PER; i++) {
-      h[i] = sh.e2[dn_slot(tid * PER + i)];
-      local += (int)h[i];
-    }
-    int total;
-    int run = block_exclusive_scan<NT>(local, sh.warp_tot, &total);
-#pragma unroll
-    for (int i = 0; i < PER; i++) {
-      const int b = tid * PER + i;
-      if (run < kp && run + (int)h[i] >= kp) {
-        sh.misc[2] = b;
-        sh.misc[3] = run;
-        sh.misc[4] = (int)h[i];
-      }
-      sh.e2[dn_slot(b)] = (uint32_t)run;  // becomes the scatter cursor, then the end
-      run += (int)h[i];
-    }
-  }
-  __syncthreads();
-  const int b2 = sh.misc[2], above = sh.misc[3], nbnd = sh.misc[4];
-  const int need = kp - above;
-  if (nbnd > DN_BND_CAP) {  // heavy ties at the level-2 boundary
-    radix_route();
-    return;
-  }
-
-  // 5. scatter
-  for (int e = tid; e < nd; e += NT) {
-    const uint2 d = dl[e];
-    const float x = __uint_as_float(d.x);
-    const int b = dn_bucket(x, smax, inv2, DN_BINS2);
-    if (b < b2) {
-      const uint32_t p = atomicAdd(&sh.e2[dn_slot(b)], 1u);
-      surv[p] = rank_key(x, (int)d.y);
-    } else if (b == b2) {
-      bnd[atomicAdd(&sh.misc[5], 1)] = rank_key(x, (int)d.y);
-    }
-  }
-  __syncthreads();
-
-  // 6. the boundary bucket ranked exactly, then every survivor within its bucket;
-  //    bucket b < b2 now spans [end(b - 1), end(b))
-  for (int e = tid; e < nbnd; e += NT) {
-    const uint64_t me = bnd[e];
-    int rank = 0;
-    for (int t = 0; t < nbnd; t++) rank += bnd[t] > me;
-    if (rank < need) out(above + rank, (int)~(uint32_t)me, (uint32_t)(me >> 32));
-  }
-  for (int s = tid; s < above; s += NT) {
-    const uint64_t me = surv[s];
-    const int b = dn_bucket(key_score((uint32_t)(me >> 32)), smax, inv2, DN_BINS2);
-    const int st = b ? (int)sh.e2[dn_slot(b - 1)] : 0, en = (int)sh.e2[dn_slot(b)];
     int rank = 0;
     for (int t = st; t < en; t++) rank += surv[t] > me;
     out(st + rank, (int)~(uint32_t)me, (uint32_t)(me >> 32));
