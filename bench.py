@@ -56,10 +56,11 @@ CONFIG_WORKLOADS = {
 }
 L2_FLUSH_BYTES = 256 << 20
 
-# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) of a kernel on
-# the 131072-token prefill, from an ncu capture of that kernel alone on the 32768-token
-# prefill scaled by the selected (query, block) pairs of the two launches, with the
-# sha256 prefix of the kernel's sources at capture time (a changed source voids it).
+# DRAM bytes per step (dram__bytes_read.sum + dram__bytes_write.sum summed over the
+# kernel's launches) on the 131072-token prefill, from an ncu capture of that kernel on
+# the 32768-token prefill scaled by the selected (query, block) pairs of the two, with
+# the sha256 prefix of the kernel's sources at capture time (a changed source voids it);
+# the bench line divides it by the launches per step.
 TRAFFIC = {
     # 32K: 957.4 MB read + 252.4 MB written, 1839104 pairs; 128K: 8130560 pairs
     "token_select_scratch": (5348619405, "45365b5016604859", ("token_select.cu", "select.cuh")),
@@ -453,8 +454,9 @@ def run_ours(args, world, rank):
     for name, e in per_kernel.items():
         t = TRAFFIC.get(name)
         # stored counters hold for the 128K launch of the kernel source they were taken on
-        e["traffic"] = (int(t[0]) if t and t[1] == source_sha(t[2]) and args.config == 4
-                        and world == 1 else None)
+        e["traffic"] = (int(round(t[0] / e["launches_per_step"]))
+                        if t and t[1] == source_sha(t[2]) and args.config == 4 and world == 1
+                        else None)
         if e["traffic"]:
             e["traffic_GBs"] = round(e["traffic"] / (e["launch_ms"] * 1e6), 1)
             if alg[name]["bound"] == "hbm":

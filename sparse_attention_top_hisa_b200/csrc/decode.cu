@@ -157,6 +157,34 @@ __device__ void decode_append_block(uint4 *stage, const DcAppend &ap, int k0, in
   if (t == 0) ap.seqlens[s] = len0 + 1;
 }
 
+// Rarely taken routes, kept out of line so that the hot path's code stays compact (every
+// decode launch starts with a cold instruction cache).
+// Heavy ties: CTA 0 runs the radix select over the candidates of every CTA of the
+// cluster (read through distributed shared memory).
+__device__ __noinline__ void decode_radix_select(DcSmem &sm, int cper, int n, int topk,
+                                                 DcOut out, DcPad pad) {
+  cg::cluster_group cl = cg::this_cluster();
+  const float NEG = -__int_as_float(0x7f800000);
+  auto key = [&](int c) -> uint32_t {
+    const int owner = c / cper;
+    const float *rc = cl.map_shared_rank(sm.cand, owner);
+    const float x = rc[c - owner * cper];
+    return x != NEG ? score_key(x) : 0u;
+  };
+  uint32_t *w = sm.u2.radix_work;
+  select_topk<DC_THREADS>(key, n, topk, sm.u1.radix, w, reinterpret_cast<int *>(w + topk),
+                          w + 2 * topk, reinterpret_cast<int *>(w + 3 * topk), out, pad);
+}
+
+// More eligible blocks than one warp selects quickly: the CTA-wide top-m.
+__device__ __noinline__ void decode_cta_select_blocks(DcSmem &sm, int E, int own, int m,
+                                                      int32_t *ob) {
+  if (!cta_select_blocks_lin<DC_THREADS>(sm.u1.allkeys, E, own, m, sm.blocks, ob, sm.whist,
+                                         sm.warp_tot, sm.bsc, reinterpret_cast<uint8_t *>(&sm.u2)))
+    cta_select_blocks<DC_THREADS>(sm.u1.allkeys, E, own, m, sm.blocks, ob, sm.whist, sm.warp_tot,
+                                  sm.bsc);
+}
+
 // appended: set when a fused step's append was done here (by warps 1..7 of CTA 0 while
 // warp 0 selects the blocks); otherwise the kernel appends after the selection.
 __device__ void decode_select_body(DcSmem &sm, const DcAppend &ap, bool &appended,
@@ -340,11 +368,8 @@ __device__ void decode_select_body(DcSmem &sm, const DcAppend &ap, bool &appende
       }
       appended = append_here;  // every thread of the CTA, warp 0 included
       __syncthreads();
-    } else if (!cta_select_blocks_lin<DC_THREADS>(sm.u1.allkeys, E, own, m, sm.blocks,
-                                                  me == 0 ? ob : nullptr, sm.whist, sm.warp_tot,
-                                                  sm.bsc, reinterpret_cast<uint8_t *>(&sm.u2))) {
-      cta_select_blocks<DC_THREADS>(sm.u1.allkeys, E, own, m, sm.blocks,
-                                    me == 0 ? ob : nullptr, sm.whist, sm.warp_tot, sm.bsc);
+    } else {
+      decode_cta_select_blocks(sm, E, own, m, me == 0 ? ob : nullptr);
     }
   } else {
     for (int i = tid; i < m; i += DC_THREADS) {
@@ -486,19 +511,7 @@ __device__ void decode_select_body(DcSmem &sm, const DcAppend &ap, bool &appende
   // the radix route over all candidates of the cluster (run by CTA 0)
   auto radix_route = [&]() {
     cl.sync();  // every CTA is done with the exchanged counts
-    if (me == 0) {
-      const int cper = bp * BLK;
-      auto key = [&](int c) -> uint32_t {
-        const int owner = c / cper;
-        const float *rc = cl.map_shared_rank(sm.cand, owner);
-        const float x = rc[c - owner * cper];
-        return x != NEG ? score_key(x) : 0u;
-      };
-      uint32_t *w = sm.u2.radix_work;
-      select_topk<DC_THREADS>(key, nsel * BLK, topk, sm.u1.radix, w,
-                              reinterpret_cast<int *>(w + topk), w + 2 * topk,
-                              reinterpret_cast<int *>(w + 3 * topk), out, pad);
-    }
+    if (me == 0) decode_radix_select(sm, bp * BLK, nsel * BLK, topk, out, pad);
     cl.sync();  // the other CTAs' candidates stay readable until CTA 0 is done
   };
   if (nvalid == 0) {
@@ -624,7 +637,8 @@ __device__ void decode_select_body(DcSmem &sm, const DcAppend &ap, bool &appende
 // The append of a fused step, by CTA 0 of the row's cluster once its selection is done
 // (every CTA of the cluster read the old length long before), when the selection did
 // not already do it beside its block top-m.
-__device__ void decode_append_tail(DcSmem &sm, const DcAppend &ap, const int32_t *cu_k, int s) {
+__device__ __noinline__ void decode_append_tail(DcSmem &sm, const DcAppend &ap,
+                                               const int32_t *cu_k, int s) {
   __syncthreads();
   const int k0 = cu_k[s], k1 = cu_k[s + 1];
   const int len0 = ap.seqlens[s];
