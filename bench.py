@@ -55,6 +55,8 @@ CONFIG_WORKLOADS = {
     5: "prefill varlen (8 seqs, q/k bf16 N(0,1), d=64, B=128, m=64, k=2048)",
 }
 L2_FLUSH_BYTES = 256 << 20
+# row ranges of the end-to-end step (their index copies overlap the next range's select)
+E2E_CHUNKS = 8
 
 # DRAM bytes per step (dram__bytes_read.sum + dram__bytes_write.sum summed over the
 # kernel's launches) on the 131072-token prefill, from an ncu capture of that kernel on
@@ -412,31 +414,86 @@ def run_ours(args, world, rank):
     value = nq_job / (ms / 1e3)  # strong scaling: the ranks share one fixed workload
 
     # ---- end to end: host buffers through the public API --------------------------
+    # Every step copies the inputs in from pinned host memory, pools, selects and copies
+    # the indices back.  The rows are selected in E2E_CHUNKS contiguous ranges, each a
+    # batch of its own (the shard layouts of sparse_attention_top_hisa_b200.shard, which
+    # reproduce the unsharded rows exactly), and each range's indices go back to the host
+    # on a copy stream while the next range is selected; "one_call" is the same with a
+    # single hisa_select and the copy after it.
+    from sparse_attention_top_hisa_b200.shard import query_cost, row_bounds, shard
     hq = torch.from_numpy(np.ascontiguousarray(w.q).view(np.int16)).view(torch.bfloat16).pin_memory()
     hk = torch.from_numpy(np.ascontiguousarray(w.k).view(np.int16)).view(torch.bfloat16).pin_memory()
     hcq = torch.from_numpy(w.cu_q.astype(np.int32)).pin_memory()
     hck = torch.from_numpy(w.cu_k.astype(np.int32)).pin_memory()
     hsl = torch.from_numpy(w.seqlens.astype(np.int32)).pin_memory()
     hout = torch.empty(nq, K, dtype=torch.int32).pin_memory()
-    e2e_steps = max(2, min(args.steps, 5))
-    e2e_ms = []
-    for i in range(e2e_steps + 1):
-        flush.fill_(i & 0xFF)
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
+    nch = E2E_CHUNKS if nq >= E2E_CHUNKS * 4096 else 1
+    copy_stream = torch.cuda.Stream()
+    # per-range layout arrays: pinned host staging and device copies, filled every step
+    hdesc = [torch.empty(3 * (w.num_seqs + 1), dtype=torch.int32).pin_memory() for _ in range(nch)]
+    ddesc = [torch.empty(3 * (w.num_seqs + 1), dtype=torch.int32, device="cuda")
+             for _ in range(nch)]
+
+    def e2e_step(chunked):
         q.copy_(hq, non_blocking=True)
         k.copy_(hk, non_blocking=True)
         cu_q.copy_(hcq, non_blocking=True)
         cu_k.copy_(hck, non_blocking=True)
         sl.copy_(hsl, non_blocking=True)
-        step()
-        hout.copy_(out, non_blocking=True)
-        b.record(stream)
-        b.synchronize()
-        if i > 0:
-            e2e_ms.append(a.elapsed_time(b))
-    e2e = max_over_ranks(sum(e2e_ms) / len(e2e_ms), world)
-    h2d = sum_over_ranks(sum(t.numel() * t.element_size() for t in (hq, hk, hcq, hck, hsl)), world)
+        if not chunked:
+            step()
+            hout.copy_(out, non_blocking=True)
+            return 0
+        H.hisa_pool_blocks(k, cu_k, sl, w.max_seqlen_k, reps=reps)
+        lay = (hcq.numpy(), hck.numpy(), hsl.numpy())
+        bounds = row_bounds(nq, nch, query_cost(*lay, B, m))
+        extra = 0
+        for c in range(nch):
+            sh = shard(*lay, nch, c, B, bounds)
+            ns = sh.num_seqs
+            hd = hdesc[c]
+            hd[:ns + 1] = torch.from_numpy(sh.cu_seqlens_q)
+            hd[ns + 1:2 * ns + 2] = torch.from_numpy(sh.cu_seqlens_k)
+            hd[2 * ns + 2:3 * ns + 2] = torch.from_numpy(sh.seqlens_k)
+            dd = ddesc[c]
+            dd[:3 * ns + 2].copy_(hd[:3 * ns + 2], non_blocking=True)
+            extra += (3 * ns + 2) * 4
+            H.hisa_select(q[sh.row0:sh.row1], k[sh.key0:sh.key1], reps[sh.rep0:], dd[:ns + 1],
+                          dd[ns + 1:2 * ns + 2], dd[2 * ns + 2:3 * ns + 2], sh.max_seqlen_k, m, K,
+                          out_idx=out[sh.row0:sh.row1], workspace=ws)
+            done = torch.cuda.Event()
+            done.record(stream)
+            copy_stream.wait_event(done)
+            with torch.cuda.stream(copy_stream):
+                hout[sh.row0:sh.row1].copy_(out[sh.row0:sh.row1], non_blocking=True)
+        stream.wait_stream(copy_stream)
+        return extra
+
+    def time_e2e(chunked):
+        times, extra = [], 0
+        for i in range(e2e_steps + 1):
+            flush.fill_(i & 0xFF)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            extra = e2e_step(chunked)
+            b.record(stream)
+            b.synchronize()
+            if i > 0:
+                times.append(a.elapsed_time(b))
+        return max_over_ranks(sum(times) / len(times), world), extra
+
+    e2e_steps = max(2, min(args.steps, 5))
+    e2e_one, _ = time_e2e(False)
+    if nch > 1:
+        ref = hout.clone()
+        e2e, desc_bytes = time_e2e(True)
+        assert torch.equal(hout, ref), "row ranges differ from the single call"
+        del ref
+    else:
+        e2e, desc_bytes = e2e_one, 0
+    assert H.hisa_device_status() == 0, "device-side error in the end-to-end steps"
+    h2d = sum_over_ranks(sum(t.numel() * t.element_size() for t in (hq, hk, hcq, hck, hsl))
+                         + desc_bytes, world)
     d2h = sum_over_ranks(hout.numel() * hout.element_size(), world)
 
     # ---- roofline of the dominant kernel -------------------------------------------
@@ -502,7 +559,9 @@ def run_ours(args, world, rank):
                                    else "single GPU")},
         "e2e": {"value": round(nq_job / (e2e / 1e3), 1), "unit": UNIT,
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-                "ms_per_step": round(e2e, 3)},
+                "ms_per_step": round(e2e, 3), "row_ranges": nch,
+                "one_call": {"value": round(nq_job / (e2e_one / 1e3), 1),
+                             "ms_per_step": round(e2e_one, 3)}},
         "gpu_launches": launches,
         "roofline": roof,
         "clocks": clocks,
