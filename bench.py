@@ -915,8 +915,10 @@ def _time_oracle(fn):
 
 def cpu_baseline(w, budget_s: float = 15.0):
     """The oracle (unchanged) on the host cores: a seeded sample of query rows of the
-    benchmark workload (the line's value), and the HISA and flat-DSA oracles timed on
-    every configuration (in full where that takes seconds, else on 4096 seeded rows)."""
+    benchmark workload (the line's value), the HISA oracle timed in full on every
+    configuration, and the flat-DSA oracle in full on the 4K and 32K prefills and on 4096
+    seeded rows of the 128K and varlen ones (its cost grows with the square of the
+    length)."""
     import oracle
     from synth import config_workload
     n = cores()
@@ -939,8 +941,8 @@ def cpu_baseline(w, budget_s: float = 15.0):
             wc.total_q, 4096, replace=False)).astype(np.int32)
         nr = wc.total_q if full else 4096
         per[str(cfg)] = {
-            "hisa": entry(nr, _time_oracle(lambda: oracle.hisa_workload(wc, rows=r, nthreads=n)),
-                          full),
+            "hisa": entry(wc.total_q,
+                          _time_oracle(lambda: oracle.hisa_workload(wc, nthreads=n)), True),
             "dsa": entry(nr, _time_oracle(lambda: oracle.dsa_workload(wc, rows=r, nthreads=n)),
                          full)}
     # decode: one step (append then select) of the 16 sequences, through the oracle's
