@@ -151,23 +151,31 @@ block_score_tc_kernel(const __grid_constant__ CUtensorMap qmap,
     __syncwarp();
     mbar_wait(&sm.bar_mma, phase, status);
     tc_fence_after();
-    for (int cc = 0; cc < npad; cc += 16) {
-      uint32_t v[16];
-      tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)cc, v);
+    // 64 columns per wait: four TMEM loads in flight (npad is warp-uniform)
+    for (int c64 = 0; c64 < npad; c64 += 64) {
+      uint32_t v[4][16];
+#pragma unroll
+      for (int j = 0; j < 4; j++)
+        if (c64 + 16 * j < npad)
+          tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(c64 + 16 * j), v[j]);
       tmem_wait_ld();
-      if (row_ok && c0 + cc < e_tile) {
-        uint32_t key[16];
 #pragma unroll
-        for (int u = 0; u < 16; u++) {
-          const int b = c0 + cc + u;
-          const bool forced = b == own || (nf >= 2 && b == own - 1) || (nf >= 3 && b == 0);
-          key[u] = (b <= own && !forced) ? score_key(__uint_as_float(v[u])) : 0u;
+      for (int j = 0; j < 4; j++) {
+        const int cc = c64 + 16 * j;
+        if (cc < npad && row_ok && c0 + cc < e_tile) {
+          uint32_t key[16];
+#pragma unroll
+          for (int u = 0; u < 16; u++) {
+            const int b = c0 + cc + u;
+            const bool forced = b == own || (nf >= 2 && b == own - 1) || (nf >= 3 && b == 0);
+            key[u] = (b <= own && !forced) ? score_key(__uint_as_float(v[j][u])) : 0u;
+          }
+          // rows are estride (a multiple of 16) keys long; columns past e_tile get 0
+          uint4 *dst = reinterpret_cast<uint4 *>(out_row + c0 + cc);
+#pragma unroll
+          for (int u = 0; u < 4; u++)
+            dst[u] = make_uint4(key[4 * u], key[4 * u + 1], key[4 * u + 2], key[4 * u + 3]);
         }
-        // rows are estride (a multiple of 16) keys long; columns past e_tile get 0
-        uint4 *dst = reinterpret_cast<uint4 *>(out_row + c0 + cc);
-#pragma unroll
-        for (int u = 0; u < 4; u++)
-          dst[u] = make_uint4(key[4 * u], key[4 * u + 1], key[4 * u + 2], key[4 * u + 3]);
       }
     }
     tc_fence_before();

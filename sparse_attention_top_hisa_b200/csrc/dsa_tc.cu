@@ -264,41 +264,49 @@ dsa_filter_tc_kernel(const __grid_constant__ CUtensorMap qmap,
       const int b = it < ns ? it * ss : it - ns;
       const bool pass2 = it >= ns;
       const int jmax = active ? pos - b * BLK : -1;  // keys 0..jmax of this block are causal
-      for (int c0 = cbeg; c0 < cend; c0 += 16) {
-        uint32_t v[16];
-        tmem_ld16(tmem + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)(st * BLK + c0), v);
+      for (int c32 = cbeg; c32 < cend; c32 += 32) {
+        // 32 columns per wait: two TMEM loads in flight
+        uint32_t vv[2][16];
+        tmem_ld16(tmem + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)(st * BLK + c32), vv[0]);
+        tmem_ld16(tmem + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)(st * BLK + c32 + 16),
+                  vv[1]);
         tmem_wait_ld();
-        if (c0 + 15 <= jmax) {  // the whole chunk is causal
-          if (!pass2) {
 #pragma unroll
-            for (int u = 0; u < 16; u++) atomicAdd(&hist[dsa_bucket(__uint_as_float(v[u]), R, inv)], 1u);
-            counted += 16;
-          } else {
+        for (int h = 0; h < 2; h++) {
+          const int c0 = c32 + 16 * h;
+          const uint32_t *v = vv[h];
+          if (c0 + 15 <= jmax) {  // the whole chunk is causal
+            if (!pass2) {
 #pragma unroll
-            for (int u = 0; u < 16; u++) {
-              const float sc = __uint_as_float(v[u]);
-              if (sc >= thr) {
-                const int p = atomicAdd(&sm.qcount[qi], 1);
-                if (p < cap) {
-                  bk[p] = sc;
-                  bj[p] = b * BLK + c0 + u;
+              for (int u = 0; u < 16; u++) atomicAdd(&hist[dsa_bucket(__uint_as_float(v[u]), R, inv)], 1u);
+              counted += 16;
+            } else {
+#pragma unroll
+              for (int u = 0; u < 16; u++) {
+                const float sc = __uint_as_float(v[u]);
+                if (sc >= thr) {
+                  const int p = atomicAdd(&sm.qcount[qi], 1);
+                  if (p < cap) {
+                    bk[p] = sc;
+                    bj[p] = b * BLK + c0 + u;
+                  }
                 }
               }
             }
-          }
-        } else if (c0 <= jmax) {  // the diagonal chunk
+          } else if (c0 <= jmax) {  // the diagonal chunk
 #pragma unroll
-          for (int u = 0; u < 16; u++) {
-            if (c0 + u <= jmax) {
-              const float sc = __uint_as_float(v[u]);
-              if (!pass2) {
-                atomicAdd(&hist[dsa_bucket(sc, R, inv)], 1u);
-                counted++;
-              } else if (sc >= thr) {
-                const int p = atomicAdd(&sm.qcount[qi], 1);
-                if (p < cap) {
-                  bk[p] = sc;
-                  bj[p] = b * BLK + c0 + u;
+            for (int u = 0; u < 16; u++) {
+              if (c0 + u <= jmax) {
+                const float sc = __uint_as_float(v[u]);
+                if (!pass2) {
+                  atomicAdd(&hist[dsa_bucket(sc, R, inv)], 1u);
+                  counted++;
+                } else if (sc >= thr) {
+                  const int p = atomicAdd(&sm.qcount[qi], 1);
+                  if (p < cap) {
+                    bk[p] = sc;
+                    bj[p] = b * BLK + c0 + u;
+                  }
                 }
               }
             }
