@@ -535,6 +535,8 @@ def run_ours(args, world, rank):
         del dout, dws
 
     details = {"hisa_step": {"ms": round(ms, 4), "queries_per_s": round(nq_job / (ms / 1e3), 1),
+                             "median_ms": round(float(np.median(step_ms)), 4),
+                             "min_ms": round(float(min(step_ms)), 4),
                              "rank_rows": [int(row0), int(row1)],
                              "kernels": {n: {"ms_per_step": round(v["ms"] / args.steps, 4),
                                              "launches": v["launches"]}
