@@ -213,3 +213,52 @@ def test_fused_decode_step_equals_append_then_select():
     assert st & (1 << 7)
     assert bool((out == -1).all()) and torch.equal(b.kc, before)
     assert bool((full == cap).all())
+
+
+def test_fused_decode_step_mixed_lengths():
+    """hisa_decode_step on sequences of very different lengths, integer inputs: one
+    sequence with a single block and two with at most m blocks (every block kept, the
+    append after the selection), two selected by one warp, and one with more than 1024
+    blocks (the CTA-wide top-m, the append after the selection); 40 steps, each
+    sequence crossing a block boundary at its own step.  Bit for bit against
+    hisa_append_keys followed by hisa_select, and the last step against the oracle."""
+    from synth import decode_workload
+    h = H()
+    lens0 = np.array([100, 250, 1000, 5100, 70000, 140000], np.int32)
+    S, steps, m, k = len(lens0), 40, 16, 512
+    dwl = decode_workload(S, int(lens0.max()), steps, 4242, m=m, topk=k, integer=True)
+    dwl.seqlens0 = lens0.copy()
+    cap = dwl.capacity
+    cu_k = dev_i32(dwl.cu_k)
+    cu_q = dev_i32(np.arange(S + 1))
+    a, b = _State(dwl), _State(dwl)
+    newk = dev_bf16(dwl.new_keys.reshape(steps, S, 64))
+    qs = dev_bf16(dwl.queries.reshape(-1, 64)).view(steps, S, 64)
+    ws = torch.empty(h.hisa_select_workspace_size(S, S, cap, m, k), dtype=torch.uint8,
+                     device="cuda")
+    outs = [torch.empty(S, k, dtype=torch.int32, device="cuda") for _ in range(2)]
+    scs = [torch.empty(S, k, dtype=torch.float32, device="cuda") for _ in range(2)]
+    bls = [torch.empty(S, m, dtype=torch.int32, device="cuda") for _ in range(2)]
+    for i in range(steps):
+        h.hisa_append_keys(a.kc, a.reps, cu_k, a.lens, newk[i].view(S, 1, 64))
+        h.hisa_select(qs[i], a.kc, a.reps, cu_q, cu_k, a.lens, cap, m, k, out_idx=outs[0],
+                      out_scores=scs[0], out_blocks=bls[0], workspace=ws)
+        h.hisa_decode_step(b.kc, b.reps, cu_k, b.lens, newk[i], qs[i], cap, m, k,
+                           out_idx=outs[1], out_scores=scs[1], out_blocks=bls[1])
+        torch.cuda.synchronize()
+        assert torch.equal(outs[0], outs[1]), i
+        assert torch.equal(scs[0], scs[1]), i
+        assert torch.equal(bls[0], bls[1]), i
+    assert h.hisa_device_status() == 0
+    assert torch.equal(a.lens, b.lens) and torch.equal(a.kc, b.kc) and torch.equal(a.reps, b.reps)
+    assert np.array_equal(b.lens.cpu().numpy(), lens0 + steps)
+    fresh = h.hisa_pool_blocks(b.kc, cu_k, b.lens, cap)
+    assert torch.equal(fresh, b.reps)
+    # the last step against the oracle, on the host copy of the cache
+    host_k = b.kc.cpu().view(torch.int16).numpy().view(np.uint16)
+    o_idx, o_sc, o_bl, _ = oracle.hisa(dwl.queries[steps - 1], host_k, np.arange(S + 1, dtype=np.int32),
+                                       dwl.cu_k, (lens0 + steps).astype(np.int32), dwl.B, m, k)
+    assert np.array_equal(bls[1].cpu().numpy(), o_bl)
+    assert np.array_equal(outs[1].cpu().numpy(), o_idx)
+    valid = o_idx >= 0
+    assert np.array_equal(scs[1].cpu().numpy()[valid].astype(np.float64), o_sc[valid])
