@@ -243,7 +243,7 @@ static void topk_emit(cand *c, int nc, int topk, int32_t *out_idx, double *out_s
 static int causal_ok(int j, int pos) { return g_mutation == 4 ? (j < pos) : (j <= pos); }
 
 /* ------------------------------------------------------------------------- */
-/* threaded driver                                                            */
+/* threaded runner over query rows                                           */
 
 enum job_kind { JOB_BLOCKS, JOB_BLOCK_SCORES, JOB_TOKENS, JOB_DSA };
 
