@@ -310,14 +310,14 @@ def test_config_prefill_32k_needles_sampled():
 
 def test_config_prefill_128k_sampled():
     w = config_workload(4)
-    _gauss_hisa_check(w, 96, 7)
-    _gauss_dsa_check(w, 24, 8)
+    _gauss_hisa_check(w, 256, 7)
+    _gauss_dsa_check(w, 256, 8)
 
 
 def test_config_varlen_sampled():
     w = config_workload(5)
-    _gauss_hisa_check(w, 128, 9)
-    _gauss_dsa_check(w, 24, 10)
+    _gauss_hisa_check(w, 256, 9)
+    _gauss_dsa_check(w, 256, 10)
 
 
 # ---------------------------------------------------------------------------
